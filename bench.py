@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the ZHA hot path on B200 (one JSON line on rank 0).
+
+Metric: microseconds per decoded token per layer (batch 1, every query head),
+plus HBM GB/s on the bytes the step must touch, next to a dense flash-decode
+kernel over the same cache.
+
+One step = what one decoded token costs one layer: zha_append of the token's
+k, v (tree maintenance: the leaf and every ancestor are recomputed) followed by
+zha_decode of its query (routing over every level, then exact attention over
+the kept leaves plus the sink).  The full tree build is timed separately and
+reported as build tokens/s.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launch stream; a 256 MiB buffer is written between steps (L2 flush)
+outside the events.  The routing of every step is replayed first in an
+untimed, traced pass (the decode is deterministic) to count the algorithmic
+bytes; the cache is then rebuilt and the timed pass runs without tracing.
+
+--impl reference times the fp64 CPU oracle on the same workload instead.
+Multi-GPU: replicas only (each rank runs the whole workload on its GPU).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "µs per decoded token per layer and HBM GB/s (ZHA vs dense) at 256K–10M ctx, 1 B200"
+UNIT = "us/token"
+DEFAULT_WORKLOAD = "wide_256k"
+FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, local):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{local}.csv")
+        self.index = str(local)
+        try:
+            uuid = str(torch.cuda.get_device_properties(local).uuid)
+            self.index = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            if vis:
+                self.index = vis.split(",")[local]
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def step_bytes(w, trace_ids, trace_cnt, n_tokens):
+    """Algorithmic bytes of one decode from its per-level kept sets.
+
+    Routing reads each node of the union frontier of a KV head once (g and b:
+    R*(d+1)*4 bytes), whatever the number of its query heads that need it;
+    attention reads the K and V rows of the union of the heads' token sets
+    once; plus the queries and outputs."""
+    c, D, d, R, G = w.c, w.D, w.d, w.R, w.group
+    e = 4 if w.kv_dtype == "f32" else 2
+    node = R * (d + 1) * 4
+    route = 0
+    attn = 0
+    slots_total = 0
+    for kh in range(w.h_kv):
+        heads = range(kh * G, (kh + 1) * G)
+        for level in range(D, 0, -1):
+            if level == D:
+                nodes = -(-n_tokens // c ** D)
+            else:
+                kept = set()
+                for h in heads:
+                    kept.update(trace_ids[level, h, :trace_cnt[level, h]].tolist())
+                nb = -(-n_tokens // c ** level)
+                nodes = sum(min(c, nb - k * c) for k in kept)
+            route += nodes * node
+            slots_total += nodes
+        leaves = set()
+        sink = False
+        for h in heads:
+            lv = trace_ids[0, h, :trace_cnt[0, h]]
+            leaves.update(lv.tolist())
+            if len(lv) == 0 or lv[0] != 0:
+                sink = True
+        toks = sum(min(c, n_tokens - lf * c) for lf in leaves) + (1 if sink and 0 not in leaves else 0)
+        attn += toks * 2 * d * e
+    qo = w.h_q * d * 8
+    return route, attn + qo, slots_total
+
+
+def append_bytes(w, n_after):
+    """Bytes one zha_append must move: the new k, v rows, the leaf's keys,
+    each ancestor's children (read) and the D recomputed nodes (written)."""
+    c, D, d, R = w.c, w.D, w.d, w.R
+    e = 4 if w.kv_dtype == "f32" else 2
+    node_w = R * (d + 2) * 4
+    node_r = R * (d + 1) * 4
+    pos = n_after - 1
+    leaf = pos // c
+    b = 2 * d * e + (n_after - leaf * c) * d * e + D * node_w
+    n = leaf
+    for level in range(2, D + 1):
+        n //= c
+        nbelow = -(-n_after // c ** (level - 1))
+        b += min(c, nbelow - n * c) * node_r
+    return b * w.h_kv
+
+
+def run_zha(args, rank, world, local):
+    import tree_indexed_sparse_b200 as zha
+
+    base = workloads.WORKLOADS[args.workload]
+    W, K = args.warmup, args.steps
+    w = dataclasses.replace(base, appends_per_step=0, appends_after=W + K)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    t0 = time.time()
+    inp = workloads.generate(w, "cuda")
+    torch.cuda.synchronize()
+    gen_s = time.time() - t0
+    dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
+    cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, device=dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    n1cap = -(-w.capacity // w.c)
+
+    # build (timed, after one warm-up build)
+    cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
+    torch.cuda.synchronize()
+    flush.zero_()
+    eb0, eb1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    eb0.record(stream)
+    cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
+    eb1.record(stream)
+    torch.cuda.synchronize()
+    build_ms = eb0.elapsed_time(eb1)
+
+    out = torch.empty(w.h_q, w.d, dtype=torch.float32, device=dev)
+    leaf_idx = torch.empty(w.h_q, n1cap, dtype=torch.int32, device=dev)
+    n_leaf = torch.empty(w.h_q, dtype=torch.int32, device=dev)
+    visited = torch.empty(w.h_q, dtype=torch.int64, device=dev)
+    qs = inp.Q
+
+    def decode(q, trace=None):
+        if trace is None:
+            zha.zha_decode(cache.ctx, q, w.p, out, leaf_idx, n1cap, n_leaf, visited, None, None, 0,
+                           stream.cuda_stream)
+        else:
+            zha.zha_decode(cache.ctx, q, w.p, out, leaf_idx, n1cap, n_leaf, visited, trace[0], trace[1],
+                           n1cap, stream.cuda_stream)
+
+    # pass A: traced, untimed -- algorithmic bytes of every step
+    tr_ids = torch.empty(w.D, w.h_q, n1cap, dtype=torch.int32, device=dev)
+    tr_cnt = torch.empty(w.D, w.h_q, dtype=torch.int32, device=dev)
+    per_step = []
+    leaves_per_head, vis_per_head = [], []
+    for i in range(W + K):
+        cache.append(inp.K_app[i], inp.V_app[i])
+        decode(qs[i % w.steps], (tr_ids, tr_cnt))
+        if i >= W:
+            ids = tr_ids.cpu().numpy()
+            cnt = tr_cnt.cpu().numpy()
+            n_now = w.n_tokens + i + 1
+            rb, ab, slots = step_bytes(w, ids, cnt, n_now)
+            per_step.append((rb, ab, append_bytes(w, n_now), slots, n_now))
+            leaves_per_head.append(n_leaf.float().mean().item())
+            vis_per_head.append(visited.float().mean().item())
+    ref_out = out.clone()
+    assert cache.status() == 0, "device status not OK after the traced pass"
+
+    # pass B: timed
+    cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(w.D + 2)]
+    zha.zha_set_phase_events(cache.ctx, ev)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_step, t_app, t_route, t_attn, t_levels = [], [], [], [], []
+    clocks = Clocks(local)
+    for i in range(W):
+        flush.zero_()
+        cache.append(inp.K_app[i], inp.V_app[i])
+        decode(qs[i % w.steps])
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    wall0 = time.time()
+    for i in range(W, W + K):
+        flush.zero_()
+        ea.record(stream)
+        cache.append(inp.K_app[i], inp.V_app[i])
+        eb.record(stream)
+        decode(qs[i % w.steps])
+        torch.cuda.synchronize()
+        a = ea.elapsed_time(eb)
+        r = ev[0].elapsed_time(ev[w.D])
+        at = ev[w.D].elapsed_time(ev[w.D + 1])
+        t_app.append(a)
+        t_route.append(r)
+        t_attn.append(at)
+        t_levels.append([ev[j].elapsed_time(ev[j + 1]) for j in range(w.D)])
+        t_step.append(ea.elapsed_time(ev[w.D + 1]))
+    torch.cuda.synchronize()
+    wall = time.time() - wall0
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    zha.zha_set_phase_events(cache.ctx, None)
+    same = torch.equal(out, ref_out)
+    total_ms = sum(t_step)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_step = total_ms / K
+    us_token = ms_step * 1000.0 / world
+
+    route_b = [s[0] for s in per_step]
+    attn_b = [s[1] for s in per_step]
+    app_b = [s[2] for s in per_step]
+    step_b = [r + a + p for r, a, p in zip(route_b, attn_b, app_b)]
+    peak, peak_kind = peaks()
+    gbs = sum(step_b) / (sum(t_step) * 1e-3) / 1e9
+    phases = {
+        "append": {"us": 1e3 * statistics.mean(t_app), "bytes": statistics.mean(app_b),
+                   "gbs": sum(app_b) / (sum(t_app) * 1e-3) / 1e9},
+        "route": {"us": 1e3 * statistics.mean(t_route), "bytes": statistics.mean(route_b),
+                  "gbs": sum(route_b) / (sum(t_route) * 1e-3) / 1e9,
+                  "us_per_level_top_down": [1e3 * statistics.mean(x) for x in zip(*t_levels)]},
+        "attention": {"us": 1e3 * statistics.mean(t_attn), "bytes": statistics.mean(attn_b),
+                      "gbs": sum(attn_b) / (sum(t_attn) * 1e-3) / 1e9},
+    }
+    dom = max(("route", "attention", "append"), key=lambda k: phases[k]["us"])
+    kernel_name = {"route": "k_route_level", "attention": "k_attend", "append": "k_append"}[dom]
+    launches_per_step = {"route": w.D, "attention": 1, "append": 1}[dom]
+    achieved = phases[dom]["gbs"]
+    roofline = {"bound": "hbm", "kernel": kernel_name, "launches_per_step": launches_per_step,
+                "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "peak_kind": f"{peak_kind} copy bandwidth (burst)", "traffic": None,
+                "algorithmic_bytes_per_step": phases[dom]["bytes"]}
+
+    # dense flash-decode over the same cache (n_tokens + W + K rows now)
+    n_dense = cache.n_tokens
+    e = 4 if w.kv_dtype == "f32" else 2
+    dense_bytes = n_dense * w.h_kv * 2 * w.d * e + w.h_q * w.d * 8
+    t_dense = []
+    dout = torch.empty_like(out)
+    for i in range(W + K):
+        flush.zero_()
+        ea.record(stream)
+        zha.zha_dense_decode(cache.ctx, qs[i % w.steps], dout, stream.cuda_stream)
+        eb.record(stream)
+        torch.cuda.synchronize()
+        if i >= W:
+            t_dense.append(ea.elapsed_time(eb))
+    dense_us = 1e3 * statistics.mean(t_dense)
+    dense = {"us_per_token": dense_us, "hbm_gbs": dense_bytes / (dense_us * 1e-6) / 1e9,
+             "frac": dense_bytes / (dense_us * 1e-6) / 1e9 / peak, "bytes": dense_bytes, "n_tokens": n_dense}
+
+    # e2e: host buffers through the API, copies inside the timed region
+    cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
+    hq = qs.cpu().pin_memory()
+    hk = inp.K_app.cpu().pin_memory()
+    hv = inp.V_app.cpu().pin_memory()
+    hout = torch.empty(w.h_q, w.d, dtype=torch.float32).pin_memory()
+    dq = torch.empty(w.h_q, w.d, dtype=torch.float32, device=dev)
+    dk = torch.empty(w.h_kv, w.d, dtype=inp.K.dtype, device=dev)
+    dv = torch.empty_like(dk)
+    t_e2e = []
+    for i in range(W + K):
+        flush.zero_()
+        ea.record(stream)
+        dq.copy_(hq[i % w.steps], non_blocking=True)
+        dk.copy_(hk[i], non_blocking=True)
+        dv.copy_(hv[i], non_blocking=True)
+        cache.append(dk, dv)
+        decode(dq)
+        hout.copy_(out, non_blocking=True)
+        eb.record(stream)
+        torch.cuda.synchronize()
+        if i >= W:
+            t_e2e.append(ea.elapsed_time(eb))
+    h2d = dq.numel() * 4 + 2 * dk.numel() * dk.element_size()
+    d2h = hout.numel() * 4
+    e2e_us = 1e3 * sum(t_e2e) / K / world
+    if world > 1:
+        tt = torch.tensor([e2e_us], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        e2e_us = float(tt.item())
+
+    res = {
+        "metric": METRIC, "value": us_token, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "n_tokens": w.n_tokens, "h_kv": w.h_kv, "h_q": w.h_q, "d": w.d,
+                   "c": w.c, "D": w.D, "R": w.R, "p": w.p, "kv_dtype": w.kv_dtype, "keys": w.keys,
+                   "step": "zha_append of one token + zha_decode of one token, all query heads, batch 1, one layer",
+                   "l2": "256 MiB written between steps, outside the per-step events",
+                   "parallelism": f"replicas x{world}"},
+        "hbm_gbs": gbs, "hbm_frac": gbs / peak,
+        "step_us": {"mean": 1e3 * statistics.mean(t_step), "median": 1e3 * statistics.median(t_step),
+                    "p10": 1e3 * float(np.percentile(t_step, 10)), "p90": 1e3 * float(np.percentile(t_step, 90))},
+        "phases": phases,
+        "roofline": roofline,
+        "dense": dense, "speedup_vs_dense": dense_us / (1e3 * statistics.mean(t_step)),
+        "build": {"ms": build_ms, "tokens_per_s": w.n_tokens / (build_ms * 1e-3)},
+        "routing": {"kept_leaves_per_head": statistics.mean(leaves_per_head),
+                    "nodes_visited_per_head": statistics.mean(vis_per_head),
+                    "keys_touched_frac": statistics.mean(leaves_per_head) * w.c / w.n_tokens,
+                    "union_slots_per_step": statistics.mean(s[3] for s in per_step),
+                    "timed_pass_reproduces_traced": bool(same)},
+        "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk,
+        "gpu_launches": K * (w.D + 2),
+        "gen_s": gen_s, "wall_timed_s": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+    return res
+
+
+def cpu_baseline(w, inp, budget_s, steps_cap=None):
+    """The fp64 oracle on the host cores: build, then as many steps (append
+    + decode of every query head) as fit in the time budget."""
+    import oracle
+
+    cores = min(16, os.cpu_count() or 1)
+    os.environ.setdefault("OMP_NUM_THREADS", str(cores))
+    K = inp.K.cpu()
+    V = inp.V.cpu()
+    ref = inp.ref.cpu()
+    t0 = time.time()
+    ht = oracle.build_heads(K, w.n_tokens, ref, w.c, w.D, capacity=w.capacity)
+    build_s = time.time() - t0
+    Q = inp.Q.cpu()
+    Ka = inp.K_app.cpu()
+    Va = inp.V_app.cpu()
+    done = 0
+    t1 = time.time()
+    n = w.n_tokens
+    while True:
+        K[:, n] = Ka[done]
+        V[:, n] = Va[done]
+        for kh in range(w.h_kv):
+            tr = ht.head(kh)
+            tr.n_tokens = n
+            oracle.append_update(tr, K[kh], ref[kh])
+        n += 1
+        ht.n_tokens = n
+        oracle.decode_heads(K, V, ht, ref, Q[done % w.steps], w.p)
+        done += 1
+        el = time.time() - t1
+        if el > budget_s or done >= (steps_cap or Ka.shape[0]):
+            break
+    us = el / done * 1e6
+    return {"value": us, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{w.name}: full fp64 build ({build_s:.1f} s, {w.n_tokens / build_s:.0f} tokens/s) then "
+                      f"{done} steps of append + decode of all {w.h_q} query heads (OpenMP over heads)",
+            "build_tokens_per_s": w.n_tokens / build_s}
+
+
+def run_reference(args, rank, world):
+    """The fp64 oracle as the reference arm, on rank 0 only."""
+    if rank != 0:
+        return None
+    base = workloads.WORKLOADS[args.workload]
+    W, K = args.warmup, args.steps
+    w = dataclasses.replace(base, appends_per_step=0, appends_after=W + K)
+    inp = workloads.generate(w, "cuda" if torch.cuda.is_available() else "cpu")
+    cb = cpu_baseline(w, inp, budget_s=args.cpu_seconds * 4, steps_cap=W + K)
+    return {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": cb["value"] / 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "n_tokens": w.n_tokens, "h_kv": w.h_kv, "h_q": w.h_q, "d": w.d,
+                       "c": w.c, "D": w.D, "R": w.R, "p": w.p, "kv_dtype": w.kv_dtype},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["zha", "reference"], default="zha")
+    ap.add_argument("--workload", choices=workloads.ORDER, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+    else:
+        res = run_zha(args, rank, world, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -74,6 +74,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.orc_build_heads.argtypes = [_P, _I32, _I64, _I64, _I32, _I32, _P, _I32, _I32, _I32, _P,
                                     _I64, _P, _I64, _P, _P]
     lib.orc_build_heads.restype = None
+    lib.orc_estimate_many.argtypes = [_P, _P, _I64, _P, _I64, _I32, _I32, _P, _P, _P]
+    lib.orc_estimate_many.restype = None
+    lib.orc_node_summary.argtypes = [_P, _I32, _I64, _I32, _P, _I32, _I32, _I32, _I64, _P, _P, _P]
+    lib.orc_node_summary.restype = None
     return lib
 
 
@@ -171,6 +175,34 @@ def estimate(m, g, ref, q, lib=None) -> float:
     return float(lib.orc_estimate(_ptr(m), _ptr(g), R, d, _ptr(ref), _ptr(q)))
 
 
+def estimate_many(m_all, g_all, level_row0: int, ids, ref, q, lib=None) -> np.ndarray:
+    """Estimates of the listed node ids of one level (a tree's m, g store;
+    the level starts at row level_row0)."""
+    lib = lib or load()
+    ref = f64(ref)
+    q = f64(q)
+    ids = np.ascontiguousarray(ids, dtype=np.int64)
+    R, d = ref.shape
+    out = np.zeros(ids.shape[0])
+    lib.orc_estimate_many(_ptr(m_all), _ptr(g_all), int(level_row0), _ptr(ids), ids.shape[0], R, d,
+                          _ptr(ref), _ptr(q), _ptr(out))
+    return out
+
+
+def node_summary(K, n_tokens: int, ref, c: int, level: int, n: int, lib=None):
+    """(m, g, b) of node n of `level`, computed from its subtree's raw keys."""
+    lib = lib or load()
+    Ka, dt = kv_array(K)
+    ref = f64(ref)
+    R, d = ref.shape
+    m = np.zeros(R)
+    g = np.zeros((R, d))
+    b = np.zeros(R)
+    lib.orc_node_summary(_ptr(Ka), dt, int(n_tokens), d, _ptr(ref), R, c, int(level), int(n), _ptr(m), _ptr(g),
+                         _ptr(b))
+    return m, g, b
+
+
 @dataclass
 class Tree:
     """Summary store of one head.  Node (level l, id n) is row
@@ -183,6 +215,10 @@ class Tree:
     n_tokens: int
     c: int
     D: int
+
+    def estimates(self, l: int, ids, ref, q, lib=None) -> np.ndarray:
+        """Estimates for query q of the listed node ids of level l."""
+        return estimate_many(self.m, self.g, int(self.level_off[l - 1]), ids, ref, q, lib=lib)
 
     def level(self, l: int):
         """(m, g, b) views of the nodes currently present at level l."""

@@ -500,3 +500,51 @@ void orc_build_heads(const void *K, int dtype, int64_t kv_stride, int64_t N, int
                   ref + (size_t)kh * R * d, R, c, D, m + kh * m_stride, g + kh * g_stride,
                   b + kh * m_stride, level_off);
 }
+
+/* ---- batch helpers for the checks (loops over the definitions above) ---- */
+
+/* est[i] = orc_estimate of node ids[i] of one level (rows level_row0 + id). */
+void orc_estimate_many(const double *m, const double *g, int64_t level_row0, const int64_t *ids,
+                       int64_t n, int R, int d, const double *ref, const double *q, double *est)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t row = level_row0 + ids[i];
+        est[i] = orc_estimate(m + row * R, g + row * R * d, R, d, ref, q);
+    }
+}
+
+/*
+ * Summary of one node (level, n) computed from the raw keys of its subtree
+ * alone: a leaf by orc_leaf_summary, a parent by orc_parent_summary over its
+ * children, each child computed the same way (recursion).  Used to check
+ * sampled nodes of trees too large to build on the host.
+ */
+void orc_node_summary(const void *K, int dtype, int64_t N, int d, const double *ref, int R, int c,
+                      int level, int64_t n, double *m, double *g, double *b)
+{
+    if (level == 1) {
+        const int64_t t0 = n * c;
+        int64_t t1 = t0 + c;
+        if (t1 > N)
+            t1 = N;
+        orc_leaf_summary(K, dtype, t0, t1, d, ref, R, m, g, b);
+        return;
+    }
+    const int64_t nbelow = orc_level_nodes(N, c, level - 1);
+    const int64_t c0 = n * c;
+    int64_t c1 = c0 + c;
+    if (c1 > nbelow)
+        c1 = nbelow;
+    const int nch = (int)(c1 - c0);
+    double *cm = (double *)malloc((size_t)nch * R * sizeof(double));
+    double *cg = (double *)malloc((size_t)nch * R * d * sizeof(double));
+    double *cb = (double *)malloc((size_t)nch * R * sizeof(double));
+    for (int ch = 0; ch < nch; ++ch)
+        orc_node_summary(K, dtype, N, d, ref, R, c, level - 1, c0 + ch, cm + (size_t)ch * R,
+                         cg + (size_t)ch * R * d, cb + (size_t)ch * R);
+    orc_parent_summary(cm, cg, nch, d, ref, R, m, g, b);
+    free(cm);
+    free(cg);
+    free(cb);
+}

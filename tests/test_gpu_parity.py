@@ -1,0 +1,220 @@
+"""CUDA path vs the fp64 oracle, through the C ABI (needs a B200).
+
+Cases are the five workloads' structures at sizes the oracle finishes in
+seconds (several top nodes, ragged tails); the full-size workloads are in
+test_gpu_fullsize.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import OUT_TOL, check_build, check_decode, oracle_trees
+
+import tree_indexed_sparse_b200 as zha
+
+pytestmark = pytest.mark.gpu
+
+W = workloads.WORKLOADS
+CASES = {
+    "tiny_f32": W["tiny_f32_16k"].scaled(16384, steps=16),
+    "wide": W["wide_256k"].scaled(16384 + 100, steps=3),
+    "deep": W["deep_256k"].scaled(16384 + 37, steps=3),
+    "light": W["light_1m"].scaled(300000 + 5, steps=3),
+}
+
+
+class Case:
+    def __init__(self, w):
+        self.w = w
+        self.inp = workloads.generate(w, "cpu")
+        self.K = self.inp.K.clone()          # host copy that also receives appended rows
+        self.V = self.inp.V.clone()
+        self.dK = self.inp.K.cuda()
+        self.dV = self.inp.V.cuda()
+        self.dref = self.inp.ref.cuda()
+        dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
+        self.cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity)
+        self.cache.build(self.dK, self.dV, w.n_tokens, self.dref)
+        self.trees = oracle_trees(self.K, self.inp.ref, w.n_tokens, w.c, w.D, capacity=w.capacity)
+        self.n = w.n_tokens
+
+    def append(self, i):
+        w = self.w
+        k = self.inp.K_app[i].cuda()
+        v = self.inp.V_app[i].cuda()
+        self.cache.append(k, v)
+        self.K[:, self.n] = self.inp.K_app[i]
+        self.V[:, self.n] = self.inp.V_app[i]
+        for kh in range(w.h_kv):
+            oracle.append_update(self.trees[kh], self.K[kh], self.inp.ref[kh])
+        self.n += 1
+
+
+_cases = {}
+
+
+def get_case(name):
+    if name not in _cases:
+        _cases[name] = Case(CASES[name])
+    return _cases[name]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_build_parity(name):
+    c = get_case(name)
+    worst = check_build(c.cache, c.trees)
+    print(f"{name}: worst relative error m={worst[0]:.2e} g={worst[1]:.2e} b={worst[2]:.2e}")
+    assert c.cache.status() == 0
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_decode_parity(name):
+    c = get_case(name)
+    w = c.w
+    trace_cap = oracle.level_nodes(w.capacity, w.c, 1)
+    amb = 0
+    app = 0
+    for s in range(w.steps):
+        for _ in range(w.appends_per_step):
+            c.append(app)
+            app += 1
+        q = c.inp.Q[s]
+        res = c.cache.decode(q.cuda(), w.p, trace_cap=trace_cap)
+        torch.cuda.synchronize()
+        assert c.cache.status() == 0
+        amb += check_decode(res, c.trees, c.K, c.V, c.inp.ref, q.double().numpy(), w.p, c.n, w.c, w.D, w.group,
+                            w.kv_dtype)
+    print(f"{name}: {w.steps} steps, ambiguous nodes {amb}")
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_dense_parity(name):
+    c = get_case(name)
+    w = c.w
+    q = c.inp.Q[0]
+    out = c.cache.dense(q.cuda()).double().cpu().numpy()
+    for h in range(w.h_q):
+        kh = h // w.group
+        ref = oracle.attend(c.K[kh], c.V[kh], np.arange(c.n), q[h].double().numpy())
+        assert np.max(np.abs(out[h] - ref)) <= OUT_TOL[w.kv_dtype], h
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "wide", "light"])
+def test_p1_is_dense(name):
+    """p = 1 keeps every leaf: the routed output is dense attention."""
+    c = get_case(name)
+    q = c.inp.Q[1].cuda()
+    res = c.cache.decode(q, 1.0)
+    dense = c.cache.dense(q)
+    tol = OUT_TOL[c.w.kv_dtype]
+    assert torch.max(torch.abs(res["out"] - dense)).item() <= tol
+    nl = oracle.level_nodes(c.n, c.w.c, 1)
+    assert torch.all(res["n_leaf"] == nl)
+
+
+def test_decode_deterministic():
+    c = get_case("light")
+    q = c.inp.Q[2].cuda()
+    cap = oracle.level_nodes(c.w.capacity, c.w.c, 1)
+    r1 = c.cache.decode(q, c.w.p, trace_cap=cap)
+    r2 = c.cache.decode(q, c.w.p, trace_cap=cap)
+    for k in ("out", "n_leaf", "visited", "trace_counts"):
+        assert torch.equal(r1[k], r2[k]), k
+    for h in range(c.w.h_q):
+        n = int(r1["n_leaf"][h])
+        assert torch.equal(r1["leaf_idx"][h, :n], r2["leaf_idx"][h, :n])
+        for level in range(c.w.D):
+            m = int(r1["trace_counts"][level, h])
+            assert torch.equal(r1["trace_ids"][level, h, :m], r2["trace_ids"][level, h, :m])
+
+
+def _small_cache(N, c, D, R, h_kv, h_q, d, dtype, seed, cap=None):
+    g = torch.Generator().manual_seed(seed)
+    cap = cap or N
+    tdt = torch.float32 if dtype == zha.ZHA_F32 else torch.bfloat16
+    K = torch.zeros(h_kv, cap, d, dtype=tdt)
+    V = torch.zeros(h_kv, cap, d, dtype=tdt)
+    K[:, :N] = torch.randn(h_kv, N, d, generator=g).to(tdt)
+    V[:, :N] = torch.randn(h_kv, N, d, generator=g).to(tdt)
+    ref = torch.randn(h_kv, R, d, generator=g)
+    if dtype == zha.ZHA_BF16:
+        ref = ref.to(torch.bfloat16).float()
+    cache = zha.ZhaCache(h_kv, h_q, d, R, c, D, dtype, cap)
+    dK, dV, dref = K.cuda(), V.cuda(), ref.cuda()
+    cache.build(dK, dV, N, dref)
+    return cache, (K, V, ref), (dK, dV, dref)
+
+
+@pytest.mark.parametrize("N,c,D,R,h_kv,h_q,d,dtype", [
+    (1, 4, 3, 16, 1, 1, 64, zha.ZHA_F32),        # a single token
+    (3, 4, 2, 16, 1, 4, 64, zha.ZHA_F32),        # one partial leaf
+    (16, 4, 2, 1, 2, 8, 128, zha.ZHA_BF16),      # exactly c^D tokens
+    (17, 4, 2, 16, 2, 8, 128, zha.ZHA_BF16),     # c^D + 1: a second top node
+    (1000, 2, 9, 1, 1, 4, 128, zha.ZHA_BF16),    # deep binary tree
+    (5000, 256, 1, 16, 1, 4, 128, zha.ZHA_BF16),  # wide leaves, ragged tail
+])
+def test_edge_shapes(N, c, D, R, h_kv, h_q, d, dtype):
+    cache, (K, V, ref), _ = _small_cache(N, c, D, R, h_kv, h_q, d, dtype, seed=N + c)
+    trees = oracle_trees(K, ref, N, c, D)
+    check_build(cache, trees)
+    kv = "f32" if dtype == zha.ZHA_F32 else "bf16"
+    g = torch.Generator().manual_seed(7)
+    for p in (0.5, 0.9, 1.0):
+        q = torch.randn(h_q, d, generator=g) * 2
+        res = cache.decode(q.cuda(), p, trace_cap=oracle.level_nodes(N, c, 1))
+        check_decode(res, trees, K, V, ref, q.double().numpy(), p, N, c, D, h_q // h_kv, kv)
+    assert cache.status() == 0
+
+
+def test_append_matches_rebuild_bitexact():
+    """Appending tokens one by one stores exactly the summaries of a fresh
+    build over the longer cache (same device functions, same order)."""
+    N, a, c, D, R, h_kv, h_q, d = 4090, 13, 4, 6, 16, 2, 8, 128
+    cache, (K, V, ref), (dK, dV, dref) = _small_cache(N, c, D, R, h_kv, h_q, d, zha.ZHA_BF16, 11, cap=N + a)
+    g = torch.Generator().manual_seed(5)
+    knew = torch.randn(a, h_kv, d, generator=g).to(torch.bfloat16)
+    vnew = torch.randn(a, h_kv, d, generator=g).to(torch.bfloat16)
+    for i in range(a):
+        cache.append(knew[i].cuda(), vnew[i].cuda())
+    K[:, N:N + a] = knew.transpose(0, 1)
+    V[:, N:N + a] = vnew.transpose(0, 1)
+    fresh = zha.ZhaCache(h_kv, h_q, d, R, c, D, zha.ZHA_BF16, N + a)
+    fK, fV = K.cuda(), V.cuda()
+    fresh.build(fK, fV, N + a, dref)
+    torch.cuda.synchronize()
+    assert cache.n_tokens == N + a
+    assert torch.equal(dK, fK) and torch.equal(dV, fV)
+    for level in range(1, D + 1):
+        for x, y in zip(cache.summaries(level), fresh.summaries(level)):
+            assert torch.equal(x, y), level
+    trees = oracle_trees(K, ref, N + a, c, D)
+    check_build(cache, trees)
+
+
+def test_errors_and_capacity():
+    N, c, D, R, h_kv, h_q, d = 64, 4, 2, 16, 1, 4, 64
+    cfg = zha.zha_config(h_kv, h_q, d, R, c, D, zha.ZHA_F32, 0, N)
+    ws = torch.empty(zha.zha_workspace_bytes(cfg), dtype=torch.uint8, device="cuda")
+    ctx = zha.zha_create(cfg, ws, ws.numel())
+    q = torch.randn(h_q, d, device="cuda")
+    out = torch.empty(h_q, d, device="cuda")
+    with pytest.raises(zha.ZhaError) as e:
+        zha.zha_decode(ctx, q, 0.9, out)
+    assert e.value.code == zha.ZHA_ERR_NOT_BUILT
+    zha.zha_destroy(ctx)
+    cache, _, _ = _small_cache(N, c, D, R, h_kv, h_q, d, zha.ZHA_F32, 3)
+    k = torch.zeros(h_kv, d, device="cuda")
+    with pytest.raises(zha.ZhaError) as e:
+        cache.append(k, k)
+    assert e.value.code == zha.ZHA_ERR_CAPACITY
+    with pytest.raises(zha.ZhaError) as e:
+        cache.decode(q, 0.0)
+    assert e.value.code == zha.ZHA_ERR_BAD_ARG
+    # a leaf list shorter than the kept set: clipped, status says capacity
+    res = cache.decode(q, 1.0, leaf_cap=2)
+    torch.cuda.synchronize()
+    assert cache.status() == zha.ZHA_ERR_CAPACITY
+    assert torch.all(res["n_leaf"] == 16)
+    assert cache.status() == 0

@@ -1,0 +1,367 @@
+// zha_api.cu -- the extern "C" boundary of libzha.so (declared in include/zha.h).
+//
+// Host-side only: argument checks, the workspace layout, and the launch
+// sequence of each call.  The library allocates no device memory; every
+// buffer belongs to the caller.
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "../../include/zha.h"
+#include "zha_internal.cuh"
+
+using namespace zha;
+
+struct zha_ctx {
+    zha_config cfg;
+    Tree t;                   // pointers into the workspace; K, V, ref set by zha_build
+    bool built;
+    unsigned char *ws;
+    int64_t ws_bytes;
+    // decode scratch (inside the workspace)
+    int32_t *kept_ids[MAXD];
+    uint8_t *kept_mask[MAXD];
+    int32_t *kept_cnt;
+    float *scores;
+    int64_t score_cap;
+    float *pmax;
+    int pmax_cap;
+    uint32_t *done;
+    int64_t *vis_acc;
+    float *part;
+    int part_cap;
+    int32_t *status;
+    unsigned char *scratch_begin;
+    int64_t scratch_bytes;
+    cudaEvent_t phase_ev[MAXD + 2];
+    int n_phase_ev;
+    int n_sm;
+    int route_cta;
+    int attn_cta;
+};
+
+namespace {
+
+constexpr int PMAX_CAP = 1024;
+constexpr int PART_CAP = 1024;
+
+int64_t align256(int64_t x) { return (x + 255) / 256 * 256; }
+
+// ceil(n / c^level), saturating at 1 once c^level exceeds n.
+int64_t level_nodes(int64_t n, int c, int level) {
+    int64_t span = 1;
+    for (int l = 0; l < level; ++l) {
+        if (span > n) return n > 0 ? 1 : 0;
+        span *= c;
+    }
+    return (n + span - 1) / span;
+}
+
+int check_config(const zha_config *cfg) {
+    if (!cfg) return ZHA_ERR_BAD_ARG;
+    if (cfg->h_kv < 1 || cfg->h_kv > 64 || cfg->h_q < cfg->h_kv || cfg->h_q % cfg->h_kv) return ZHA_ERR_BAD_ARG;
+    if (cfg->d <= 0 || cfg->R <= 0 || cfg->c < 2 || cfg->D < 1 || cfg->D > MAXD) return ZHA_ERR_BAD_ARG;
+    if (cfg->kv_dtype != ZHA_F32 && cfg->kv_dtype != ZHA_BF16) return ZHA_ERR_BAD_ARG;
+    if (cfg->capacity_tokens < 1 || cfg->capacity_tokens > (int64_t)0x7fffffff) return ZHA_ERR_BAD_ARG;
+    const int G = cfg->h_q / cfg->h_kv;
+    if (!compiled_combo(cfg->kv_dtype, cfg->d, cfg->R, G)) return ZHA_ERR_UNSUPPORTED;
+    return ZHA_OK;
+}
+
+// Byte layout of the workspace.  Each region starts 256-byte aligned.
+struct Layout {
+    int64_t node_cap[MAXD];
+    int64_t g_off[MAXD], b_off[MAXD], m_off[MAXD];
+    int64_t kid_off[MAXD], kmask_off[MAXD];
+    int64_t kcnt_off, scores_off, pmax_off, done_off, vis_off, part_off, status_off;
+    int64_t scratch_off, total;
+    int64_t score_cap;
+};
+
+void make_layout(const zha_config *cfg, Layout *L) {
+    const int G = cfg->h_q / cfg->h_kv;
+    int64_t off = 0;
+    for (int l = 1; l <= cfg->D; ++l) {
+        const int64_t nc = level_nodes(cfg->capacity_tokens, cfg->c, l);
+        L->node_cap[l - 1] = nc;
+        L->g_off[l - 1] = off;
+        off = align256(off + (int64_t)cfg->h_kv * nc * cfg->R * cfg->d * 4);
+        L->b_off[l - 1] = off;
+        off = align256(off + (int64_t)cfg->h_kv * nc * cfg->R * 4);
+        L->m_off[l - 1] = off;
+        off = align256(off + (int64_t)cfg->h_kv * nc * cfg->R * 4);
+    }
+    L->scratch_off = off;
+    for (int l = 1; l <= cfg->D; ++l) {
+        L->kid_off[l - 1] = off;
+        off = align256(off + (int64_t)cfg->h_kv * L->node_cap[l - 1] * 4);
+        L->kmask_off[l - 1] = off;
+        off = align256(off + (int64_t)cfg->h_kv * L->node_cap[l - 1]);
+    }
+    // frontier slots: every top node, or the children of the kept nodes one level up
+    int64_t sc = L->node_cap[cfg->D - 1];
+    for (int l = 1; l < cfg->D; ++l) sc = std::max(sc, (int64_t)cfg->c * L->node_cap[l]);
+    L->score_cap = sc;
+    L->kcnt_off = off;
+    off = align256(off + (int64_t)MAXD * cfg->h_kv * 4);
+    L->scores_off = off;
+    off = align256(off + (int64_t)cfg->h_kv * sc * G * 4);
+    L->pmax_off = off;
+    off = align256(off + (int64_t)cfg->h_kv * PMAX_CAP * G * 4);
+    L->done_off = off;
+    off = align256(off + (int64_t)(MAXD + 2) * cfg->h_kv * 4);
+    L->vis_off = off;
+    off = align256(off + (int64_t)cfg->h_q * 8);
+    L->part_off = off;
+    off = align256(off + (int64_t)PART_CAP * cfg->h_kv * G * (cfg->d + 2) * 4);
+    L->status_off = off;
+    off = align256(off + 4);
+    L->total = off;
+}
+
+bool fault_injected(const char *what) {
+    const char *f = std::getenv("ZHA_FAULT");
+    return f && std::strcmp(f, what) == 0;
+}
+
+void fill_tree_levels(zha_ctx *ctx) {
+    Tree &t = ctx->t;
+    for (int l = 1; l <= t.D; ++l) t.n_level[l - 1] = (int32_t)level_nodes(t.n_tokens, t.c, l);
+}
+
+Decode make_decode(zha_ctx *ctx) {
+    Decode dc;
+    std::memset(&dc, 0, sizeof dc);
+    dc.t = ctx->t;
+    for (int l = 0; l < MAXD; ++l) {
+        dc.kept_ids[l] = ctx->kept_ids[l];
+        dc.kept_mask[l] = ctx->kept_mask[l];
+    }
+    dc.kept_cnt = ctx->kept_cnt;
+    dc.scores = ctx->scores;
+    dc.score_cap = ctx->score_cap;
+    dc.pmax = ctx->pmax;
+    dc.pmax_cap = ctx->pmax_cap;
+    dc.done = ctx->done;
+    dc.vis_acc = ctx->vis_acc;
+    dc.part = ctx->part;
+    dc.part_cap = ctx->part_cap;
+    dc.status = ctx->status;
+    return dc;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t zha_workspace_bytes(const zha_config *cfg) {
+    const int rc = check_config(cfg);
+    if (rc != ZHA_OK) return rc;
+    Layout L;
+    make_layout(cfg, &L);
+    return L.total;
+}
+
+int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_ctx **out) {
+    if (!out) return ZHA_ERR_BAD_ARG;
+    *out = nullptr;
+    const int rc = check_config(cfg);
+    if (rc != ZHA_OK) return rc;
+    Layout L;
+    make_layout(cfg, &L);
+    if (!d_workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(d_workspace) & 255u))
+        return ZHA_ERR_BAD_ARG;
+    zha_ctx *ctx = new (std::nothrow) zha_ctx;
+    if (!ctx) return ZHA_ERR_BAD_ARG;
+    std::memset(ctx, 0, sizeof *ctx);
+    ctx->cfg = *cfg;
+    unsigned char *ws = static_cast<unsigned char *>(d_workspace);
+    ctx->ws = ws;
+    ctx->ws_bytes = ws_bytes;
+    Tree &t = ctx->t;
+    t.h_kv = cfg->h_kv;
+    t.h_q = cfg->h_q;
+    t.G = cfg->h_q / cfg->h_kv;
+    t.d = cfg->d;
+    t.R = cfg->R;
+    t.c = cfg->c;
+    t.D = cfg->D;
+    t.kv_dtype = cfg->kv_dtype;
+    t.c_log2 = -1;
+    for (int s = 0; s < 31; ++s)
+        if ((1 << s) == cfg->c) t.c_log2 = s;
+    t.kv_cap = cfg->capacity_tokens;
+    t.scale = (float)(1.0 / std::sqrt((double)cfg->d));
+    for (int l = 1; l <= cfg->D; ++l) {
+        t.node_cap[l - 1] = L.node_cap[l - 1];
+        t.g[l - 1] = reinterpret_cast<float *>(ws + L.g_off[l - 1]);
+        t.b[l - 1] = reinterpret_cast<float *>(ws + L.b_off[l - 1]);
+        t.m[l - 1] = reinterpret_cast<float *>(ws + L.m_off[l - 1]);
+        ctx->kept_ids[l - 1] = reinterpret_cast<int32_t *>(ws + L.kid_off[l - 1]);
+        ctx->kept_mask[l - 1] = reinterpret_cast<uint8_t *>(ws + L.kmask_off[l - 1]);
+    }
+    ctx->kept_cnt = reinterpret_cast<int32_t *>(ws + L.kcnt_off);
+    ctx->scores = reinterpret_cast<float *>(ws + L.scores_off);
+    ctx->score_cap = L.score_cap;
+    ctx->pmax = reinterpret_cast<float *>(ws + L.pmax_off);
+    ctx->pmax_cap = PMAX_CAP;
+    ctx->done = reinterpret_cast<uint32_t *>(ws + L.done_off);
+    ctx->vis_acc = reinterpret_cast<int64_t *>(ws + L.vis_off);
+    ctx->part = reinterpret_cast<float *>(ws + L.part_off);
+    ctx->part_cap = PART_CAP;
+    ctx->status = reinterpret_cast<int32_t *>(ws + L.status_off);
+    ctx->scratch_begin = ws + L.scratch_off;
+    ctx->scratch_bytes = L.total - L.scratch_off;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&ctx->n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        delete ctx;
+        return ZHA_ERR_CUDA;
+    }
+    ctx->route_cta = std::max(1, ctx->n_sm / cfg->h_kv) * cfg->h_kv;
+    if (ctx->route_cta / cfg->h_kv > PMAX_CAP) ctx->route_cta = PMAX_CAP * cfg->h_kv;
+    ctx->attn_cta = std::min(PART_CAP, 2 * ctx->n_sm);
+    if (cudaMemset(ctx->scratch_begin, 0, (size_t)ctx->scratch_bytes) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess) {
+        delete ctx;
+        return ZHA_ERR_CUDA;
+    }
+    *out = ctx;
+    return ZHA_OK;
+}
+
+void zha_destroy(zha_ctx *ctx) { delete ctx; }
+
+int zha_build(zha_ctx *ctx, void *d_K, void *d_V, int64_t n_tokens, const float *d_ref_q, int32_t c, int32_t D,
+              void *stream) {
+    if (!ctx || !d_K || !d_V || !d_ref_q) return ZHA_ERR_BAD_ARG;
+    if (c != ctx->cfg.c || D != ctx->cfg.D) return ZHA_ERR_BAD_ARG;
+    if (n_tokens < 1) return ZHA_ERR_BAD_ARG;
+    if (n_tokens > ctx->cfg.capacity_tokens) return ZHA_ERR_CAPACITY;
+    if (((reinterpret_cast<uintptr_t>(d_K) | reinterpret_cast<uintptr_t>(d_V)) & 15u) ||
+        (reinterpret_cast<uintptr_t>(d_ref_q) & 15u))
+        return ZHA_ERR_BAD_ARG;
+    Tree &t = ctx->t;
+    t.K = d_K;
+    t.V = d_V;
+    t.ref = d_ref_q;
+    t.n_tokens = n_tokens;
+    fill_tree_levels(ctx);
+    if (fault_injected("cuda_launch")) return ZHA_ERR_CUDA;
+    if (launch_build(t, static_cast<cudaStream_t>(stream), ctx->n_sm) != cudaSuccess) return ZHA_ERR_CUDA;
+    ctx->built = true;
+    return ZHA_OK;
+}
+
+int zha_append(zha_ctx *ctx, const void *d_k, const void *d_v, void *stream) {
+    if (!ctx || !d_k || !d_v) return ZHA_ERR_BAD_ARG;
+    if (!ctx->built) return ZHA_ERR_NOT_BUILT;
+    if (ctx->t.n_tokens >= ctx->cfg.capacity_tokens || fault_injected("capacity")) return ZHA_ERR_CAPACITY;
+    Tree t = ctx->t;
+    t.n_tokens += 1;
+    for (int l = 1; l <= t.D; ++l) t.n_level[l - 1] = (int32_t)level_nodes(t.n_tokens, t.c, l);
+    if (launch_append(t, d_k, d_v, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZHA_ERR_CUDA;
+    ctx->t = t;
+    return ZHA_OK;
+}
+
+int zha_decode(zha_ctx *ctx, const float *d_q, float p, float *d_out, int32_t *d_leaf_idx, int32_t leaf_cap,
+               int32_t *d_n_leaf, int64_t *d_nodes_visited, int32_t *d_trace_ids, int32_t *d_trace_counts,
+               int32_t trace_cap, void *stream) {
+    if (!ctx || !d_q || !d_out) return ZHA_ERR_BAD_ARG;
+    if (!ctx->built) return ZHA_ERR_NOT_BUILT;
+    if (!(p > 0.f) || std::isnan(p)) return ZHA_ERR_BAD_ARG;
+    if ((d_leaf_idx && leaf_cap < 0) || (d_trace_ids && (!d_trace_counts || trace_cap < 0))) return ZHA_ERR_BAD_ARG;
+    if ((reinterpret_cast<uintptr_t>(d_q) | reinterpret_cast<uintptr_t>(d_out)) & 15u) return ZHA_ERR_BAD_ARG;
+    Decode dc = make_decode(ctx);
+    dc.q = d_q;
+    dc.p = p;
+    dc.out = d_out;
+    dc.leaf_idx = d_leaf_idx;
+    dc.leaf_cap = d_leaf_idx ? leaf_cap : 0;
+    dc.n_leaf = d_n_leaf;
+    dc.visited = d_nodes_visited;
+    dc.trace_ids = d_trace_ids;
+    dc.trace_cnt = d_trace_ids ? d_trace_counts : nullptr;
+    dc.trace_cap = d_trace_ids ? trace_cap : 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t smem = route_smem_bytes(ctx->t.G);
+    const bool ev = ctx->n_phase_ev > 0;
+    if (ev && cudaEventRecord(ctx->phase_ev[0], s) != cudaSuccess) return ZHA_ERR_CUDA;
+    for (int l = ctx->t.D; l >= 1; --l) {
+        if (launch_route_level(dc, l, ctx->route_cta, smem, s) != cudaSuccess) return ZHA_ERR_CUDA;
+        if (ev && cudaEventRecord(ctx->phase_ev[ctx->t.D + 1 - l], s) != cudaSuccess) return ZHA_ERR_CUDA;
+    }
+    if (launch_attend(dc, ctx->attn_cta, s) != cudaSuccess) return ZHA_ERR_CUDA;
+    if (ev && cudaEventRecord(ctx->phase_ev[ctx->t.D + 1], s) != cudaSuccess) return ZHA_ERR_CUDA;
+    return ZHA_OK;
+}
+
+int zha_dense_decode(zha_ctx *ctx, const float *d_q, float *d_out, void *stream) {
+    if (!ctx || !d_q || !d_out) return ZHA_ERR_BAD_ARG;
+    if (!ctx->built) return ZHA_ERR_NOT_BUILT;
+    if ((reinterpret_cast<uintptr_t>(d_q) | reinterpret_cast<uintptr_t>(d_out)) & 15u) return ZHA_ERR_BAD_ARG;
+    Decode dc = make_decode(ctx);
+    dc.q = d_q;
+    dc.out = d_out;
+    const int per = std::max(1, std::min(ctx->part_cap, 2 * ctx->n_sm) / ctx->cfg.h_kv);
+    if (launch_dense(dc, per * ctx->cfg.h_kv, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZHA_ERR_CUDA;
+    return ZHA_OK;
+}
+
+int zha_device_status(zha_ctx *ctx, int32_t *out_status, void *stream) {
+    if (!ctx || !out_status) return ZHA_ERR_BAD_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t host = 0;
+    if (cudaMemcpyAsync(&host, ctx->status, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemsetAsync(ctx->status, 0, sizeof host, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+        return ZHA_ERR_CUDA;
+    *out_status = host;
+    return ZHA_OK;
+}
+
+int zha_set_phase_events(zha_ctx *ctx, void *const *events, int32_t n_events) {
+    if (!ctx) return ZHA_ERR_BAD_ARG;
+    if (n_events == 0) {
+        ctx->n_phase_ev = 0;
+        return ZHA_OK;
+    }
+    if (!events || n_events != ctx->cfg.D + 2) return ZHA_ERR_BAD_ARG;
+    for (int i = 0; i < n_events; ++i) {
+        if (!events[i]) return ZHA_ERR_BAD_ARG;
+        ctx->phase_ev[i] = static_cast<cudaEvent_t>(events[i]);
+    }
+    ctx->n_phase_ev = n_events;
+    return ZHA_OK;
+}
+
+int64_t zha_n_tokens(const zha_ctx *ctx) { return ctx && ctx->built ? ctx->t.n_tokens : 0; }
+
+int zha_summary_layout(const zha_ctx *ctx, int32_t level, int64_t *g_offset, int64_t *b_offset, int64_t *m_offset,
+                       int64_t *node_cap) {
+    if (!ctx || level < 1 || level > ctx->cfg.D) return ZHA_ERR_BAD_ARG;
+    const unsigned char *ws = ctx->ws;
+    if (g_offset) *g_offset = reinterpret_cast<const unsigned char *>(ctx->t.g[level - 1]) - ws;
+    if (b_offset) *b_offset = reinterpret_cast<const unsigned char *>(ctx->t.b[level - 1]) - ws;
+    if (m_offset) *m_offset = reinterpret_cast<const unsigned char *>(ctx->t.m[level - 1]) - ws;
+    if (node_cap) *node_cap = ctx->t.node_cap[level - 1];
+    return ZHA_OK;
+}
+
+const char *zha_strerror(int code) {
+    switch (code) {
+        case ZHA_OK: return "ok";
+        case ZHA_ERR_BAD_ARG: return "invalid argument";
+        case ZHA_ERR_CAPACITY: return "capacity exceeded";
+        case ZHA_ERR_NOT_BUILT: return "tree not built";
+        case ZHA_ERR_CUDA: return "CUDA runtime error";
+        case ZHA_ERR_TIMEOUT: return "device wait timed out";
+        case ZHA_ERR_UNSUPPORTED: return "configuration not compiled";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

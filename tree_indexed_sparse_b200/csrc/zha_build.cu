@@ -1,0 +1,379 @@
+// zha_build.cu -- summary-tree build and incremental append (sm_100a).
+//
+// Leaf summary ("ZHA 用树形稀疏注意力改造现有大模型", section
+// "稀疏注意力为什么还会被索引拖慢": chunk summaries from reference queries, a
+// tangent-plane estimate of the chunk's log attention mass, max over planes):
+//   s_ij = r_j.k_i / sqrt(d),  m_j = logsumexp_i s_ij,
+//   g_j  = sum_i exp(s_ij - m_j) k_i,  b_j = m_j - r_j.g_j / sqrt(d).
+// Parent summary ("Zyphra 分层注意力（ZHA）…", section
+// "机制拆解：树形索引如何高效筛选长上下文": summaries grouped and compressed
+// recursively):
+//   e_ch,j = max_j' (b_ch,j' + r_j.g_ch,j' / sqrt(d))   (child estimate at r_j)
+//   m_j = logsumexp_ch e_ch,j,  g_j = sum_ch exp(e_ch,j - m_j) g_ch,j,
+//   b_j = m_j - r_j.g_j / sqrt(d).
+// Append (tree maintenance, rit.work article, section "Замеры подтверждают
+// качество, а предельный выигрыш пока рассчитан"): the new row's leaf and its
+// ancestors are recomputed by the same device functions as the build, so an
+// appended tree is bit-identical to a tree built over the longer cache.
+//
+// Work layout: one warp per leaf tile / per parent node.  Lane l owns the
+// d-slice [l*VEC, (l+1)*VEC) of every key, reference query and g row; dot
+// products are per-lane fmaf chains followed by a 32-lane reduce-scatter.
+// The kernels are bound by HBM for R = 1 and by fp32 FMA for R = 16.
+#include <algorithm>
+
+#include "zha_device.cuh"
+#include "zha_internal.cuh"
+
+namespace zha {
+
+template <int HD, int R>
+__device__ __forceinline__ void load_ref(const float *ref_h, float (&rj)[R][HD / 32], int lane) {
+#pragma unroll
+    for (int j = 0; j < R; ++j) Vec<float, HD / 32>::load(ref_h + j * HD + lane * (HD / 32), rj[j]);
+}
+
+// Tokens per leaf tile processed by one warp: a whole number of leaves and at
+// least one reduce-scatter batch (32 / R tokens).
+__host__ __device__ inline int leaf_tile_tokens(int c, int R) {
+    const int tpr = 32 / R;
+    return ((tpr + c - 1) / c) * c;
+}
+
+template <typename KT, int HD, int R>
+struct LeafOps {
+    static constexpr int VEC = HD / 32;
+    static constexpr int TPR = 32 / R;
+
+    // Summaries of the leaves covering tokens [tok0, tok0 + ntok) of one head
+    // (tok0 a multiple of c).  sh: warp-private shared scratch of
+    // ntok*R + (ntok/c + 1)*R floats.
+    static __device__ void tile(const KT *__restrict__ Kh, int64_t tok0, int ntok, int c,
+                                const float (&rj)[R][VEC], float scale, float *__restrict__ gL,
+                                float *__restrict__ bL, float *__restrict__ mL, float *sh, int lane) {
+        float *s_sh = sh;
+        const int nleaf = (ntok + c - 1) / c;
+        float *m_sh = sh + ntok * R;
+        const int64_t leaf0 = tok0 / c;
+        // pass 1: scaled scores of every (token, plane)
+        for (int t0 = 0; t0 < ntok; t0 += TPR) {
+            float v[32];
+#pragma unroll
+            for (int t = 0; t < TPR; ++t) {
+                const int i = t0 + t;
+                float k[VEC];
+                if (i < ntok) {
+                    Vec<KT, VEC>::load(Kh + (tok0 + i) * HD + lane * VEC, k);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) k[e] = 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < R; ++j) v[t * R + j] = lane_dot<VEC>(rj[j], k);
+            }
+            reduce_scatter<32>(v, lane);
+            const int i = t0 + lane / R;
+            if (i < ntok) s_sh[i * R + (lane % R)] = v[0] * scale;
+        }
+        __syncwarp();
+        // log mass per (leaf, plane) in token order; weights in place
+        for (int pair = lane; pair < nleaf * R; pair += 32) {
+            const int lf = pair / R, j = pair % R;
+            const int i0 = lf * c, i1 = min(i0 + c, ntok);
+            float mx = -INFINITY;
+            for (int i = i0; i < i1; ++i) mx = fmaxf(mx, s_sh[i * R + j]);
+            float sum = 0.f;
+            for (int i = i0; i < i1; ++i) sum += expf(s_sh[i * R + j] - mx);
+            const float m = mx + logf(sum);
+            for (int i = i0; i < i1; ++i) s_sh[i * R + j] = expf(s_sh[i * R + j] - m);
+            m_sh[pair] = m;
+            mL[(leaf0 + lf) * R + j] = m;
+        }
+        __syncwarp();
+        // g_j = sum_i w_ij k_i (token order), then the plane offsets
+        for (int lf = 0; lf < nleaf; ++lf) {
+            const int i0 = lf * c, i1 = min(i0 + c, ntok);
+            float acc[R][VEC];
+#pragma unroll
+            for (int j = 0; j < R; ++j)
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[j][e] = 0.f;
+            for (int i = i0; i < i1; ++i) {
+                float k[VEC];
+                Vec<KT, VEC>::load(Kh + (tok0 + i) * HD + lane * VEC, k);
+#pragma unroll
+                for (int j = 0; j < R; ++j) {
+                    const float w = s_sh[i * R + j];
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) acc[j][e] = fmaf(w, k[e], acc[j][e]);
+                }
+            }
+            const int64_t node = leaf0 + lf;
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+                float *dst = gL + (node * R + j) * HD + lane * VEC;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) dst[e] = acc[j][e];
+                const float dot = warp_sum(lane_dot<VEC>(rj[j], acc[j]));
+                if (lane == (j & 31)) bL[node * R + j] = m_sh[lf * R + j] - scale * dot;
+            }
+        }
+        __syncwarp();
+    }
+};
+
+template <int HD, int R>
+struct ParentOps {
+    static constexpr int VEC = HD / 32;
+
+    // Summary of level-l node n from its nch children (rows ch0 .. ch0+nch-1
+    // of level l-1; pointers for this head).  sh: warp-private shared scratch
+    // of nch*R + R floats.
+    static __device__ void node(const float *__restrict__ gC, const float *__restrict__ bC, int64_t ch0,
+                                int nch, const float (&rj)[R][VEC], float scale, float *__restrict__ gP,
+                                float *__restrict__ bP, float *__restrict__ mP, int64_t n, float *sh,
+                                int lane) {
+        float *e_sh = sh;
+        float *m_sh = sh + nch * R;
+        // child estimates at every reference query
+        if constexpr (R == 1) {
+            for (int c0 = 0; c0 < nch; c0 += 32) {
+                float v[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const int ch = c0 + t;
+                    if (ch < nch) {
+                        float gs[VEC];
+                        Vec<float, VEC>::load(gC + (ch0 + ch) * HD + lane * VEC, gs);
+                        v[t] = lane_dot<VEC>(rj[0], gs);
+                    } else {
+                        v[t] = 0.f;
+                    }
+                }
+                reduce_scatter<32>(v, lane);
+                const int ch = c0 + lane;
+                if (ch < nch) e_sh[ch] = bC[ch0 + ch] + scale * v[0];
+            }
+        } else {
+            constexpr int JP = 32 / R;
+            for (int ch = 0; ch < nch; ++ch) {
+                float emax = -INFINITY;
+                for (int jp0 = 0; jp0 < R; jp0 += JP) {
+                    float v[32];
+#pragma unroll
+                    for (int t = 0; t < JP; ++t) {
+                        float gs[VEC];
+                        Vec<float, VEC>::load(gC + ((ch0 + ch) * R + jp0 + t) * HD + lane * VEC, gs);
+#pragma unroll
+                        for (int j = 0; j < R; ++j) v[t * R + j] = lane_dot<VEC>(rj[j], gs);
+                    }
+                    reduce_scatter<32>(v, lane);
+                    const float val = bC[(ch0 + ch) * R + jp0 + lane / R] + scale * v[0];
+                    emax = fmaxf(emax, val);
+                }
+#pragma unroll
+                for (int off = R; off < 32; off <<= 1) emax = fmaxf(emax, __shfl_xor_sync(FULL, emax, off));
+                if (lane < R) e_sh[ch * R + lane] = emax;
+            }
+        }
+        __syncwarp();
+        if (lane < R) {
+            const int j = lane;
+            float mx = -INFINITY;
+            for (int ch = 0; ch < nch; ++ch) mx = fmaxf(mx, e_sh[ch * R + j]);
+            float sum = 0.f;
+            for (int ch = 0; ch < nch; ++ch) sum += expf(e_sh[ch * R + j] - mx);
+            const float m = mx + logf(sum);
+            for (int ch = 0; ch < nch; ++ch) e_sh[ch * R + j] = expf(e_sh[ch * R + j] - m);
+            m_sh[j] = m;
+            mP[n * R + j] = m;
+        }
+        __syncwarp();
+        float acc[R][VEC];
+#pragma unroll
+        for (int j = 0; j < R; ++j)
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[j][e] = 0.f;
+        for (int ch = 0; ch < nch; ++ch) {
+#pragma unroll
+            for (int j = 0; j < R; ++j) {
+                float gs[VEC];
+                Vec<float, VEC>::load(gC + ((ch0 + ch) * R + j) * HD + lane * VEC, gs);
+                const float w = e_sh[ch * R + j];
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[j][e] = fmaf(w, gs[e], acc[j][e]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < R; ++j) {
+            float *dst = gP + (n * R + j) * HD + lane * VEC;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) dst[e] = acc[j][e];
+            const float dot = warp_sum(lane_dot<VEC>(rj[j], acc[j]));
+            if (lane == (j & 31)) bP[n * R + j] = m_sh[j] - scale * dot;
+        }
+        __syncwarp();
+    }
+};
+
+// ---- kernels ---------------------------------------------------------------
+
+template <typename KT, int HD, int R>
+__global__ void __launch_bounds__(BUILD_THREADS) k_build_leaves(Tree t) {
+    extern __shared__ __align__(16) float bsm[];
+    constexpr int VEC = HD / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int tt = leaf_tile_tokens(t.c, R);
+    float *sh = bsm + warp * (tt * R + (tt / t.c + 1) * R);
+    const int64_t tiles = (t.n_tokens + tt - 1) / tt;
+    const int64_t total = tiles * t.h_kv;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    float rj[R][VEC];
+    int cur_kh = -1;
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp; w < total; w += nwarps) {
+        const int kh = (int)(w / tiles);
+        const int64_t tile = w % tiles;
+        if (kh != cur_kh) {
+            load_ref<HD, R>(t.ref + (int64_t)kh * R * HD, rj, lane);
+            cur_kh = kh;
+        }
+        const int64_t tok0 = tile * tt;
+        const int ntok = (int)min((int64_t)tt, t.n_tokens - tok0);
+        const KT *Kh = reinterpret_cast<const KT *>(t.K) + (int64_t)kh * t.kv_cap * HD;
+        const int64_t nc = t.node_cap[0];
+        LeafOps<KT, HD, R>::tile(Kh, tok0, ntok, t.c, rj, t.scale, t.g[0] + (int64_t)kh * nc * R * HD,
+                                 t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, sh, lane);
+    }
+}
+
+template <int HD, int R>
+__global__ void __launch_bounds__(BUILD_THREADS) k_build_parents(Tree t, int level) {
+    extern __shared__ __align__(16) float bsm[];
+    constexpr int VEC = HD / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float *sh = bsm + warp * (t.c * R + R);
+    const int64_t nodes = t.n_level[level - 1];
+    const int64_t nbelow = t.n_level[level - 2];
+    const int64_t total = nodes * t.h_kv;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t capP = t.node_cap[level - 1], capC = t.node_cap[level - 2];
+    float rj[R][VEC];
+    int cur_kh = -1;
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp; w < total; w += nwarps) {
+        const int kh = (int)(w / nodes);
+        const int64_t n = w % nodes;
+        if (kh != cur_kh) {
+            load_ref<HD, R>(t.ref + (int64_t)kh * R * HD, rj, lane);
+            cur_kh = kh;
+        }
+        const int64_t ch0 = n * t.c;
+        const int nch = (int)min((int64_t)t.c, nbelow - ch0);
+        ParentOps<HD, R>::node(t.g[level - 2] + (int64_t)kh * capC * R * HD, t.b[level - 2] + (int64_t)kh * capC * R,
+                               ch0, nch, rj, t.scale, t.g[level - 1] + (int64_t)kh * capP * R * HD,
+                               t.b[level - 1] + (int64_t)kh * capP * R, t.m[level - 1] + (int64_t)kh * capP * R,
+                               n, sh, lane);
+    }
+}
+
+// One warp per KV head: store the new row, then recompute the leaf holding it
+// and every ancestor.  t.n_tokens and t.n_level already count the new token.
+template <typename KT, int HD, int R>
+__global__ void __launch_bounds__(32) k_append(Tree t, const KT *__restrict__ knew, const KT *__restrict__ vnew) {
+    extern __shared__ __align__(16) float bsm[];
+    constexpr int VEC = HD / 32;
+    const int lane = threadIdx.x;
+    const int kh = blockIdx.x;
+    const int64_t pos = t.n_tokens - 1;
+    KT *Kh = const_cast<KT *>(reinterpret_cast<const KT *>(t.K)) + (int64_t)kh * t.kv_cap * HD;
+    KT *Vh = const_cast<KT *>(reinterpret_cast<const KT *>(t.V)) + (int64_t)kh * t.kv_cap * HD;
+    for (int e = lane; e < HD; e += 32) {
+        Kh[pos * HD + e] = knew[kh * HD + e];
+        Vh[pos * HD + e] = vnew[kh * HD + e];
+    }
+    __syncwarp();
+    float rj[R][VEC];
+    load_ref<HD, R>(t.ref + (int64_t)kh * R * HD, rj, lane);
+    int64_t n = pos / t.c;
+    {
+        const int64_t tok0 = n * t.c;
+        const int ntok = (int)(t.n_tokens - tok0);
+        const int64_t nc = t.node_cap[0];
+        LeafOps<KT, HD, R>::tile(Kh, tok0, ntok, t.c, rj, t.scale, t.g[0] + (int64_t)kh * nc * R * HD,
+                                 t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, bsm, lane);
+    }
+    for (int level = 2; level <= t.D; ++level) {
+        n /= t.c;
+        const int64_t ch0 = n * t.c;
+        const int nch = (int)min((int64_t)t.c, (int64_t)t.n_level[level - 2] - ch0);
+        const int64_t capP = t.node_cap[level - 1], capC = t.node_cap[level - 2];
+        ParentOps<HD, R>::node(t.g[level - 2] + (int64_t)kh * capC * R * HD, t.b[level - 2] + (int64_t)kh * capC * R,
+                               ch0, nch, rj, t.scale, t.g[level - 1] + (int64_t)kh * capP * R * HD,
+                               t.b[level - 1] + (int64_t)kh * capP * R, t.m[level - 1] + (int64_t)kh * capP * R,
+                               n, bsm, lane);
+    }
+}
+
+// ---- dispatch ----------------------------------------------------------------
+
+template <typename KT, int HD, int R>
+static cudaError_t build_impl(const Tree &t, cudaStream_t s, int n_sm) {
+    const int warps = BUILD_THREADS / 32;
+    const int tt = leaf_tile_tokens(t.c, R);
+    size_t smem = (size_t)warps * (tt * R + (tt / t.c + 1) * R) * sizeof(float);
+    cudaError_t err = cudaFuncSetAttribute(k_build_leaves<KT, HD, R>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    const int64_t tiles = ((t.n_tokens + tt - 1) / tt) * t.h_kv;
+    int grid = (int)std::min<int64_t>((tiles + warps - 1) / warps, (int64_t)n_sm * 8);
+    k_build_leaves<KT, HD, R><<<grid, BUILD_THREADS, smem, s>>>(t);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    size_t psmem = (size_t)warps * (t.c * R + R) * sizeof(float);
+    err = cudaFuncSetAttribute(k_build_parents<HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+    if (err != cudaSuccess) return err;
+    for (int level = 2; level <= t.D; ++level) {
+        const int64_t work = (int64_t)t.n_level[level - 1] * t.h_kv;
+        int pgrid = (int)std::min<int64_t>((work + warps - 1) / warps, (int64_t)n_sm * 8);
+        k_build_parents<HD, R><<<pgrid, BUILD_THREADS, psmem, s>>>(t, level);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+}
+
+template <typename KT, int HD, int R>
+static cudaError_t append_impl(const Tree &t, const void *k, const void *v, cudaStream_t s) {
+    const int tt = leaf_tile_tokens(t.c, R);
+    const int rows = tt > t.c ? tt : t.c;
+    size_t smem = (size_t)(rows * R + (rows / t.c + 1) * R) * sizeof(float);
+    const size_t psmem = (size_t)(t.c * R + R) * sizeof(float);
+    if (psmem > smem) smem = psmem;
+    cudaError_t err = cudaFuncSetAttribute(k_append<KT, HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    k_append<KT, HD, R><<<t.h_kv, 32, smem, s>>>(t, reinterpret_cast<const KT *>(k), reinterpret_cast<const KT *>(v));
+    return cudaGetLastError();
+}
+
+#define ZHA_BUILD_DISPATCH(FN, ...)                                                           \
+    do {                                                                                      \
+        if (t.kv_dtype == 1) {                                                                \
+            if (t.d == 128 && t.R == 16) return FN<uint16_t, 128, 16>(__VA_ARGS__);           \
+            if (t.d == 128 && t.R == 1) return FN<uint16_t, 128, 1>(__VA_ARGS__);             \
+            if (t.d == 64 && t.R == 16) return FN<uint16_t, 64, 16>(__VA_ARGS__);             \
+            if (t.d == 64 && t.R == 1) return FN<uint16_t, 64, 1>(__VA_ARGS__);               \
+        } else {                                                                              \
+            if (t.d == 128 && t.R == 16) return FN<float, 128, 16>(__VA_ARGS__);              \
+            if (t.d == 128 && t.R == 1) return FN<float, 128, 1>(__VA_ARGS__);                \
+            if (t.d == 64 && t.R == 16) return FN<float, 64, 16>(__VA_ARGS__);                \
+            if (t.d == 64 && t.R == 1) return FN<float, 64, 1>(__VA_ARGS__);                  \
+        }                                                                                     \
+        return cudaErrorInvalidValue;                                                         \
+    } while (0)
+
+cudaError_t launch_build(const Tree &t, cudaStream_t s, int n_sm) { ZHA_BUILD_DISPATCH(build_impl, t, s, n_sm); }
+
+cudaError_t launch_append(const Tree &t, const void *k, const void *v, cudaStream_t s) {
+    ZHA_BUILD_DISPATCH(append_impl, t, k, v, s);
+}
+
+}  // namespace zha

@@ -18,8 +18,9 @@ Recipe (one generator, seeded with the workload's seed; draws in this order):
 4. values ``V ~ N(0, I)``, one KV head at a time;
 5. needles: every (step, query head) owns ``needles`` positions in its KV
    head, all distinct within the KV head; a quarter of them (when the
-   workload asks for a tail) lie in the last 4,096 tokens, the rest are
-   uniform over ``[1, N - 4096)`` (over ``[1, N)`` without a tail).  The key
+   workload asks for a tail) lie in the last 4,096 tokens (the last N/2 for
+   N < 8,192), the rest are uniform over the tokens before that window from
+   token 1 on (over ``[1, N)`` without a tail).  The key
    at a needle of query ``q`` is ``3 * q / |q| * sqrt(d) + eps`` with
    ``eps ~ N(0, 0.1 I)`` (variance 0.1);
 6. the cache is cast to its storage dtype (bf16 or fp32);
@@ -161,8 +162,9 @@ def generate(w: Workload, device: str = "cpu") -> Inputs:
         if w.needle_tail:
             n_tail = w.steps * G * (w.needles // 4)
             n_body = per_kv - n_tail
-            tail = (N - TAIL) + torch.randperm(TAIL, generator=gen, device=device)[:n_tail]
-            body = 1 + torch.randperm(N - TAIL - 1, generator=gen, device=device)[:n_body]
+            win = min(TAIL, N // 2)
+            tail = (N - win) + torch.randperm(win, generator=gen, device=device)[:n_tail]
+            body = 1 + torch.randperm(N - win - 1, generator=gen, device=device)[:n_body]
             # per query: needles//4 tail positions then the body positions
             tail = tail.view(w.steps * G, w.needles // 4)
             body = body.view(w.steps * G, w.needles - w.needles // 4)
