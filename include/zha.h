@@ -179,15 +179,15 @@ int zha_dense_decode(zha_ctx *ctx, const float *d_q, float *d_out, void *stream)
 int zha_device_status(zha_ctx *ctx, int32_t *out_status, void *stream);
 
 /*
- * Profiling hook: record CUDA events between the kernels of zha_decode.
- *   events    array of n_events cudaEvent_t (passed as void*), owned by the
- *             caller and kept alive while set; NULL with n_events = 0 clears.
- *   n_events  D + 2: events[0] is recorded on the decode stream before the
- *             first routing kernel, events[i] (1 <= i <= D) after the routing
- *             kernel of level D + 1 - i, events[D + 1] after attention.
- * Returns ZHA_ERR_BAD_ARG for any other count.  No effect on results.
+ * Profiling hook: zha_decode runs as one kernel; when a buffer is set, the
+ * kernel writes the GPU global timer (nanoseconds) at its phase boundaries:
+ *   d_ns  caller-owned device buffer of D + 3 int64 (8-byte aligned), kept
+ *         alive while set; NULL clears.  d_ns[0] = start, d_ns[i] (1..D) =
+ *         end of the routing level D + 1 - i, d_ns[D + 1] = end of the
+ *         attention over the kept tokens, d_ns[D + 2] = end of the merge.
+ * No effect on results.
  */
-int zha_set_phase_events(zha_ctx *ctx, void *const *events, int32_t n_events);
+int zha_set_phase_timer(zha_ctx *ctx, int64_t *d_ns);
 
 /* Tokens currently in the cache (host-side count; 0 before zha_build). */
 int64_t zha_n_tokens(const zha_ctx *ctx);

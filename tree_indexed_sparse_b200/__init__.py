@@ -12,7 +12,8 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libzha.so")
+# ZHA_LIB selects another build of the same library (e.g. an instrumented one)
+LIB_PATH = os.environ.get("ZHA_LIB") or os.path.join(_HERE, "libzha.so")
 
 ZHA_OK = 0
 ZHA_ERR_BAD_ARG = -1
@@ -26,7 +27,7 @@ ZHA_BF16 = 1
 
 # every symbol include/zha.h declares
 EXPORTS = ["zha_workspace_bytes", "zha_create", "zha_destroy", "zha_build", "zha_append", "zha_decode",
-           "zha_dense_decode", "zha_device_status", "zha_set_phase_events", "zha_n_tokens",
+           "zha_dense_decode", "zha_device_status", "zha_set_phase_timer", "zha_n_tokens",
            "zha_summary_layout", "zha_strerror"]
 
 
@@ -65,8 +66,8 @@ def _load() -> ctypes.CDLL:
     lib.zha_dense_decode.restype = ctypes.c_int
     lib.zha_device_status.argtypes = [P, ctypes.POINTER(I32), P]
     lib.zha_device_status.restype = ctypes.c_int
-    lib.zha_set_phase_events.argtypes = [P, ctypes.POINTER(P), I32]
-    lib.zha_set_phase_events.restype = ctypes.c_int
+    lib.zha_set_phase_timer.argtypes = [P, P]
+    lib.zha_set_phase_timer.restype = ctypes.c_int
     lib.zha_n_tokens.argtypes = [P]
     lib.zha_n_tokens.restype = I64
     lib.zha_summary_layout.argtypes = [P, I32, ctypes.POINTER(I64), ctypes.POINTER(I64),
@@ -141,22 +142,10 @@ def zha_device_status(ctx, stream=None) -> int:
     return int(st.value)
 
 
-def zha_set_phase_events(ctx, events) -> None:
-    """events: a list of D + 2 torch.cuda.Event (or raw cudaEvent_t ints), or
-    None to clear.  Keep the events alive while they are set."""
-    if not events:
-        _check(lib.zha_set_phase_events(ctx, None, 0), "zha_set_phase_events")
-        return
-    handles = []
-    for e in events:
-        if hasattr(e, "cuda_event"):
-            if not e.cuda_event:  # torch creates the CUDA event on first record
-                e.record()
-            handles.append(e.cuda_event)
-        else:
-            handles.append(int(e))
-    arr = (ctypes.c_void_p * len(handles))(*handles)
-    _check(lib.zha_set_phase_events(ctx, arr, len(handles)), "zha_set_phase_events")
+def zha_set_phase_timer(ctx, d_ns) -> None:
+    """d_ns: device int64 tensor of D + 3 entries for the decode phase stamps
+    (global timer, ns), or None to clear.  Keep it alive while set."""
+    _check(lib.zha_set_phase_timer(ctx, _vp(d_ns)), "zha_set_phase_timer")
 
 
 def zha_n_tokens(ctx) -> int:
@@ -193,9 +182,10 @@ class ZhaCache:
         self._keep = ()
 
     def close(self) -> None:
-        if getattr(self, "ctx", None):
+        # at interpreter shutdown the module globals may already be gone
+        if getattr(self, "ctx", None) and lib is not None and zha_destroy is not None:
             zha_destroy(self.ctx)
-            self.ctx = None
+        self.ctx = None
 
     def __del__(self):
         self.close()

@@ -25,6 +25,7 @@ struct zha_ctx {
     uint8_t *kept_mask[MAXD];
     int32_t *kept_cnt;
     float *scores;
+    int32_t *slot_node;
     int64_t score_cap;
     float *pmax;
     int pmax_cap;
@@ -35,8 +36,9 @@ struct zha_ctx {
     int32_t *status;
     unsigned char *scratch_begin;
     int64_t scratch_bytes;
-    cudaEvent_t phase_ev[MAXD + 2];
-    int n_phase_ev;
+    unsigned *gbar;
+    int64_t *phase_ns;            // caller's device buffer for phase stamps, or null
+    int decode_cta;
     int n_sm;
     int route_cta;
     int attn_cta;
@@ -75,7 +77,7 @@ struct Layout {
     int64_t node_cap[MAXD];
     int64_t g_off[MAXD], b_off[MAXD], m_off[MAXD];
     int64_t kid_off[MAXD], kmask_off[MAXD];
-    int64_t kcnt_off, scores_off, pmax_off, done_off, vis_off, part_off, status_off;
+    int64_t kcnt_off, scores_off, snode_off, pmax_off, done_off, vis_off, part_off, gbar_off, status_off;
     int64_t scratch_off, total;
     int64_t score_cap;
 };
@@ -108,6 +110,8 @@ void make_layout(const zha_config *cfg, Layout *L) {
     off = align256(off + (int64_t)MAXD * cfg->h_kv * 4);
     L->scores_off = off;
     off = align256(off + (int64_t)cfg->h_kv * sc * G * 4);
+    L->snode_off = off;
+    off = align256(off + (int64_t)cfg->h_kv * sc * 4);
     L->pmax_off = off;
     off = align256(off + (int64_t)cfg->h_kv * PMAX_CAP * G * 4);
     L->done_off = off;
@@ -115,7 +119,9 @@ void make_layout(const zha_config *cfg, Layout *L) {
     L->vis_off = off;
     off = align256(off + (int64_t)cfg->h_q * 8);
     L->part_off = off;
-    off = align256(off + (int64_t)PART_CAP * cfg->h_kv * G * (cfg->d + 2) * 4);
+    off = align256(off + (int64_t)PART_CAP * cfg->h_kv * G * (cfg->d + 4) * 4);
+    L->gbar_off = off;
+    off = align256(off + 16);
     L->status_off = off;
     off = align256(off + 4);
     L->total = off;
@@ -141,6 +147,7 @@ Decode make_decode(zha_ctx *ctx) {
     }
     dc.kept_cnt = ctx->kept_cnt;
     dc.scores = ctx->scores;
+    dc.slot_node = ctx->slot_node;
     dc.score_cap = ctx->score_cap;
     dc.pmax = ctx->pmax;
     dc.pmax_cap = ctx->pmax_cap;
@@ -148,6 +155,8 @@ Decode make_decode(zha_ctx *ctx) {
     dc.vis_acc = ctx->vis_acc;
     dc.part = ctx->part;
     dc.part_cap = ctx->part_cap;
+    dc.gbar = ctx->gbar;
+    dc.phase_ns = ctx->phase_ns;
     dc.status = ctx->status;
     return dc;
 }
@@ -204,6 +213,7 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
     }
     ctx->kept_cnt = reinterpret_cast<int32_t *>(ws + L.kcnt_off);
     ctx->scores = reinterpret_cast<float *>(ws + L.scores_off);
+    ctx->slot_node = reinterpret_cast<int32_t *>(ws + L.snode_off);
     ctx->score_cap = L.score_cap;
     ctx->pmax = reinterpret_cast<float *>(ws + L.pmax_off);
     ctx->pmax_cap = PMAX_CAP;
@@ -211,6 +221,7 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
     ctx->vis_acc = reinterpret_cast<int64_t *>(ws + L.vis_off);
     ctx->part = reinterpret_cast<float *>(ws + L.part_off);
     ctx->part_cap = PART_CAP;
+    ctx->gbar = reinterpret_cast<unsigned *>(ws + L.gbar_off);
     ctx->status = reinterpret_cast<int32_t *>(ws + L.status_off);
     ctx->scratch_begin = ws + L.scratch_off;
     ctx->scratch_bytes = L.total - L.scratch_off;
@@ -221,9 +232,20 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
         delete ctx;
         return ZHA_ERR_CUDA;
     }
-    ctx->route_cta = std::max(1, ctx->n_sm / cfg->h_kv) * cfg->h_kv;
-    if (ctx->route_cta / cfg->h_kv > PMAX_CAP) ctx->route_cta = PMAX_CAP * cfg->h_kv;
-    ctx->attn_cta = std::min(PART_CAP, 2 * ctx->n_sm);
+    ctx->attn_cta = std::min(PART_CAP, ctx->n_sm);  // one CTA per SM, one wave
+    // the decode kernel: one resident CTA per SM (cooperative launch), a
+    // multiple of h_kv so that every KV head gets the same number of CTAs
+    {
+        Decode probe = make_decode(ctx);
+        const int per_sm = decode_blocks_per_sm(probe);
+        if (per_sm < 1) {
+            delete ctx;
+            return ZHA_ERR_CUDA;
+        }
+        int n = std::min(std::min(ctx->n_sm, PART_CAP), PMAX_CAP * cfg->h_kv);
+        n = std::max(1, n / cfg->h_kv) * cfg->h_kv;
+        ctx->decode_cta = n;
+    }
     if (cudaMemset(ctx->scratch_begin, 0, (size_t)ctx->scratch_bytes) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess) {
         delete ctx;
@@ -287,16 +309,7 @@ int zha_decode(zha_ctx *ctx, const float *d_q, float p, float *d_out, int32_t *d
     dc.trace_ids = d_trace_ids;
     dc.trace_cnt = d_trace_ids ? d_trace_counts : nullptr;
     dc.trace_cap = d_trace_ids ? trace_cap : 0;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const size_t smem = route_smem_bytes(ctx->t.G);
-    const bool ev = ctx->n_phase_ev > 0;
-    if (ev && cudaEventRecord(ctx->phase_ev[0], s) != cudaSuccess) return ZHA_ERR_CUDA;
-    for (int l = ctx->t.D; l >= 1; --l) {
-        if (launch_route_level(dc, l, ctx->route_cta, smem, s) != cudaSuccess) return ZHA_ERR_CUDA;
-        if (ev && cudaEventRecord(ctx->phase_ev[ctx->t.D + 1 - l], s) != cudaSuccess) return ZHA_ERR_CUDA;
-    }
-    if (launch_attend(dc, ctx->attn_cta, s) != cudaSuccess) return ZHA_ERR_CUDA;
-    if (ev && cudaEventRecord(ctx->phase_ev[ctx->t.D + 1], s) != cudaSuccess) return ZHA_ERR_CUDA;
+    if (launch_decode(dc, ctx->decode_cta, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZHA_ERR_CUDA;
     return ZHA_OK;
 }
 
@@ -307,8 +320,7 @@ int zha_dense_decode(zha_ctx *ctx, const float *d_q, float *d_out, void *stream)
     Decode dc = make_decode(ctx);
     dc.q = d_q;
     dc.out = d_out;
-    const int per = std::max(1, std::min(ctx->part_cap, 2 * ctx->n_sm) / ctx->cfg.h_kv);
-    if (launch_dense(dc, per * ctx->cfg.h_kv, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZHA_ERR_CUDA;
+    if (launch_dense(dc, ctx->attn_cta, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZHA_ERR_CUDA;
     return ZHA_OK;
 }
 
@@ -319,22 +331,18 @@ int zha_device_status(zha_ctx *ctx, int32_t *out_status, void *stream) {
     if (cudaMemcpyAsync(&host, ctx->status, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaMemsetAsync(ctx->status, 0, sizeof host, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
         return ZHA_ERR_CUDA;
+    // after a timed-out wait the grid barrier words are reset for the next call
+    if (host == ZHA_ERR_TIMEOUT &&
+        (cudaMemsetAsync(ctx->gbar, 0, 16, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess))
+        return ZHA_ERR_CUDA;
     *out_status = host;
     return ZHA_OK;
 }
 
-int zha_set_phase_events(zha_ctx *ctx, void *const *events, int32_t n_events) {
+int zha_set_phase_timer(zha_ctx *ctx, int64_t *d_ns) {
     if (!ctx) return ZHA_ERR_BAD_ARG;
-    if (n_events == 0) {
-        ctx->n_phase_ev = 0;
-        return ZHA_OK;
-    }
-    if (!events || n_events != ctx->cfg.D + 2) return ZHA_ERR_BAD_ARG;
-    for (int i = 0; i < n_events; ++i) {
-        if (!events[i]) return ZHA_ERR_BAD_ARG;
-        ctx->phase_ev[i] = static_cast<cudaEvent_t>(events[i]);
-    }
-    ctx->n_phase_ev = n_events;
+    if (d_ns && (reinterpret_cast<uintptr_t>(d_ns) & 7u)) return ZHA_ERR_BAD_ARG;
+    ctx->phase_ns = d_ns;
     return ZHA_OK;
 }
 

@@ -320,17 +320,24 @@ static cudaError_t build_impl(const Tree &t, cudaStream_t s, int n_sm) {
     const int warps = BUILD_THREADS / 32;
     const int tt = leaf_tile_tokens(t.c, R);
     size_t smem = (size_t)warps * (tt * R + (tt / t.c + 1) * R) * sizeof(float);
-    cudaError_t err = cudaFuncSetAttribute(k_build_leaves<KT, HD, R>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
+    cudaError_t err;
+    static size_t leaf_attr = 0, parent_attr = 0;
+    if (smem > leaf_attr) {
+        err = cudaFuncSetAttribute(k_build_leaves<KT, HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        leaf_attr = smem;
+    }
     const int64_t tiles = ((t.n_tokens + tt - 1) / tt) * t.h_kv;
     int grid = (int)std::min<int64_t>((tiles + warps - 1) / warps, (int64_t)n_sm * 8);
     k_build_leaves<KT, HD, R><<<grid, BUILD_THREADS, smem, s>>>(t);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     size_t psmem = (size_t)warps * (t.c * R + R) * sizeof(float);
-    err = cudaFuncSetAttribute(k_build_parents<HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
-    if (err != cudaSuccess) return err;
+    if (psmem > parent_attr) {
+        err = cudaFuncSetAttribute(k_build_parents<HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
+        if (err != cudaSuccess) return err;
+        parent_attr = psmem;
+    }
     for (int level = 2; level <= t.D; ++level) {
         const int64_t work = (int64_t)t.n_level[level - 1] * t.h_kv;
         int pgrid = (int)std::min<int64_t>((work + warps - 1) / warps, (int64_t)n_sm * 8);
@@ -348,8 +355,12 @@ static cudaError_t append_impl(const Tree &t, const void *k, const void *v, cuda
     size_t smem = (size_t)(rows * R + (rows / t.c + 1) * R) * sizeof(float);
     const size_t psmem = (size_t)(t.c * R + R) * sizeof(float);
     if (psmem > smem) smem = psmem;
-    cudaError_t err = cudaFuncSetAttribute(k_append<KT, HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
+    static size_t attr = 0;
+    if (smem > attr) {
+        cudaError_t err = cudaFuncSetAttribute(k_append<KT, HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        attr = smem;
+    }
     k_append<KT, HD, R><<<t.h_kv, 32, smem, s>>>(t, reinterpret_cast<const KT *>(k), reinterpret_cast<const KT *>(v));
     return cudaGetLastError();
 }

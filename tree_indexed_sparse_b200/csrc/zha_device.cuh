@@ -258,3 +258,109 @@ __device__ __forceinline__ uint32_t block_max_u32(uint32_t x, uint32_t *sh) {
 }
 
 }  // namespace zha
+
+namespace zha {
+
+// ---- helpers over the first 256 threads of a CTA (named barrier 1) ---------
+//
+// The decode kernel runs 9 warps per CTA; routing phases use warps 0-7 and
+// synchronise them with `bar.sync 1, 256` while warp 8 stays out.
+
+constexpr int GT = 256;  // threads of a group
+
+__device__ __forceinline__ void gsync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ unsigned long long g_scan_u64(unsigned long long x, unsigned long long *sh,
+                                                         unsigned long long *total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    unsigned long long v = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        unsigned long long y = __shfl_up_sync(FULL, v, off);
+        if (lane >= off) v += y;
+    }
+    if (lane == 31) sh[wid] = v;
+    gsync();
+    unsigned long long base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < GT / 32; ++w) {
+        const unsigned long long s = sh[w];
+        if (w < wid) base += s;
+        tot += s;
+    }
+    gsync();
+    *total = tot;
+    return base + v;
+}
+
+__device__ __forceinline__ uint32_t g_scan_u32(uint32_t x, uint32_t *sh, uint32_t *total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint32_t v = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        uint32_t y = __shfl_up_sync(FULL, v, off);
+        if (lane >= off) v += y;
+    }
+    if (lane == 31) sh[wid] = v;
+    gsync();
+    uint32_t base = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < GT / 32; ++w) {
+        const uint32_t s = sh[w];
+        if (w < wid) base += s;
+        tot += s;
+    }
+    gsync();
+    *total = tot;
+    return base + v;
+}
+
+__device__ __forceinline__ uint32_t g_min_u32(uint32_t x, uint32_t *sh) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) x = min(x, __shfl_xor_sync(FULL, x, off));
+    if (lane == 0) sh[wid] = x;
+    gsync();
+    uint32_t r = 0xffffffffu;
+#pragma unroll
+    for (int w = 0; w < GT / 32; ++w) r = min(r, sh[w]);
+    gsync();
+    return r;
+}
+
+__device__ __forceinline__ uint32_t g_max_u32(uint32_t x, uint32_t *sh) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) x = max(x, __shfl_xor_sync(FULL, x, off));
+    if (lane == 0) sh[wid] = x;
+    gsync();
+    uint32_t r = 0u;
+#pragma unroll
+    for (int w = 0; w < GT / 32; ++w) r = max(r, sh[w]);
+    gsync();
+    return r;
+}
+
+// Sums of NV u64 values per thread over the group (fixed tree order).
+template <int NV>
+__device__ __forceinline__ void g_sum_u64(unsigned long long (&v)[NV], unsigned long long *red) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        unsigned long long x = v[i];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+        if (lane == 0) red[wid * NV + i] = x;
+    }
+    gsync();
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        unsigned long long s = 0;
+#pragma unroll
+        for (int w = 0; w < GT / 32; ++w) s += red[w * NV + i];
+        v[i] = s;
+    }
+    gsync();
+}
+
+}  // namespace zha

@@ -41,14 +41,17 @@ struct Decode {
     int32_t *kept_ids[MAXD];      // level l: [h_kv][node_cap[l-1]] ascending union kept ids
     uint8_t *kept_mask[MAXD];     // head bitmask per kept id
     int32_t *kept_cnt;            // [MAXD][h_kv]
-    float *scores;                // [h_kv][score_cap][G]
+    float *scores;                // [h_kv][score_cap][G]; -inf where the head does not need the slot
+    int32_t *slot_node;           // [h_kv][score_cap] node id of each frontier slot
     int64_t score_cap;
     float *pmax;                  // [h_kv][pmax_cap][G]
     int pmax_cap;
     uint32_t *done;               // [MAXD][h_kv] level tickets, then [h_kv] attention tickets
     int64_t *vis_acc;             // [h_q]
-    float *part;                  // attention partials [part_cap][h_kv][G][d+2]
+    float *part;                  // attention partials [part_cap][h_kv][G][d+4]
     int part_cap;
+    unsigned *gbar;               // grid barrier: arrivals, generation, abort flag
+    int64_t *phase_ns;            // nullable: globaltimer stamps per decode phase
     int32_t *status;
     float *out;
     int32_t *leaf_idx;
@@ -60,6 +63,10 @@ struct Decode {
     int32_t trace_cap;
 };
 
+// device status codes (the values of include/zha.h)
+constexpr int32_t ZHA_CAPACITY_CODE = -2;
+constexpr int32_t ZHA_TIMEOUT_CODE = -5;
+
 // status word helpers (first error wins)
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
     atomicCAS(status, 0, code);
@@ -68,9 +75,8 @@ __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
 // host-side launchers; each returns a cudaError_t (0 on success)
 cudaError_t launch_build(const Tree &t, cudaStream_t s, int n_sm);
 cudaError_t launch_append(const Tree &t, const void *k, const void *v, cudaStream_t s);
-cudaError_t launch_route_level(const Decode &dc, int level, int n_cta, size_t smem, cudaStream_t s);
-size_t route_smem_bytes(int G);
-cudaError_t launch_attend(const Decode &dc, int n_cta, cudaStream_t s);
+cudaError_t launch_decode(const Decode &dc, int n_cta, cudaStream_t s);
+int decode_blocks_per_sm(const Decode &dc);
 cudaError_t launch_dense(const Decode &dc, int n_cta, cudaStream_t s);
 bool compiled_combo(int kv_dtype, int d, int R, int G);
 
