@@ -173,6 +173,36 @@ int zha_decode(zha_ctx *ctx, const float *d_q, float p, float *d_out, int32_t *d
 int zha_dense_decode(zha_ctx *ctx, const float *d_q, float *d_out, void *stream);
 
 /*
+ * Dense flash-decode straight from a KV cache, with no context and no
+ * workspace.  The pages have no counterpart: this serves layers that keep
+ * plain dense attention inside an engine that reserves all of its device
+ * memory up front and may not allocate while it serves, so it has no
+ * workspace to hand over.  The split partials and merge tickets live in a
+ * fixed scratch array of ZHA_STATIC_SCRATCH_BYTES inside the library's device
+ * image; the call allocates nothing.
+ *   cfg              h_kv, h_q, d, kv_dtype, capacity_tokens as for a context
+ *                    (R, c, D are ignored)
+ *   d_K, d_V         [h_kv][capacity_tokens][d] kv_dtype, 16-byte aligned
+ *   n_tokens         rows attended per KV head, 1 <= n_tokens <= capacity
+ *   d_q, d_out       [h_q][d] fp32, 16-byte aligned
+ *   d_status         caller's device int32; a device-side failure (an
+ *                    exhausted bounded wait) writes ZHA_ERR_TIMEOUT there if
+ *                    it holds ZHA_OK; the caller reads and clears it
+ * Same arithmetic and grid as zha_dense_decode.  Returns ZHA_ERR_CAPACITY
+ * when the partials, h_q * (d + 4) * 4 bytes per SM (one CTA per SM, at most
+ * 1024), plus (16 + 2) * h_kv * 4 bytes of tickets, exceed
+ * ZHA_STATIC_SCRATCH_BYTES (for d = 128 on 148 SMs: h_q <= 107).
+ * The first call on each device looks up the scratch's device address
+ * (cudaGetSymbolAddress, with that device current), so make it before any
+ * stream capture begins.  Every call clears the tickets on `stream` first.
+ * One call at a time per device: calls in flight together, on any streams or
+ * host threads, share the scratch and corrupt each other's outputs.
+ */
+#define ZHA_STATIC_SCRATCH_BYTES (8 * 1024 * 1024)
+int zha_dense_decode_static(const zha_config *cfg, const void *d_K, const void *d_V, int64_t n_tokens,
+                            const float *d_q, float *d_out, int32_t *d_status, void *stream);
+
+/*
  * Copy the device status word to *out_status and clear it.  Synchronises
  * `stream` first.  ZHA_OK means every decode since the last read was valid.
  */

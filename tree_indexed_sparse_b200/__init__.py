@@ -27,7 +27,7 @@ ZHA_BF16 = 1
 
 # every symbol include/zha.h declares
 EXPORTS = ["zha_workspace_bytes", "zha_create", "zha_destroy", "zha_build", "zha_append", "zha_decode",
-           "zha_dense_decode", "zha_device_status", "zha_set_phase_timer", "zha_n_tokens",
+           "zha_dense_decode", "zha_dense_decode_static", "zha_device_status", "zha_set_phase_timer", "zha_n_tokens",
            "zha_summary_layout", "zha_strerror"]
 
 
@@ -64,6 +64,8 @@ def _load() -> ctypes.CDLL:
     lib.zha_decode.restype = ctypes.c_int
     lib.zha_dense_decode.argtypes = [P, P, P, P]
     lib.zha_dense_decode.restype = ctypes.c_int
+    lib.zha_dense_decode_static.argtypes = [CFG, P, P, I64, P, P, P, P]
+    lib.zha_dense_decode_static.restype = ctypes.c_int
     lib.zha_device_status.argtypes = [P, ctypes.POINTER(I32), P]
     lib.zha_device_status.restype = ctypes.c_int
     lib.zha_set_phase_timer.argtypes = [P, P]
@@ -134,6 +136,11 @@ def zha_decode(ctx, d_q, p: float, d_out, d_leaf_idx=None, leaf_cap: int = 0, d_
 
 def zha_dense_decode(ctx, d_q, d_out, stream=None) -> None:
     _check(lib.zha_dense_decode(ctx, _vp(d_q), _vp(d_out), _vp(stream)), "zha_dense_decode")
+
+
+def zha_dense_decode_static(cfg: zha_config, d_K, d_V, n_tokens: int, d_q, d_out, d_status, stream=None) -> None:
+    _check(lib.zha_dense_decode_static(ctypes.byref(cfg), _vp(d_K), _vp(d_V), int(n_tokens), _vp(d_q), _vp(d_out),
+                                       _vp(d_status), _vp(stream)), "zha_dense_decode_static")
 
 
 def zha_device_status(ctx, stream=None) -> int:
