@@ -190,8 +190,8 @@ int zha_dense_decode(zha_ctx *ctx, const float *d_q, float *d_out, void *stream)
  *                    it holds ZHA_OK; the caller reads and clears it
  * Same arithmetic and grid as zha_dense_decode.  Returns ZHA_ERR_CAPACITY
  * when the partials, h_q * (d + 4) * 4 bytes per SM (one CTA per SM, at most
- * 1024), plus (16 + 2) * h_kv * 4 bytes of tickets, exceed
- * ZHA_STATIC_SCRATCH_BYTES (for d = 128 on 148 SMs: h_q <= 107).
+ * 256), plus h_kv * 4 bytes of tickets, exceed ZHA_STATIC_SCRATCH_BYTES
+ * (for d = 128 on 148 SMs: h_q <= 107).
  * The first call on each device looks up the scratch's device address
  * (cudaGetSymbolAddress, with that device current), so make it before any
  * stream capture begins.  Every call clears the tickets on `stream` first.
@@ -212,9 +212,10 @@ int zha_device_status(zha_ctx *ctx, int32_t *out_status, void *stream);
  * Profiling hook: zha_decode runs as one kernel; when a buffer is set, the
  * kernel writes the GPU global timer (nanoseconds) at its phase boundaries:
  *   d_ns  caller-owned device buffer of D + 3 int64 (8-byte aligned), kept
- *         alive while set; NULL clears.  d_ns[0] = start, d_ns[i] (1..D) =
- *         end of the routing level D + 1 - i, d_ns[D + 1] = end of the
- *         attention over the kept tokens, d_ns[D + 2] = end of the merge.
+ *         alive while set; NULL clears.  d_ns[0] = start, d_ns[D] = end of
+ *         the routing (every level), d_ns[D + 1] = end of this CTA's share of
+ *         the attention over the kept tokens, d_ns[D + 2] = end of the merge;
+ *         d_ns[1 .. D-1] are not written.
  * No effect on results.
  */
 int zha_set_phase_timer(zha_ctx *ctx, int64_t *d_ns);

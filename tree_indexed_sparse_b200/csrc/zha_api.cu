@@ -20,34 +20,18 @@ struct zha_ctx {
     bool built;
     unsigned char *ws;
     int64_t ws_bytes;
-    // decode scratch (inside the workspace)
-    int32_t *kept_ids[MAXD];
-    uint8_t *kept_mask[MAXD];
-    int32_t *kept_cnt;
-    float *scores;
-    int32_t *slot_node;
-    int64_t score_cap;
-    float *pmax;
-    int pmax_cap;
-    uint32_t *done;
-    int64_t *vis_acc;
-    float *part;
-    int part_cap;
-    int32_t *status;
+    Decode scratch;           // decode scratch pointers (inside the workspace); t and outputs unset
     unsigned char *scratch_begin;
     int64_t scratch_bytes;
-    unsigned *gbar;
-    int64_t *phase_ns;            // caller's device buffer for phase stamps, or null
+    int64_t *phase_ns;        // caller's device buffer for phase stamps, or null
     int decode_cta;
     int n_sm;
-    int route_cta;
     int attn_cta;
 };
 
 namespace {
 
-constexpr int PMAX_CAP = 1024;
-constexpr int PART_CAP = 1024;
+constexpr int PART_CAP = SEG_CAP;  // attention partial records per KV head (one per CTA)
 
 int64_t align256(int64_t x) { return (x + 255) / 256 * 256; }
 
@@ -74,56 +58,67 @@ int check_config(const zha_config *cfg) {
 
 // Byte layout of the workspace.  Each region starts 256-byte aligned.
 struct Layout {
-    int64_t node_cap[MAXD];
+    int64_t node_cap[MAXD], slot_cap[MAXD];
     int64_t g_off[MAXD], b_off[MAXD], m_off[MAXD];
     int64_t kid_off[MAXD], kmask_off[MAXD];
-    int64_t kcnt_off, scores_off, snode_off, pmax_off, done_off, vis_off, part_off, gbar_off, status_off;
+    int64_t seg_off, hseg_off, lvl_off, cur_off, scores_off, snode_off, skeep_off, tmax_off, tcnt_off, tsum_off;
+    int64_t hcnt_off, hmass_off, cw_off, cs_off, ccnt_off, ticket_off, part_off, sync_off, status_off;
     int64_t scratch_off, total;
     int64_t score_cap;
 };
 
 void make_layout(const zha_config *cfg, Layout *L) {
     const int G = cfg->h_q / cfg->h_kv;
+    const int64_t H = cfg->h_kv;
     int64_t off = 0;
     for (int l = 1; l <= cfg->D; ++l) {
         const int64_t nc = level_nodes(cfg->capacity_tokens, cfg->c, l);
         L->node_cap[l - 1] = nc;
         L->g_off[l - 1] = off;
-        off = align256(off + (int64_t)cfg->h_kv * nc * cfg->R * cfg->d * 4);
+        off = align256(off + H * nc * cfg->R * cfg->d * 4);
         L->b_off[l - 1] = off;
-        off = align256(off + (int64_t)cfg->h_kv * nc * cfg->R * 4);
+        off = align256(off + H * nc * cfg->R * 4);
         L->m_off[l - 1] = off;
-        off = align256(off + (int64_t)cfg->h_kv * nc * cfg->R * 4);
+        off = align256(off + H * nc * cfg->R * 4);
     }
+    // frontier slots of level l: every top node, or c children of each node
+    // of level l + 1
+    int64_t sc = 0;
+    for (int l = 1; l <= cfg->D; ++l) {
+        L->slot_cap[l - 1] = (l == cfg->D) ? L->node_cap[l - 1] : (int64_t)cfg->c * L->node_cap[l];
+        sc = std::max(sc, L->slot_cap[l - 1]);
+    }
+    L->score_cap = sc;
     L->scratch_off = off;
     for (int l = 1; l <= cfg->D; ++l) {
         L->kid_off[l - 1] = off;
-        off = align256(off + (int64_t)cfg->h_kv * L->node_cap[l - 1] * 4);
+        off = align256(off + H * L->slot_cap[l - 1] * 4);
         L->kmask_off[l - 1] = off;
-        off = align256(off + (int64_t)cfg->h_kv * L->node_cap[l - 1]);
+        off = align256(off + H * L->slot_cap[l - 1]);
     }
-    // frontier slots: every top node, or the children of the kept nodes one level up
-    int64_t sc = L->node_cap[cfg->D - 1];
-    for (int l = 1; l < cfg->D; ++l) sc = std::max(sc, (int64_t)cfg->c * L->node_cap[l]);
-    L->score_cap = sc;
-    L->kcnt_off = off;
-    off = align256(off + (int64_t)MAXD * cfg->h_kv * 4);
-    L->scores_off = off;
-    off = align256(off + (int64_t)cfg->h_kv * sc * G * 4);
-    L->snode_off = off;
-    off = align256(off + (int64_t)cfg->h_kv * sc * 4);
-    L->pmax_off = off;
-    off = align256(off + (int64_t)cfg->h_kv * PMAX_CAP * G * 4);
-    L->done_off = off;
-    off = align256(off + (int64_t)(MAXD + 2) * cfg->h_kv * 4);
-    L->vis_off = off;
-    off = align256(off + (int64_t)cfg->h_q * 8);
-    L->part_off = off;
-    off = align256(off + (int64_t)PART_CAP * cfg->h_kv * G * (cfg->d + 4) * 4);
-    L->gbar_off = off;
-    off = align256(off + 16);
-    L->status_off = off;
-    off = align256(off + 4);
+    auto take = [&](int64_t &at, int64_t bytes) {
+        at = off;
+        off = align256(off + bytes);
+    };
+    take(L->seg_off, (int64_t)MAXD * H * SEG_CAP * 4);
+    take(L->hseg_off, (int64_t)MAXD * H * SEG_CAP * G * 4);
+    take(L->lvl_off, (int64_t)MAXD * H * 2 * 4);
+    take(L->cur_off, H * 4);
+    take(L->scores_off, H * sc * G * 4);
+    take(L->snode_off, H * sc * 4);
+    take(L->skeep_off, H * sc + 4);
+    take(L->tmax_off, H * SEG_CAP * G * 4);
+    take(L->tcnt_off, H * SEG_CAP * G * 4);
+    take(L->tsum_off, H * SEG_CAP * G * 8);
+    take(L->hcnt_off, H * HIST_ROUNDS * G * NB * 4);
+    take(L->hmass_off, H * HIST_ROUNDS * G * NB * 8);
+    take(L->cw_off, H * G * CAND_MAX * 8);
+    take(L->cs_off, H * G * CAND_MAX * 4);
+    take(L->ccnt_off, H * G * 4);
+    take(L->ticket_off, H * 4);
+    take(L->part_off, (int64_t)PART_CAP * H * G * (cfg->d + 4) * 4);
+    take(L->sync_off, (H + 3) * 4);
+    take(L->status_off, 4);
     L->total = off;
 }
 
@@ -138,26 +133,9 @@ void fill_tree_levels(zha_ctx *ctx) {
 }
 
 Decode make_decode(zha_ctx *ctx) {
-    Decode dc;
-    std::memset(&dc, 0, sizeof dc);
+    Decode dc = ctx->scratch;
     dc.t = ctx->t;
-    for (int l = 0; l < MAXD; ++l) {
-        dc.kept_ids[l] = ctx->kept_ids[l];
-        dc.kept_mask[l] = ctx->kept_mask[l];
-    }
-    dc.kept_cnt = ctx->kept_cnt;
-    dc.scores = ctx->scores;
-    dc.slot_node = ctx->slot_node;
-    dc.score_cap = ctx->score_cap;
-    dc.pmax = ctx->pmax;
-    dc.pmax_cap = ctx->pmax_cap;
-    dc.done = ctx->done;
-    dc.vis_acc = ctx->vis_acc;
-    dc.part = ctx->part;
-    dc.part_cap = ctx->part_cap;
-    dc.gbar = ctx->gbar;
     dc.phase_ns = ctx->phase_ns;
-    dc.status = ctx->status;
     return dc;
 }
 
@@ -203,26 +181,38 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
         if ((1 << s) == cfg->c) t.c_log2 = s;
     t.kv_cap = cfg->capacity_tokens;
     t.scale = (float)(1.0 / std::sqrt((double)cfg->d));
+    Decode &d = ctx->scratch;
+    std::memset(&d, 0, sizeof d);
     for (int l = 1; l <= cfg->D; ++l) {
         t.node_cap[l - 1] = L.node_cap[l - 1];
         t.g[l - 1] = reinterpret_cast<float *>(ws + L.g_off[l - 1]);
         t.b[l - 1] = reinterpret_cast<float *>(ws + L.b_off[l - 1]);
         t.m[l - 1] = reinterpret_cast<float *>(ws + L.m_off[l - 1]);
-        ctx->kept_ids[l - 1] = reinterpret_cast<int32_t *>(ws + L.kid_off[l - 1]);
-        ctx->kept_mask[l - 1] = reinterpret_cast<uint8_t *>(ws + L.kmask_off[l - 1]);
+        d.kept_ids[l - 1] = reinterpret_cast<int32_t *>(ws + L.kid_off[l - 1]);
+        d.kept_mask[l - 1] = reinterpret_cast<uint8_t *>(ws + L.kmask_off[l - 1]);
+        d.slot_cap[l - 1] = L.slot_cap[l - 1];
     }
-    ctx->kept_cnt = reinterpret_cast<int32_t *>(ws + L.kcnt_off);
-    ctx->scores = reinterpret_cast<float *>(ws + L.scores_off);
-    ctx->slot_node = reinterpret_cast<int32_t *>(ws + L.snode_off);
-    ctx->score_cap = L.score_cap;
-    ctx->pmax = reinterpret_cast<float *>(ws + L.pmax_off);
-    ctx->pmax_cap = PMAX_CAP;
-    ctx->done = reinterpret_cast<uint32_t *>(ws + L.done_off);
-    ctx->vis_acc = reinterpret_cast<int64_t *>(ws + L.vis_off);
-    ctx->part = reinterpret_cast<float *>(ws + L.part_off);
-    ctx->part_cap = PART_CAP;
-    ctx->gbar = reinterpret_cast<unsigned *>(ws + L.gbar_off);
-    ctx->status = reinterpret_cast<int32_t *>(ws + L.status_off);
+    d.seg = reinterpret_cast<uint32_t *>(ws + L.seg_off);
+    d.hseg = reinterpret_cast<uint32_t *>(ws + L.hseg_off);
+    d.lvl = reinterpret_cast<int32_t *>(ws + L.lvl_off);
+    d.cur = reinterpret_cast<int32_t *>(ws + L.cur_off);
+    d.scores = reinterpret_cast<float *>(ws + L.scores_off);
+    d.slot_node = reinterpret_cast<int32_t *>(ws + L.snode_off);
+    d.slot_keep = reinterpret_cast<uint8_t *>(ws + L.skeep_off);
+    d.score_cap = L.score_cap;
+    d.tmax = reinterpret_cast<float *>(ws + L.tmax_off);
+    d.tcnt = reinterpret_cast<uint32_t *>(ws + L.tcnt_off);
+    d.tsum = reinterpret_cast<unsigned long long *>(ws + L.tsum_off);
+    d.hist_cnt = reinterpret_cast<uint32_t *>(ws + L.hcnt_off);
+    d.hist_mass = reinterpret_cast<unsigned long long *>(ws + L.hmass_off);
+    d.cand_w = reinterpret_cast<unsigned long long *>(ws + L.cw_off);
+    d.cand_slot = reinterpret_cast<uint32_t *>(ws + L.cs_off);
+    d.cand_cnt = reinterpret_cast<uint32_t *>(ws + L.ccnt_off);
+    d.ticket = reinterpret_cast<uint32_t *>(ws + L.ticket_off);
+    d.part = reinterpret_cast<float *>(ws + L.part_off);
+    d.part_cap = PART_CAP;
+    d.sync = reinterpret_cast<unsigned *>(ws + L.sync_off);
+    d.status = reinterpret_cast<int32_t *>(ws + L.status_off);
     ctx->scratch_begin = ws + L.scratch_off;
     ctx->scratch_bytes = L.total - L.scratch_off;
 
@@ -234,7 +224,7 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
     }
     ctx->attn_cta = std::min(PART_CAP, ctx->n_sm);  // one CTA per SM, one wave
     // the decode kernel: one resident CTA per SM (cooperative launch), a
-    // multiple of h_kv so that every KV head gets the same number of CTAs
+    // multiple of h_kv so that every KV head gets a team of the same size
     {
         Decode probe = make_decode(ctx);
         const int per_sm = decode_blocks_per_sm(probe);
@@ -242,7 +232,7 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
             delete ctx;
             return ZHA_ERR_CUDA;
         }
-        int n = std::min(std::min(ctx->n_sm, PART_CAP), PMAX_CAP * cfg->h_kv);
+        int n = std::min(ctx->n_sm, PART_CAP);
         n = std::max(1, n / cfg->h_kv) * cfg->h_kv;
         ctx->decode_cta = n;
     }
@@ -328,12 +318,14 @@ int zha_device_status(zha_ctx *ctx, int32_t *out_status, void *stream) {
     if (!ctx || !out_status) return ZHA_ERR_BAD_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     int32_t host = 0;
-    if (cudaMemcpyAsync(&host, ctx->status, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemsetAsync(ctx->status, 0, sizeof host, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+    if (cudaMemcpyAsync(&host, ctx->scratch.status, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemsetAsync(ctx->scratch.status, 0, sizeof host, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
         return ZHA_ERR_CUDA;
-    // after a timed-out wait the grid barrier words are reset for the next call
+    // after a timed-out wait the barrier words, tickets and boundary lists may
+    // be left raised: clear the decode scratch for the next call
     if (host == ZHA_ERR_TIMEOUT &&
-        (cudaMemsetAsync(ctx->gbar, 0, 16, s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess))
+        (cudaMemsetAsync(ctx->scratch_begin, 0, (size_t)ctx->scratch_bytes, s) != cudaSuccess ||
+         cudaStreamSynchronize(s) != cudaSuccess))
         return ZHA_ERR_CUDA;
     *out_status = host;
     return ZHA_OK;

@@ -14,8 +14,7 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_dense(const __grid_constant__ 
     __shared__ int s_last[64];
     const int warp = threadIdx.x >> 5;
     const int h_kv = a.t.h_kv, nb = gridDim.x, b = blockIdx.x;
-    if (threadIdx.x == 0) stage_map_init<true>(a, map);
-    __syncthreads();
+    stage_map_init<true>(a, map);
     attn_stages<KT, HD, G, true>(a, map, smem, b, nb);
     __threadfence();
     __syncthreads();
@@ -25,10 +24,9 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_dense(const __grid_constant__ 
         map.ctas(kh, nb, bf, bl);
         int last = 0;
         if (bl >= 0 && b >= bf && b <= bl) {
-            unsigned *tick = a.done + MAXD * h_kv + h_kv + kh;
-            const unsigned tk = atomicAdd(tick, 1u);
+            const unsigned tk = atomicAdd(a.ticket + kh, 1u);
             last = (tk == (unsigned)(bl - bf));
-            if (last) *tick = 0u;
+            if (last) a.ticket[kh] = 0u;
         }
         s_last[kh] = last;
     }
@@ -38,7 +36,7 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_dense(const __grid_constant__ 
         __threadfence();
         int bf, bl;
         map.ctas(kh, nb, bf, bl);
-        if (warp < ACW) combine_kvh<KT, HD, G>(a, kh, bf, bl + 1, false, reinterpret_cast<float *>(smem));
+        if (warp < ACW) combine_kvh<KT, HD, G>(a, map, kh, bf, bl + 1, false, reinterpret_cast<float *>(smem));
         __syncthreads();
     }
 }

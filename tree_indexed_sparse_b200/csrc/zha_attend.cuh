@@ -1,5 +1,5 @@
 // zha_attend.cuh -- exact attention over a token set, split over the CTAs of a
-// grid with a warp-specialised bulk-copy pipeline (sm_100a).
+// grid, fed by a warp-specialised bulk-copy pipeline (sm_100a).
 //
 // Attention ("ZHA 用树形稀疏注意力改造现有大模型", section "稀疏注意力为什么还会被索引拖慢":
 // the first token is always kept as the attention sink; rit.work article,
@@ -8,14 +8,25 @@
 //   o_h = sum_{i in T_h} softmax_i(q_h.k_i / sqrt(d)) v_i,
 //   T_h = tokens of the leaf chunks head h kept  U  {0},  fp32 accumulation.
 //
-// The union leaf list of each KV head (every leaf kept by any of its G query
-// heads, with the head bitmask) is flattened into stages of TT tokens; the
+// The union leaf list of each KV head (every leaf any of its G query heads
+// kept, with the head bitmask) is flattened into stages of TT tokens; the
 // grid's CTAs take contiguous ranges of stages over all KV heads.  In each CTA
-// one producer warp (warp 8) turns a stage into runs of contiguous K/V rows,
-// writes the per-token head masks, and issues one cp.async.bulk per run into
-// a ring of shared-memory stages guarded by mbarriers; warps 0-7 take TT/8
-// tokens each per stage.  Every K and V row crosses HBM once and serves all G
-// heads of its group (GQA sharing).  Each CTA leaves one partial (max, sum,
+// one producer warp (warp 8) maps a stage's tokens to K/V rows, writes the
+// per-token head masks and issues one cp.async.bulk per K row and per V row
+// into a ring of shared-memory stages guarded by mbarriers.  Rows land at a
+// padded stride (16 bytes past the row for bf16) so that the consumers'
+// 8-row matrix loads hit eight different bank groups.  Every K and V row
+// crosses HBM once and serves all G heads of its group (GQA sharing).
+//
+// Consumers, warps 0-7, 16 tokens each; stage j goes to warps 4(j%2)..+3:
+//   bf16 K/V: tensor cores (mma.sync m16n8k16, fp32 accumulate).  The queries
+//     and the probabilities are split into bf16 high and low parts (x = hi +
+//     lo to ~2^-16 relative), rows h and 8+h of the A operand, so that the
+//     fp32 accuracy of q.k and p.v is kept; K and V are exact in bf16.
+//       S^T[16 x 8 tokens] = [q_hi; q_lo] x K^T, s_h = S[h] + S[8+h]
+//       O[16 x d]         += [p_hi; p_lo] x V,  o_h = O[h] + O[8+h]
+//   fp32 K/V: fp32 FMA (each lane a column slice of every row).
+// Online softmax in the log2 domain.  Each CTA leaves one partial (max, sum,
 // output) per head per KV head it touched; combine_kvh merges them.
 #pragma once
 
@@ -31,48 +42,232 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr int ACW = 8;                         // consumer warps
 constexpr int A_THREADS = (ACW + 1) * 32;      // + one producer warp
 constexpr int TT = 64;                         // tokens per stage
-constexpr int TW = TT / ACW;                   // tokens per consumer warp per stage
-constexpr int LEAF_WIN = 2048;                 // leaf ids the producer keeps in shared memory
+constexpr int TW = 16;                         // tokens per consumer warp per stage
+constexpr int CW_STAGE = TT / TW;              // consumer warps per stage (4)
+constexpr int LEAF_WIN = 1024;                 // leaf ids the producer keeps in shared memory
+constexpr size_t STAGE_BUDGET = 176 * 1024;    // shared memory for the stage ring
+static_assert(CW_STAGE * 2 == ACW, "two halves of consumer warps alternate over stages");
 
 // One partial record: o[HD], max, sum, two pads (16-byte aligned records).
 template <int HD>
 constexpr int prec() { return HD + 4; }
 
-template <typename KT, int HD, int G>
-struct AttnCfg {
+// A stage holds TT tokens as NG groups of GR consecutive tokens.  Each group
+// is filled by bulk copies of whole runs of rows (one copy for a run of GR
+// contiguous rows); groups sit GS bytes apart, 16 bytes more than their rows,
+// so that row w of the eight groups falls in eight different bank groups.
+// Token slot t = GR*group + w sits at row_off(t); K groups first, then V.
+template <typename KT, int HD>
+struct StageCfg {
     static constexpr int ES = (int)sizeof(KT);
-    static constexpr int RB = HD * ES;            // row bytes
-    static constexpr int LPR = RB / 16;           // lanes per row (16-byte slices)
-    static constexpr int RPL = 32 / LPR;          // rows per warp-wide access
-    static constexpr int EPL = 16 / ES;           // elements per lane per row
-    static constexpr int RPB = TW / RPL;          // rows per lane per stage
-    static constexpr int NV = RPB * G;            // partial dots per lane
-    static constexpr int NVP = NV > LPR ? NV : LPR;  // padded to the reduce width
-    static constexpr int STAGE_BYTES = 2 * TT * RB;
-    static constexpr int STAGES = (128 * 1024) / STAGE_BYTES > 4 ? 4 : (128 * 1024) / STAGE_BYTES;
-    static_assert(LPR >= 1 && LPR <= 32 && RPB >= 1, "row layout");
-    static_assert(LPR % G == 0, "row slices must cover the heads");
+    static constexpr int RB = HD * ES;                      // row bytes
+    static constexpr int GR = 8;                            // rows per group
+    static constexpr int NG = TT / GR;                      // groups per stage
+    static constexpr int GS = GR * RB + 16;                 // group stride
+    static constexpr int HALF = NG * GS;                    // K part (V part follows)
+    static constexpr int STAGE_BYTES = 2 * HALF;
+    static constexpr int S0 = (int)(STAGE_BUDGET / STAGE_BYTES);
+    static constexpr int STAGES = S0 > 6 ? 6 : S0;
+    static_assert(STAGES >= 2, "stage ring");
+    static_assert(RB % 16 == 0 && GS % 16 == 0, "bulk copies need 16-byte aligned rows");
+    static_assert(NG == 8, "a matrix load takes one row from each of the eight groups");
+    static __device__ __forceinline__ int row_off(int t) { return (t >> 3) * GS + (t & 7) * RB; }
 };
 
 template <typename KT, int HD, int G>
 struct ASmem {
-    using C = AttnCfg<KT, HD, G>;
+    using C = StageCfg<KT, HD>;
     static constexpr size_t off_meta = (size_t)C::STAGES * C::STAGE_BYTES;
-    static constexpr size_t off_bar = off_meta + C::STAGES * TT;            // full[ST], empty[ST]
+    static constexpr size_t off_bar = (off_meta + C::STAGES * TT + 15) / 16 * 16;  // full[ST], empty[ST]
     static constexpr size_t off_abort = off_bar + 2 * C::STAGES * 8;
     static constexpr size_t off_merge = (off_abort + 16 + 15) / 16 * 16;
-    static constexpr size_t off_pw = off_merge + (size_t)ACW * G * (HD + 2) * 4;
-    static constexpr size_t off_win = off_pw + ACW * 32 * 4;               // producer's leaf-id window
+    static constexpr size_t off_pw = off_merge + (size_t)ACW * G * (HD + 2) * 4;   // FMA consumers' p slots
+    static constexpr size_t off_win = off_pw + (size_t)ACW * 32 * 4;                // producer's leaf-id window
     static constexpr size_t bytes = off_win + (size_t)LEAF_WIN * 5;
 };
 
+// ---- tensor-core consumer (bf16) ------------------------------------------
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// bf16x2 of (lo, hi): lo in the low half.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Split (x0, x1) into bf16 high parts and bf16 low parts (x - hi).
+__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    hi = pack_bf16(x0, x1);
+    lo = pack_bf16(x0 - bf_lo(hi), x1 - bf_hi(hi));
+}
+
+template <int HD, int G>
+struct MmaAttn {
+    static constexpr int KS = HD / 16;  // k-steps of q.k
+    static constexpr int NT = HD / 8;   // n-tiles of the output
+    uint32_t qa[KS][4];                 // A fragments of [q_hi; q_lo] (scaled, log2 domain)
+    float o[NT][4];                     // rows g (p_hi) and g+8 (p_lo), columns nt*8 + 2*c4 + {0,1}
+    float m;                            // running max of head g (replicated over the quad)
+    float l;                            // this thread's partial denominator
+
+    __device__ void init() {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+        m = -INFINITY;
+        l = 0.f;
+    }
+
+    // q rows of KV head kh into A fragments; thread (g = lane/4, c4 = lane%4)
+    // holds rows g (hi) and g+8 (lo) for g < G.
+    __device__ void load_q(const float *q, int kh, float qscale, int lane) {
+        const int g = lane >> 2, c4 = lane & 3;
+        const float *qh = q + (int64_t)(kh * G + (g < G ? g : 0)) * HD;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int d0 = ks * 16 + 2 * c4;
+            if (g < G) {
+                const float2 x01 = *reinterpret_cast<const float2 *>(qh + d0);
+                const float2 x89 = *reinterpret_cast<const float2 *>(qh + d0 + 8);
+                split_bf16(x01.x * qscale, x01.y * qscale, qa[ks][0], qa[ks][1]);
+                split_bf16(x89.x * qscale, x89.y * qscale, qa[ks][2], qa[ks][3]);
+            } else {
+                qa[ks][0] = qa[ks][1] = qa[ks][2] = qa[ks][3] = 0u;
+            }
+        }
+    }
+
+    // The 16 tokens of consumer slot wq of a stage: rows w1 = 2 wq and
+    // w2 = 2 wq + 1 of each of the 8 groups.  Column n of the first score tile
+    // is token 8n + w1, of the second 8n + w2; the same order is the k order
+    // of p.v.  sK/sV: the stage's K and V parts, msk: its 64 head masks.
+    template <typename SC>
+    __device__ void tokens(const unsigned char *sK, const unsigned char *sV, const uint8_t *msk, int wq, int lane) {
+        const int g = lane >> 2, c4 = lane & 3;
+        const int w1 = 2 * wq, w2 = 2 * wq + 1;
+        const int mi = lane >> 3, r = lane & 7;  // this lane addresses row r of matrix mi
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            // matrices: (w1, dims lo), (w1, dims hi), (w2, lo), (w2, hi) of a k-step
+            const int w = (mi >> 1) ? w2 : w1;
+            const uint32_t base = smem_addr(sK) + (uint32_t)(r * SC::GS + w * SC::RB + (mi & 1) * 16);
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t kb[4];
+                ldsm_x4(kb, base + ks * 32);
+                mma_bf16(s0, qa[ks], kb[0], kb[1]);
+                mma_bf16(s1, qa[ks], kb[2], kb[3]);
+            }
+        }
+        const uint32_t hb = g < G ? (1u << g) : 0u;
+        float x[4];
+        x[0] = (msk[16 * c4 + w1] & hb) ? s0[0] + s0[2] : -INFINITY;
+        x[1] = (msk[16 * c4 + 8 + w1] & hb) ? s0[1] + s0[3] : -INFINITY;
+        x[2] = (msk[16 * c4 + w2] & hb) ? s1[0] + s1[2] : -INFINITY;
+        x[3] = (msk[16 * c4 + 8 + w2] & hb) ? s1[1] + s1[3] : -INFINITY;
+        float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 1));
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
+        const float mn = fmaxf(m, mt);
+        if (mn > m && m != -INFINITY) {
+            const float alpha = exp2f(m - mn);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[nt][e] *= alpha;
+            l *= alpha;
+        }
+        m = mn;
+        float p[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) p[t] = (x[t] == -INFINITY) ? 0.f : exp2f(x[t] - mn);
+        l += (p[0] + p[1]) + (p[2] + p[3]);
+        uint32_t pa[4];
+        split_bf16(p[0], p[1], pa[0], pa[1]);
+        split_bf16(p[2], p[3], pa[2], pa[3]);
+        {
+            // matrices: (w1 tokens, dims lo), (w2, lo), (w1, hi), (w2, hi) of a column pair
+            const int w = (mi & 1) ? w2 : w1;
+            const uint32_t base = smem_addr(sV) + (uint32_t)(r * SC::GS + w * SC::RB + (mi >> 1) * 16);
+#pragma unroll
+            for (int i = 0; i < HD / 16; ++i) {
+                uint32_t vb[4];
+                ldsm_x4_t(vb, base + i * 32);
+                mma_bf16(o[2 * i], pa, vb[0], vb[1]);
+                mma_bf16(o[2 * i + 1], pa, vb[2], vb[3]);
+            }
+        }
+    }
+
+    // This warp's state into merge [G][HD+2] = (o, m, l).
+    __device__ void store(float *wsm, int lane) {
+        const int g = lane >> 2, c4 = lane & 3;
+        float lt = l;
+        lt += __shfl_xor_sync(FULL, lt, 1);
+        lt += __shfl_xor_sync(FULL, lt, 2);
+        if (g < G) {
+            float *row = wsm + g * (HD + 2);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int d = nt * 8 + 2 * c4;
+                row[d] = o[nt][0] + o[nt][2];
+                row[d + 1] = o[nt][1] + o[nt][3];
+            }
+            if (c4 == 0) {
+                row[HD] = m;
+                row[HD + 1] = lt;
+            }
+        }
+    }
+};
+
+// ---- fp32 FMA consumer -------------------------------------------------------
+
+template <int HD, int G>
+struct FmaCfg {
+    static constexpr int RB = HD * 4;             // row bytes
+    static constexpr int LPR = RB / 16;           // lanes per row (16-byte slices)
+    static constexpr int RPL = 32 / LPR;          // rows per warp-wide access
+    static constexpr int EPL = 4;                 // elements per lane per row
+    // tokens per pass: one partial per lane after the reduce (RPB * G <= LPR)
+    static constexpr int SUBT = (LPR / G) * RPL < TW ? (LPR / G) * RPL : TW;
+    static constexpr int RPB = SUBT / RPL;        // rows per lane per pass
+    static constexpr int NV = RPB * G;            // partial dots per lane
+    static constexpr int NVP = NV > LPR ? NV : LPR;  // padded to the reduce width
+    static_assert(LPR >= 1 && LPR <= 32 && RPB >= 1, "row layout");
+    static_assert(LPR % G == 0, "row slices must cover the heads");
+    static_assert(NV <= LPR && TW % SUBT == 0, "one partial per lane");
+};
+
 // Online-softmax state of one consumer warp for the G heads of one KV head.
-template <typename KT, int HD, int G>
-struct WarpAttn {
-    using C = AttnCfg<KT, HD, G>;
+template <int HD, int G>
+struct FmaAttn {
+    using C = FmaCfg<HD, G>;
     float m[G];          // running max (log2 domain), replicated over lanes
     float l;             // partial denominator of this lane's head (lane % G)
     float o[G][C::EPL];  // partial outputs of this lane's column slice
+    float qs[G][C::EPL];
 
     __device__ void init() {
 #pragma unroll
@@ -84,19 +279,39 @@ struct WarpAttn {
         l = 0.f;
     }
 
-    // The warp's TW tokens of one stage: K rows sK[t], V rows sV[t], head
-    // masks msk[t] (0 = not a token of any head) for t in [0, TW).
-    __device__ void tokens(const KT *sK, const KT *sV, const uint8_t *msk, const float (&qs)[G][C::EPL],
-                           float *pw, int lane) {
+    __device__ void load_q(const float *q, int kh, float qscale, int lane) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float *qh = q + (int64_t)(kh * G + h) * HD + (lane % C::LPR) * C::EPL;
+#pragma unroll
+            for (int e = 0; e < C::EPL; ++e) qs[h][e] = qh[e] * qscale;
+        }
+    }
+
+    // The warp's TW tokens (token i of consumer slot wq is stage slot
+    // 8 (i % 8) + 2 wq + i / 8), in passes of SUBT.
+    template <typename SC>
+    __device__ void tokens(const unsigned char *sK, const unsigned char *sV, const uint8_t *msk, int wq, float *pw,
+                           int lane) {
+#pragma unroll 1
+        for (int i0 = 0; i0 < TW; i0 += C::SUBT) pass<SC>(sK, sV, msk, wq, i0, pw, lane);
+    }
+
+    template <typename SC>
+    __device__ void pass(const unsigned char *sK, const unsigned char *sV, const uint8_t *msk, int wq, int i0, float *pw,
+                         int lane) {
         const int grp = lane / C::LPR, col = (lane % C::LPR) * C::EPL;
         float v[C::NVP];
         uint32_t mr[C::RPB];
+        int off[C::RPB];
 #pragma unroll
         for (int r = 0; r < C::RPB; ++r) {
-            const int t = r * C::RPL + grp;
+            const int i = i0 + r * C::RPL + grp;
+            const int t = 8 * (i & 7) + 2 * wq + (i >> 3);
+            off[r] = SC::row_off(t);
             mr[r] = msk[t];
             float k[C::EPL];
-            Vec<KT, C::EPL>::load(sK + t * HD + col, k);
+            Vec<float, C::EPL>::load(reinterpret_cast<const float *>(sK + off[r]) + col, k);
 #pragma unroll
             for (int h = 0; h < G; ++h) v[r * G + h] = mr[r] ? lane_dot<C::EPL>(qs[h], k) : 0.f;
         }
@@ -112,7 +327,7 @@ struct WarpAttn {
         const float s = ((m_me >> my_h) & 1u) ? v[0] : -INFINITY;
         float bmax = s;
 #pragma unroll
-        for (int off = G; off < 32; off <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(FULL, bmax, off));
+        for (int o2 = G; o2 < 32; o2 <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(FULL, bmax, o2));
         float alpha[G];
         float mnew_me = 0.f, alpha_me = 1.f;
         bool rescale = false;
@@ -142,7 +357,7 @@ struct WarpAttn {
         for (int r = 0; r < C::RPB; ++r) {
             if (!mr[r]) continue;
             float vv[C::EPL];
-            Vec<KT, C::EPL>::load(sV + (r * C::RPL + grp) * HD + col, vv);
+            Vec<float, C::EPL>::load(reinterpret_cast<const float *>(sV + off[r]) + col, vv);
 #pragma unroll
             for (int h = 0; h < G; ++h)
 #pragma unroll
@@ -150,9 +365,7 @@ struct WarpAttn {
         }
     }
 
-    // Fold the row groups and lanes; afterwards lanes [0, LPR) hold o for the
-    // columns [lane*EPL, ...) and every lane holds lsum[h].
-    __device__ void finish(float (&lsum)[G], int lane) {
+    __device__ void store(float *wsm, int lane) {
 #pragma unroll
         for (int off = C::LPR; off < 32; off <<= 1)
 #pragma unroll
@@ -162,32 +375,40 @@ struct WarpAttn {
         float lt = l;
 #pragma unroll
         for (int off = G; off < 32; off <<= 1) lt += __shfl_xor_sync(FULL, lt, off);
+        float lsum[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) lsum[h] = __shfl_sync(FULL, lt, h);
+        if (lane < C::LPR) {
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int e = 0; e < C::EPL; ++e) wsm[h * (HD + 2) + lane * C::EPL + e] = o[h][e];
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                wsm[h * (HD + 2) + HD] = m[h];
+                wsm[h * (HD + 2) + HD + 1] = lsum[h];
+            }
+        }
     }
 };
 
-// Merge the consumer warps' states (fixed order) into one partial per head
-// and store it at dst [G][HD+4] = (o[HD], m, l, pad).  Consumer threads only.
 template <typename KT, int HD, int G>
-__device__ __noinline__ void flush_partial(WarpAttn<KT, HD, G> &st, float *merge, float *dst, int warp, int lane) {
-    using C = AttnCfg<KT, HD, G>;
-    float lsum[G];
-    st.finish(lsum, lane);
-    float *wsm = merge + warp * G * (HD + 2);
-    if (lane < C::LPR) {
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int e = 0; e < C::EPL; ++e) wsm[h * (HD + 2) + lane * C::EPL + e] = st.o[h][e];
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            wsm[h * (HD + 2) + HD] = st.m[h];
-            wsm[h * (HD + 2) + HD + 1] = lsum[h];
-        }
-    }
+struct Consumer;
+template <int HD, int G>
+struct Consumer<uint16_t, HD, G> {
+    using T = MmaAttn<HD, G>;
+};
+template <int HD, int G>
+struct Consumer<float, HD, G> {
+    using T = FmaAttn<HD, G>;
+};
+
+// Merge the consumer warps' states (fixed order) into one partial per head
+// at dst [G][HD+4] = (o[HD], m, l, pad).  Consumer warps only.
+template <int HD, int G>
+__device__ __noinline__ void merge_partials(const float *merge, float *dst, int warp, int lane) {
     gsync();
 #pragma unroll 1
     for (int idx = warp * 32 + lane; idx < G * (HD + 2); idx += ACW * 32) {
@@ -209,11 +430,25 @@ __device__ __noinline__ void flush_partial(WarpAttn<KT, HD, G> &st, float *merge
     gsync();
 }
 
-// Stage space: KV head kh owns stages [pref[kh], pref[kh+1]).
+// x / c for token positions (< 2^32): a shift when c is a power of two.
+__device__ __forceinline__ uint32_t div_c(uint32_t x, int c, int clog) {
+    return clog >= 0 ? (x >> clog) : x / (uint32_t)c;
+}
+
+// ---- the stage map -------------------------------------------------------------
+
+// Stage space: KV head kh owns stages [pref[kh], pref[kh+1]).  For the routed
+// attention, KV head kh's kept leaves are the level-1 segments: T1[kh] ranks,
+// frontier S1[kh], per-rank kept counts with exclusive prefix
+// spref[soff[kh] .. soff[kh] + T1[kh]].
 struct StageMap {
     int64_t pref[65];
     int64_t cnt[64];   // union kept leaves per KV head (gather)
     int h_kv;
+    int T1[64];
+    int32_t S1[64];
+    int soff[65];
+    uint32_t spref[SEG_CAP + 65];
     __device__ void locate(int64_t i, int &kh, int64_t &st) const {
         kh = 0;
         while (kh + 1 < h_kv && i >= pref[kh + 1]) ++kh;
@@ -229,20 +464,73 @@ struct StageMap {
             bl = (int)((p1 * nb - 1) / U);
         }
     }
+    // Position in kept_ids[0] (KV head kh's rows) of kept leaf rank k.
+    __device__ int64_t leaf_at(int kh, int64_t k) const {
+        const uint32_t *p = spref + soff[kh];
+        const int T = T1[kh];
+        int lo = 0, hi = T - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if ((int64_t)p[mid] <= k) lo = mid;
+            else hi = mid - 1;
+        }
+        return (int64_t)S1[kh] * lo / T + (k - p[lo]);
+    }
 };
 
-// Fill the stage map (thread 0) -- call before attn_stages, then sync the CTA.
+// Fill the stage map; all threads of the CTA call it, then it is valid after
+// the __syncthreads inside.  Gather: the level-1 segments written by routing.
 template <bool DENSE>
 __device__ void stage_map_init(const Decode &a, StageMap &map) {
-    int64_t acc = 0;
-    map.h_kv = a.t.h_kv;
-    for (int kh = 0; kh < a.t.h_kv; ++kh) {
-        map.pref[kh] = acc;
-        map.cnt[kh] = DENSE ? 0 : __ldcg(a.kept_cnt + kh);
-        const int64_t ntok = DENSE ? a.t.n_tokens : map.cnt[kh] * a.t.c;
-        acc += (ntok + TT - 1) / TT;
+    const int h_kv = a.t.h_kv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        map.h_kv = h_kv;
+        int off = 0;
+        for (int kh = 0; kh < h_kv; ++kh) {
+            const int T = DENSE ? 1 : __ldcg(a.lvl + (int64_t)kh * 2);
+            map.T1[kh] = T;
+            map.S1[kh] = DENSE ? 0 : __ldcg(a.lvl + (int64_t)kh * 2 + 1);
+            map.soff[kh] = off;
+            off += T + 1;
+        }
+        map.soff[h_kv] = off;
     }
-    map.pref[a.t.h_kv] = acc;
+    __syncthreads();
+    if (!DENSE) {
+        // per KV head (one warp each): prefix of the level-1 per-rank counts
+        for (int kh = warp; kh < h_kv; kh += A_THREADS / 32) {
+            const int T = map.T1[kh];
+            const uint32_t *sg = a.seg + (int64_t)kh * SEG_CAP;
+            uint32_t carry = 0u;
+            for (int r0 = 0; r0 < T; r0 += 32) {
+                const uint32_t x = r0 + lane < T ? __ldcg(sg + r0 + lane) : 0u;
+                uint32_t v = x;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const uint32_t y = __shfl_up_sync(FULL, v, off);
+                    if (lane >= off) v += y;
+                }
+                if (r0 + lane < T) map.spref[map.soff[kh] + r0 + lane + 1] = carry + v;
+                carry += __shfl_sync(FULL, v, 31);
+            }
+            if (lane == 0) {
+                map.spref[map.soff[kh]] = 0u;
+                map.cnt[kh] = carry;
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int64_t acc = 0;
+        for (int kh = 0; kh < h_kv; ++kh) {
+            map.pref[kh] = acc;
+            const int64_t ntok = DENSE ? a.t.n_tokens : map.cnt[kh] * a.t.c;
+            acc += (ntok + TT - 1) / TT;
+        }
+        map.pref[h_kv] = acc;
+    }
+    __syncthreads();
 }
 
 // This CTA's share of the attention: stages [U*b/nb, U*(b+1)/nb).  Leaves one
@@ -250,21 +538,21 @@ __device__ void stage_map_init(const Decode &a, StageMap &map) {
 // touch).  All 9 warps of the CTA call it.
 template <typename KT, int HD, int G, bool DENSE>
 __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char *smem, int b, int nb) {
-    using C = AttnCfg<KT, HD, G>;
+    using C = StageCfg<KT, HD>;
     using SM = ASmem<KT, HD, G>;
+    constexpr int ST = C::STAGES, RB = C::RB, GR = C::GR;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int h_kv = a.t.h_kv, c = a.t.c;
+    const int h_kv = a.t.h_kv, c = a.t.c, clog = a.t.c_log2;
     uint8_t *meta = smem + SM::off_meta;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::off_bar);
-    uint64_t *empty = full + C::STAGES;
+    uint64_t *empty = full + ST;
     volatile int *abort = reinterpret_cast<volatile int *>(smem + SM::off_abort);
     float *merge = reinterpret_cast<float *>(smem + SM::off_merge);
-    float *pw = reinterpret_cast<float *>(smem + SM::off_pw) + warp * 32;
     const int64_t N = a.t.n_tokens;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < ST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], ACW);
+            mbar_init(&empty[s], CW_STAGE);
         }
         *abort = 0;
         mbar_init_fence();
@@ -282,8 +570,8 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
         int64_t win_k0 = 0;
         int64_t issued = 0;
         for (int64_t j = 0; j < n; ++j) {
-            const int slot = (int)(j % C::STAGES);
-            const uint32_t round = (uint32_t)(j / C::STAGES);
+            const int slot = (int)(j % ST);
+            const uint32_t round = (uint32_t)(j / ST);
             if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1u, abort)) {
                 set_status(a.status, ZHA_TIMEOUT_CODE);
                 *abort = 1;
@@ -292,119 +580,157 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
             int kh;
             int64_t st;
             map.locate(u0 + j, kh, st);
-            const KT *Kh = reinterpret_cast<const KT *>(a.t.K) + (int64_t)kh * a.t.kv_cap * HD;
-            const KT *Vh = reinterpret_cast<const KT *>(a.t.V) + (int64_t)kh * a.t.kv_cap * HD;
+            const unsigned char *Kh = reinterpret_cast<const unsigned char *>(a.t.K) + (int64_t)kh * a.t.kv_cap * C::RB;
+            const unsigned char *Vh = reinterpret_cast<const unsigned char *>(a.t.V) + (int64_t)kh * a.t.kv_cap * C::RB;
             unsigned char *sK = smem + (size_t)slot * C::STAGE_BYTES;
-            unsigned char *sV = sK + TT * C::RB;
             uint8_t *mt = meta + slot * TT;
             const int64_t t0 = st * TT;
-            // this lane's runs: rows of one leaf piece each (gather; a stage
-            // touches at most TT/c + 2 <= 34 leaves, so at most 2 per lane),
-            // or the whole stage (dense, lane 0)
-            int64_t row0[2] = {0, 0};
-            int dst0[2] = {0, 0}, nrows[2] = {0, 0};
-            if (DENSE) {
-                if (lane == 0) {
-                    row0[0] = t0;
-                    nrows[0] = (int)min((int64_t)TT, N - t0);
-                }
-                for (int t = lane; t < TT; t += 32) mt[t] = (t0 + t < N) ? 0xffu : 0u;
-            } else {
-                const int64_t L = map.cnt[kh];
-                const int64_t kbase = (int64_t)kh * a.t.node_cap[0];
-                const int64_t kf = t0 / c;
-                const int64_t kl = min(L - 1, (t0 + TT - 1) / c);
-                if (kh != win_kh || kl >= win_k0 + LEAF_WIN) {
-                    // refill the window from leaf kf on: independent coalesced loads
+            int64_t L = 0;
+            if (!DENSE) {
+                L = map.cnt[kh];
+                const int64_t kf = (int64_t)div_c((uint32_t)t0, c, clog);
+                const int64_t kl = min(L - 1, (int64_t)div_c((uint32_t)(t0 + TT - 1), c, clog));
+                if (kh != win_kh || kl >= win_k0 + LEAF_WIN || kf < win_k0) {
+                    // refill the window from leaf rank kf up to the last leaf
+                    // this CTA needs in this KV head: independent loads
+                    const int64_t jl = min(u1, map.pref[kh + 1]) - 1 - map.pref[kh];
+                    const int64_t klast = min(L - 1, (int64_t)div_c((uint32_t)(jl * TT + TT - 1), c, clog));
+                    const int nwin = (int)min((int64_t)LEAF_WIN, klast - kf + 1);
                     win_kh = kh;
                     win_k0 = kf;
-                    for (int i = lane; i < LEAF_WIN && kf + i < L; i += 32) {
-                        win_ids[i] = __ldcg(a.kept_ids[0] + kbase + kf + i);
-                        win_msk[i] = __ldcg(a.kept_mask[0] + kbase + kf + i);
+                    const int64_t kbase = (int64_t)kh * a.slot_cap[0];
+#pragma unroll 4
+                    for (int i = lane; i < nwin; i += 32) {
+                        const int64_t at = kbase + map.leaf_at(kh, kf + i);
+                        win_ids[i] = __ldcg(a.kept_ids[0] + at);
+                        win_msk[i] = __ldcg(a.kept_mask[0] + at);
                     }
                     __syncwarp();
                 }
-                int q = 0;
-                for (int64_t k = kf + lane; k * c < t0 + TT && k < L && q < 2; k += 32, ++q) {
-                    const int64_t a0 = max(t0, k * c), a1 = min(t0 + TT, (k + 1) * c);
-                    const int64_t leaf = win_ids[k - win_k0];
-                    const int64_t r0 = leaf * c + (a0 - k * c);
-                    const int64_t r1 = min(leaf * c + (a1 - k * c), N);
-                    const uint32_t mk = win_msk[k - win_k0];
-                    for (int64_t t = a0; t < a1; ++t) mt[t - t0] = (leaf * c + (t - k * c) < N) ? (uint8_t)mk : 0;
-                    row0[q] = r0;
-                    dst0[q] = (int)(a0 - t0);
-                    nrows[q] = (int)max((int64_t)0, r1 - r0);
-                }
-                // tokens past the end of the list
-                const int64_t tend = L * c;
-                for (int t = lane; t < TT; t += 32)
-                    if (t0 + t >= tend) mt[t] = 0;
             }
-            uint32_t bytes = (uint32_t)(nrows[0] + nrows[1]) * C::RB * 2;
+            // lane gi < 8: K rows of group gi; lane 8 + gi: V rows of group gi
+            const int gi = lane & 7;
+            const bool act = lane < 16;
+            const bool isV = lane >= 8;
+            int64_t row[GR];
+            uint32_t nvalid = 0u;
+#pragma unroll
+            for (int w = 0; w < GR; ++w) {
+                const int64_t u = t0 + gi * GR + w;
+                int64_t r = -1;
+                uint32_t mk = 0u;
+                if (act) {
+                    if (DENSE) {
+                        if (u < N) {
+                            r = u;
+                            mk = 0xffu;
+                        }
+                    } else {
+                        const int64_t k = div_c((uint32_t)u, c, clog);
+                        if (k < L) {
+                            const int64_t rr = (int64_t)win_ids[k - win_k0] * c + (u - k * c);
+                            if (rr < N) {
+                                r = rr;
+                                mk = win_msk[k - win_k0];
+                            }
+                        }
+                    }
+                }
+                row[w] = r;
+                nvalid += r >= 0;
+                if (act && !isV) mt[gi * GR + w] = (uint8_t)mk;
+            }
+            uint32_t bytes = nvalid * RB;
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) bytes += __shfl_xor_sync(FULL, bytes, off);
+            unsigned char *dst = sK + (isV ? C::HALF : 0) + gi * C::GS;
+            // rows without a token: zeros, so that 0 * row stays 0 in the
+            // products (the fence orders these generic stores before later
+            // bulk copies into the same rows)
+            if (act && nvalid < (uint32_t)GR) {
+#pragma unroll
+                for (int w = 0; w < GR; ++w) {
+                    if (row[w] >= 0) continue;
+                    uint4 *z = reinterpret_cast<uint4 *>(dst + w * RB);
+                    for (int i = 0; i < RB / 16; ++i) z[i] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
             __syncwarp();
+            if (act) {
+                // one copy per run of consecutive rows
+                const unsigned char *src = isV ? Vh : Kh;
+                int w0 = 0;
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                if (nrows[q] > 0) {
-                    bulk_g2s(sK + (size_t)dst0[q] * C::RB, Kh + row0[q] * HD, (uint32_t)nrows[q] * C::RB, &full[slot]);
-                    bulk_g2s(sV + (size_t)dst0[q] * C::RB, Vh + row0[q] * HD, (uint32_t)nrows[q] * C::RB, &full[slot]);
+                for (int w = 1; w <= GR; ++w) {
+                    const bool brk = (w == GR) || row[w] < 0 || row[w - 1] < 0 || row[w] != row[w - 1] + 1;
+                    if (brk) {
+                        if (row[w0] >= 0)
+                            bulk_g2s(dst + w0 * RB, src + row[w0] * RB, (uint32_t)((w - w0) * RB), &full[slot]);
+                        w0 = w;
+                    }
                 }
             }
             issued = j + 1;
         }
         // on an abort, wait (bounded) for the copies already in flight
         if (*abort) {
-            for (int64_t j = (issued > C::STAGES ? issued - C::STAGES : 0); j < issued; ++j)
-                mbar_wait(&full[j % C::STAGES], (uint32_t)((j / C::STAGES) & 1), nullptr);
+            for (int64_t j = (issued > ST ? issued - ST : 0); j < issued; ++j)
+                mbar_wait(&full[j % ST], (uint32_t)((j / ST) & 1), nullptr);
         }
     } else {
         // ---------------- consumer warps ----------------
         for (int idx = warp * 32 + lane; idx < h_kv * G; idx += ACW * 32)
             a.part[(((int64_t)b * h_kv + idx / G) * G + idx % G) * prec<HD>() + HD] = -INFINITY;
         gsync();
-        WarpAttn<KT, HD, G> st;
+        typename Consumer<KT, HD, G>::T st;
         st.init();
-        float qs[G][C::EPL];
+        const int half = warp / CW_STAGE, wq = warp % CW_STAGE;
+        const float qscale = a.t.scale * LOG2E;
         int kh_cur = -1;
         for (int64_t j = 0; j < n; ++j) {
-            const int slot = (int)(j % C::STAGES);
-            const uint32_t round = (uint32_t)(j / C::STAGES);
-            // every consumer warp takes the same branches below whatever the
-            // wait returned, so the named barriers inside the flushes match
+            int kh;
+            int64_t stage_in_kh;
+            map.locate(u0 + j, kh, stage_in_kh);
+            if (kh != kh_cur) {
+                // every consumer warp sees every stage's KV head, so the
+                // named barriers inside the flushes match
+                if (kh_cur >= 0) {
+                    st.store(merge + warp * G * (HD + 2), lane);
+                    merge_partials<HD, G>(merge, a.part + ((int64_t)b * h_kv + kh_cur) * G * prec<HD>(), warp, lane);
+                }
+                kh_cur = kh;
+                st.init();
+                st.load_q(a.q, kh, qscale, lane);
+            }
+            if ((int)(j & 1) != half) continue;
+            const int slot = (int)(j % ST);
+            const uint32_t round = (uint32_t)(j / ST);
             const bool ok = mbar_wait(&full[slot], round & 1u, abort);
             if (!ok) {
                 set_status(a.status, ZHA_TIMEOUT_CODE);
                 *abort = 1;
             }
-            int kh;
-            int64_t stage_in_kh;
-            map.locate(u0 + j, kh, stage_in_kh);
-            if (kh != kh_cur) {
-                if (kh_cur >= 0)
-                    flush_partial<KT, HD, G>(st, merge, a.part + ((int64_t)b * h_kv + kh_cur) * G * prec<HD>(), warp,
-                                             lane);
-                kh_cur = kh;
-                st.init();
-                const float qscale = a.t.scale * LOG2E;
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float *qh = a.q + (int64_t)(kh * G + h) * HD + (lane % C::LPR) * C::EPL;
-#pragma unroll
-                    for (int e = 0; e < C::EPL; ++e) qs[h][e] = qh[e] * qscale;
+            const unsigned char *sK = smem + (size_t)slot * C::STAGE_BYTES;
+            const unsigned char *sV = sK + C::HALF;
+            const uint8_t *msk = meta + slot * TT;
+            if (ok) {
+                if constexpr (sizeof(KT) == 2) {
+                    st.template tokens<C>(sK, sV, msk, wq, lane);
+                } else {
+                    float *pws = reinterpret_cast<float *>(smem + SM::off_pw) + warp * 32;
+                    st.template tokens<C>(sK, sV, msk, wq, pws, lane);
                 }
             }
-            const KT *sK = reinterpret_cast<const KT *>(smem + (size_t)slot * C::STAGE_BYTES) + warp * TW * HD;
-            const KT *sV = sK + TT * HD;
-            if (ok) st.tokens(sK, sV, meta + slot * TT + warp * TW, qs, pw, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[slot]);
         }
-        if (kh_cur >= 0)
-            flush_partial<KT, HD, G>(st, merge, a.part + ((int64_t)b * h_kv + kh_cur) * G * prec<HD>(), warp, lane);
+        if (kh_cur >= 0) {
+            st.store(merge + warp * G * (HD + 2), lane);
+            merge_partials<HD, G>(merge, a.part + ((int64_t)b * h_kv + kh_cur) * G * prec<HD>(), warp, lane);
+        }
     }
 }
 
@@ -414,7 +740,8 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
 // each thread sweeps four output columns over the partials in a fixed order.
 // `sm` holds 2*G*(b1-b0) + 4*G floats.
 template <typename KT, int HD, int G>
-__device__ __noinline__ void combine_kvh(const Decode &a, int kh, int b0, int b1, bool gather, float *sm) {
+__device__ __noinline__ void combine_kvh(const Decode &a, const StageMap &map, int kh, int b0, int b1, bool gather,
+                                         float *sm) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n = max(0, b1 - b0);
     float *wv = sm;              // [G][n]: max, then weight
@@ -435,9 +762,11 @@ __device__ __noinline__ void combine_kvh(const Decode &a, int kh, int b0, int b1
         const int h = warp;
         bool add = false;
         if (gather) {
-            const int64_t kbase = (int64_t)kh * a.t.node_cap[0];
-            const bool has0 = __ldcg(a.kept_cnt + kh) > 0 && __ldcg(a.kept_ids[0] + kbase) == 0 &&
-                              ((__ldcg(a.kept_mask[0] + kbase) >> h) & 1u);
+            bool has0 = false;
+            if (map.cnt[kh] > 0) {
+                const int64_t at = (int64_t)kh * a.slot_cap[0] + map.leaf_at(kh, 0);
+                has0 = __ldcg(a.kept_ids[0] + at) == 0 && ((__ldcg(a.kept_mask[0] + at) >> h) & 1u);
+            }
             add = !has0;
         }
         float s0 = -INFINITY;

@@ -1,70 +1,31 @@
 // zha_decode.cu -- one decoded token for every query head, in one persistent
 // cooperative kernel (sm_100a): every routing level, then the routed
-// attention, with bounded grid barriers between the phases.
+// attention.
 //
 // Routing ("ZHA 用树形稀疏注意力改造现有大模型", section "稀疏注意力为什么还会被索引拖慢":
 // score the top nodes, keep the smallest set whose estimated mass reaches p,
 // expand only their children, repeat down to the raw entries; "Zyphra
 // 分层注意力（ZHA）…", section "机制拆解：树形索引如何高效筛选长上下文"):
-//   level D .. 1:
-//     a frontier small enough for one SM (<= SMALL_BYTES of summaries per KV
-//     head) is scored and cut by the CTA that owns its KV head, with no
-//     fan-in; a larger one is scored by every CTA of the grid (each KV head
-//     gets gridDim/h_kv CTAs), then, after a grid barrier, cut by its owner;
-//     a grid barrier ends the level.
-//   attention over the kept leaves plus the sink token, split over every CTA
-//   (zha_attend.cuh), a grid barrier, and the owner CTAs merge the partials.
+//   the grid's CTAs are split into h_kv teams of nbk = gridDim / h_kv CTAs,
+//   one per KV head, which route independently, level D .. 1:
+//     a frontier whose summaries fit SMALL_BYTES is scored and cut by the
+//     team's first CTA alone, with no inter-CTA barrier, and so are the small
+//     levels that follow it; the rest of the team waits at one team barrier;
+//     a larger frontier is split over the whole team (zha_route.cuh).
+//   a grid barrier ends the routing; every CTA then writes the leaf lists and
+//   traces of its own segments while the attention over the kept leaves plus
+//   the sink token runs split over every CTA (zha_attend.cuh); the last CTA
+//   to finish a KV head's stages merges its partials (ticket).
 // The grid is one CTA per SM, launched cooperatively so that the barriers
 // cannot deadlock; every barrier wait is bounded by a clock budget, after
-// which the kernel records ZHA_ERR_TIMEOUT, raises a shared abort flag and
-// returns.
+// which the kernel records ZHA_ERR_TIMEOUT, raises the abort word and leaves.
 #include "zha_attend.cuh"
 #include "zha_route.cuh"
-#include "zha_select.cuh"
+#include "zha_sync.cuh"
 
 namespace zha {
 
 constexpr int64_t SMALL_BYTES = 256 * 1024;
-
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Grid barrier over all CTAs (cooperative launch: all are resident).  gbar[0]
-// counts arrivals, gbar[1] is the generation, gbar[2] the abort flag.
-__device__ __noinline__ bool grid_sync(const Decode &a) {
-    __shared__ int s_ok;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        unsigned *count = a.gbar, *gen = a.gbar + 1, *abortf = a.gbar + 2;
-        const unsigned g = ld_acquire_u32(gen);
-        __threadfence();
-        int ok = 1;
-        if (atomicAdd(count, 1u) == gridDim.x - 1) {
-            atomicExch(count, 0u);
-            __threadfence();
-            atomicAdd(gen, 1u);
-        } else {
-            const long long t0 = clock64();
-            while (ld_acquire_u32(gen) == g) {
-                if (ld_acquire_u32(abortf)) { ok = 0; break; }
-                if (clock64() - t0 > WAIT_BUDGET_CYCLES) {
-                    set_status(a.status, ZHA_TIMEOUT_CODE);
-                    atomicExch(abortf, 1u);
-                    ok = 0;
-                    break;
-                }
-                __nanosleep(32);
-            }
-        }
-        __threadfence();
-        s_ok = ok && !ld_acquire_u32(abortf);
-    }
-    __syncthreads();
-    return s_ok != 0;
-}
 
 __device__ __forceinline__ void stamp(const Decode &a, int i) {
     if (a.phase_ns && blockIdx.x == 0 && threadIdx.x == 0) {
@@ -74,51 +35,200 @@ __device__ __forceinline__ void stamp(const Decode &a, int i) {
     }
 }
 
+// Per-head lists of one CTA's segments: level-1 leaf ids (leaf_idx, n_leaf)
+// and, when requested, every level's kept ids (trace).  Positions come from
+// the lower ranks' per-head counts.  Warps 0-7.
+template <int G>
+__device__ __noinline__ void write_lists(const Decode &a, int kh, int tr) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int D = a.t.D;
+    for (int task = warp; task < D * G; task += GT / 32) {
+        const int l = 1 + task / G, h = task % G;
+        const bool leaf = (l == 1);
+        const bool tr_on = a.trace_ids != nullptr;
+        if (!leaf && !tr_on) continue;
+        const int32_t *lv = lvl_ptr(a, l, kh);
+        const int T = __ldcg(lv);
+        const int64_t S = __ldcg(lv + 1);
+        const int hq = kh * G + h;
+        const uint32_t *hs = hseg_ptr(a, l, kh);
+        // lower ranks' counts and the total of head h
+        uint32_t before = 0u, total = 0u;
+        for (int r = lane; r < T; r += 32) {
+            const uint32_t x = __ldcg(hs + (int64_t)r * G + h);
+            total += x;
+            if (r < tr) before += x;
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+            before += __shfl_xor_sync(FULL, before, off);
+            total += __shfl_xor_sync(FULL, total, off);
+        }
+        if (tr == 0 && lane == 0) {
+            if (leaf && a.n_leaf) a.n_leaf[hq] = (int32_t)total;
+            if (leaf && a.leaf_idx && total > (uint32_t)a.leaf_cap) set_status(a.status, ZHA_CAPACITY_CODE);
+            if (tr_on) {
+                a.trace_cnt[(int64_t)(l - 1) * a.t.h_q + hq] = (int32_t)total;
+                if (total > (uint32_t)a.trace_cap) set_status(a.status, ZHA_CAPACITY_CODE);
+            }
+        }
+        if (tr >= T) continue;
+        const uint32_t n = __ldcg(seg_ptr(a, l, kh) + tr);
+        const int64_t src = (int64_t)kh * a.slot_cap[l - 1] + seg_start(S, T, tr);
+        const int32_t *ids = a.kept_ids[l - 1] + src;
+        const uint8_t *msk = a.kept_mask[l - 1] + src;
+        uint32_t pos = before;
+        for (uint32_t i0 = 0; i0 < n; i0 += 32) {
+            const uint32_t i = i0 + lane;
+            const bool mine = i < n && ((__ldcg(msk + i) >> h) & 1u);
+            const unsigned bal = __ballot_sync(FULL, mine);
+            if (mine) {
+                const uint32_t p = pos + __popc(bal & ((1u << lane) - 1u));
+                const int32_t id = __ldcg(ids + i);
+                if (leaf && a.leaf_idx && p < (uint32_t)a.leaf_cap) a.leaf_idx[(int64_t)hq * a.leaf_cap + p] = id;
+                if (tr_on && p < (uint32_t)a.trace_cap)
+                    a.trace_ids[((int64_t)(l - 1) * a.t.h_q + hq) * a.trace_cap + p] = id;
+            }
+            pos += __popc(bal);
+        }
+    }
+}
+
+// All routing levels of KV head kh as rank tr of a team of T CTAs.  Warps 0-7.
+template <int HD, int R, int G>
+__device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, unsigned char *smem, TeamSync &ts) {
+    using SM = RouteSmem<G>;
+    uint32_t *pref = reinterpret_cast<uint32_t *>(smem + SM::off_pref);
+    uint32_t *scratch = reinterpret_cast<uint32_t *>(smem + SM::off_misc) + 8;
+    const int D = a.t.D;
+    const int64_t node_bytes = (int64_t)R * (HD + 1) * 4;
+    int64_t vis[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) vis[h] = 0;
+    int l = D;
+    int Tp = 1;       // team size and frontier size of level l + 1
+    int64_t Sp = 0;
+    int64_t S = a.t.n_level[D - 1];
+    auto small = [&](int64_t s) { return T == 1 || (s <= SOLO_MAX && s * node_bytes <= SMALL_BYTES); };
+#pragma unroll 1
+    while (l >= 1) {
+        if (small(S)) {
+            if (tr == 0) {
+                TeamSync solo = ts;
+                solo.T = 1;
+#pragma unroll 1
+                for (;;) {
+                    uint32_t F[G];
+                    route_level<HD, R, G>(a, l, kh, 1, 0, S, Tp, Sp, smem, solo, F);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) vis[h] += F[h];
+                    Tp = 1;
+                    Sp = S;
+                    --l;
+                    if (l < 1) break;
+                    S = load_segments(a, l + 1, kh, 1, pref, scratch) * a.t.c;
+                    if (!small(S)) break;
+                }
+                if (threadIdx.x == 0) a.cur[kh] = l;
+            }
+            if (T > 1) {
+                if (!ts.sync()) return false;
+                l = __ldcg(a.cur + kh);
+                if (l >= 1) {
+                    const int32_t *lv = lvl_ptr(a, l + 1, kh);
+                    Tp = __ldcg(lv);
+                    Sp = __ldcg(lv + 1);
+                    S = load_segments(a, l + 1, kh, Tp, pref, scratch) * a.t.c;
+                }
+            }
+        } else {
+            uint32_t F[G];
+            if (!route_level<HD, R, G>(a, l, kh, T, tr, S, Tp, Sp, smem, ts, F)) return false;
+#pragma unroll
+            for (int h = 0; h < G; ++h) vis[h] += F[h];
+            Tp = T;
+            Sp = S;
+            --l;
+            if (l >= 1) S = load_segments(a, l + 1, kh, Tp, pref, scratch) * a.t.c;
+        }
+    }
+    if (tr == 0 && threadIdx.x < G && a.visited) {
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+            if (h == (int)threadIdx.x) a.visited[kh * G + h] = vis[h];
+    }
+    return true;
+}
+
 template <typename KT, int HD, int R, int G>
 __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__ Decode a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ StageMap map;
+    __shared__ int s_flag;
+    __shared__ int s_last[64];
     const int warp = threadIdx.x >> 5;
     const int nb = gridDim.x, b = blockIdx.x;
     const int h_kv = a.t.h_kv;
-    const int nbk = nb / h_kv;  // CTAs per KV head when a level is scored by the whole grid
-    float *wsm = reinterpret_cast<float *>(smem);
+    const int nbk = nb / h_kv;  // CTAs per KV head team
+    unsigned *words = a.sync;
+    unsigned *abortw = words + h_kv + 2;
     stamp(a, 0);
-    for (int l = a.t.D; l >= 1; --l) {
-        int64_t smax = 0;
-        for (int kh = 0; kh < h_kv; ++kh) smax = max(smax, frontier_size(a, l, kh));
-        const bool small = smax * (int64_t)(R * HD * 4) <= SMALL_BYTES;
-        if (small) {
-            if (b < h_kv && warp < ACW) {
-                const int64_t S = frontier_size(a, l, b);
-                route_score<HD, R, G>(a, l, b, 0, 1, S, wsm);
-                select_kvh<HD, R, G>(a, l, b, S, 1, smem);
-            }
-        } else {
-            if (b < nbk * h_kv && warp < ACW)
-                route_score<HD, R, G>(a, l, b % h_kv, b / h_kv, nbk, frontier_size(a, l, b % h_kv), wsm);
-            if (!grid_sync(a)) return;
-            if (b < h_kv && warp < ACW) select_kvh<HD, R, G>(a, l, b, frontier_size(a, l, b), nbk, smem);
-        }
-        if (!grid_sync(a)) return;
-        stamp(a, a.t.D - l + 1);
+    const bool router = b < nbk * h_kv;
+    const int kh = router ? b / nbk : 0, tr = router ? b % nbk : 0;
+    bool ok = true;
+    if (router && warp < ACW) {
+        TeamSync ts{words + kh, abortw, a.status, &s_flag, nbk, 0u};
+        ok = route_kvh<HD, R, G>(a, kh, tr, nbk, smem, ts);
     }
-    if (threadIdx.x == 0) stage_map_init<false>(a, map);
+    __shared__ int s_ok;
+    if (threadIdx.x == 0) s_ok = 1;
     __syncthreads();
-    attn_stages<KT, HD, G, false>(a, map, smem, b, nb);
-    if (!grid_sync(a)) return;
-    stamp(a, a.t.D + 1);
-    if (b < h_kv && warp < ACW) {
-        int bf, bl;
-        map.ctas(b, nb, bf, bl);
-        combine_kvh<KT, HD, G>(a, b, bf, bl + 1, true, reinterpret_cast<float *>(smem));
+    if (!ok && threadIdx.x == 0) s_ok = 0;
+    __syncthreads();
+    unsigned gepoch = 0;
+    if (s_ok && grid_barrier(words + h_kv, nb, gepoch, abortw, a.status, &s_flag)) {
+        stamp(a, a.t.D);
+        stage_map_init<false>(a, map);
+        if (router && warp < ACW) write_lists<G>(a, kh, tr);
+        attn_stages<KT, HD, G, false>(a, map, smem, b, nb);
+        stamp(a, a.t.D + 1);
+        // the last CTA to finish a KV head's stages merges its partials
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x < h_kv) {
+            const int k = threadIdx.x;
+            int bf, bl;
+            map.ctas(k, nb, bf, bl);
+            int last = 0;
+            if (bl >= 0 && b >= bf && b <= bl) {
+                const unsigned tk = atomicAdd(a.ticket + k, 1u);
+                last = (tk == (unsigned)(bl - bf));
+                if (last) a.ticket[k] = 0u;
+            }
+            s_last[k] = last;
+        }
+        __syncthreads();
+        for (int k = 0; k < h_kv; ++k) {
+            if (!s_last[k]) continue;
+            __threadfence();
+            int bf, bl;
+            map.ctas(k, nb, bf, bl);
+            if (warp < ACW) combine_kvh<KT, HD, G>(a, map, k, bf, bl + 1, true, reinterpret_cast<float *>(smem));
+            __syncthreads();
+        }
+        stamp(a, a.t.D + 2);
     }
-    stamp(a, a.t.D + 2);
+    kernel_exit(words, h_kv + 3, h_kv + 1);
+}
+
+template <typename KT, int HD, int R, int G>
+static size_t decode_smem() {
+    return std::max(RouteSmem<G>::bytes, ASmem<KT, HD, G>::bytes);
 }
 
 template <typename KT, int HD, int R, int G>
 static cudaError_t decode_impl(const Decode &dc, int n_cta, cudaStream_t s) {
-    const size_t smem = std::max(SelectSmem<G>::bytes, ASmem<KT, HD, G>::bytes);
+    const size_t smem = decode_smem<KT, HD, R, G>();
     static size_t attr = 0;
     if (smem > attr) {
         cudaError_t err =
@@ -134,7 +244,7 @@ static cudaError_t decode_impl(const Decode &dc, int n_cta, cudaStream_t s) {
 
 template <typename KT, int HD, int R, int G>
 static int decode_occupancy() {
-    const size_t smem = std::max(SelectSmem<G>::bytes, ASmem<KT, HD, G>::bytes);
+    const size_t smem = decode_smem<KT, HD, R, G>();
     static size_t attr = 0;
     if (smem > attr) {
         if (cudaFuncSetAttribute(k_decode<KT, HD, R, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=

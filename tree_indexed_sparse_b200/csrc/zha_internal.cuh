@@ -7,13 +7,11 @@
 namespace zha {
 
 constexpr int MAXD = 16;          // deepest tree supported
-constexpr int ROUTE_THREADS = 256;
-constexpr int ATTN_THREADS = 256;
 constexpr int BUILD_THREADS = 256;
-constexpr int NB = 1024;          // coarse top-p buckets per frontier
-constexpr float BUCKETS_PER_UNIT = 32.f;  // bucket width 1/32 of a log-mass unit
-constexpr int CAND_MAX = 256;     // boundary candidates ranked exactly
-constexpr int STAGE_BYTES = 128 * 1024;   // frontier scores staged in shared memory
+constexpr int NB = 1024;          // top-p buckets per round
+constexpr int CAND_MAX = 1024;    // boundary candidates ranked exactly per head
+constexpr int SEG_CAP = 256;      // most CTAs in one KV head's team (grid <= 256 CTAs)
+constexpr int HIST_ROUNDS = 3;    // bucket widths 1/32, 1/32768, 1/2^25 of a log-mass unit
 
 // Summary store of every level (pointers for KV head 0; head stride is
 // node_cap[l] rows).  g: [node][R][d], b and m: [node][R].
@@ -33,24 +31,39 @@ struct Tree {
     float scale;                  // 1/sqrt(d)
 };
 
-// Decode scratch plus outputs of one zha_decode call.
+// Decode scratch plus outputs of one zha_decode call.  Routing state is kept
+// per level l (index l-1) and KV head in "segment" layout: the CTA of team rank
+// r that cut level l writes its kept nodes, ascending, at the start of its own
+// slot range [S*r/T, S*(r+1)/T) of the level's frontier (S slots, T ranks);
+// seg[] holds how many.  Concatenating the segments in rank order gives the
+// kept nodes in ascending id order.
 struct Decode {
     Tree t;
     const float *q;               // [h_q][d]
     float p;
-    int32_t *kept_ids[MAXD];      // level l: [h_kv][node_cap[l-1]] ascending union kept ids
-    uint8_t *kept_mask[MAXD];     // head bitmask per kept id
-    int32_t *kept_cnt;            // [MAXD][h_kv]
-    float *scores;                // [h_kv][score_cap][G]; -inf where the head does not need the slot
-    int32_t *slot_node;           // [h_kv][score_cap] node id of each frontier slot
+    int32_t *kept_ids[MAXD];      // [h_kv][slot_cap[l-1]] kept node ids (segments)
+    uint8_t *kept_mask[MAXD];     // [h_kv][slot_cap[l-1]] heads that kept the node
+    int64_t slot_cap[MAXD];       // frontier slots per KV head at level l
+    uint32_t *seg;                // [MAXD][h_kv][SEG_CAP] kept nodes per team rank
+    uint32_t *hseg;               // [MAXD][h_kv][SEG_CAP][G] kept nodes per team rank and head
+    int32_t *lvl;                 // [MAXD][h_kv][2] team size and frontier size of level l
+    int32_t *cur;                 // [h_kv] next level after a one-CTA run
+    float *scores;                // [h_kv][score_cap][G] scores when a rank's slots overflow shared memory
+    int32_t *slot_node;           // [h_kv][score_cap] node of each slot (same case)
+    uint8_t *slot_keep;           // [h_kv][score_cap] kept heads of each slot (same case)
     int64_t score_cap;
-    float *pmax;                  // [h_kv][pmax_cap][G]
-    int pmax_cap;
-    uint32_t *done;               // [MAXD][h_kv] level tickets, then [h_kv] attention tickets
-    int64_t *vis_acc;             // [h_q]
+    float *tmax;                  // [h_kv][SEG_CAP][G] per-rank maximum estimate
+    uint32_t *tcnt;               // [h_kv][SEG_CAP][G] per-rank frontier count
+    unsigned long long *tsum;     // [h_kv][SEG_CAP][G] per-rank boundary mass (slot-order cut)
+    uint32_t *hist_cnt;           // [h_kv][HIST_ROUNDS][G][NB]
+    unsigned long long *hist_mass;  // [h_kv][HIST_ROUNDS][G][NB]
+    unsigned long long *cand_w;   // [h_kv][G][CAND_MAX]
+    uint32_t *cand_slot;          // [h_kv][G][CAND_MAX]
+    uint32_t *cand_cnt;           // [h_kv][G]
+    uint32_t *ticket;             // [h_kv] merge tickets of the attention partials
     float *part;                  // attention partials [part_cap][h_kv][G][d+4]
     int part_cap;
-    unsigned *gbar;               // grid barrier: arrivals, generation, abort flag
+    unsigned *sync;               // barrier words, see zha_sync.cuh
     int64_t *phase_ns;            // nullable: globaltimer stamps per decode phase
     int32_t *status;
     float *out;

@@ -1,70 +1,301 @@
-// zha_route.cuh -- frontier scoring of one routing level (sm_100a).
+// zha_route.cuh -- one routing level of one KV head, cut by a team of CTAs.
 //
-// Routing ("ZHA 用树形稀疏注意力改造现有大模型", section "稀疏注意力为什么还会被索引拖慢";
-// "Zyphra 分层注意力（ZHA）…", section "机制拆解：树形索引如何高效筛选长上下文"): at
-// each level the query scores every node of the frontier -- every top node,
-// then the children of the nodes kept one level up -- with the tangent-plane
-// estimate est(q) = max_j (b_j + q.g_j / sqrt(d)).
+// Routing ("ZHA 用树形稀疏注意力改造现有大模型", section "稀疏注意力为什么还会被索引拖慢":
+// the query scores the top nodes, keeps the smallest set whose estimated mass
+// reaches p and expands only their children, down to the raw entries;
+// "Zyphra 分层注意力（ZHA）…", section "机制拆解：树形索引如何高效筛选长上下文").
+// For query head h with frontier F_h at a level: est_n = max_j (b_j + q.g_j/√d)
+// (the tangent-plane estimate), P_n = softmax over F_h, order by P descending
+// with ties to the lower node id, keep the shortest prefix whose cumulative P
+// reaches p; p >= 1 keeps every node.
 //
 // The frontier of KV head kh is the union over its G query heads: the
-// children of every node kept by any head, each carrying the bitmask of heads
-// that kept its parent.  A node's summary is read from HBM once and scored for
-// all G heads (a [R x d] x [d x G] product per node): lane l of a warp owns
-// the d-slice [l*VEC, (l+1)*VEC) of every g row, forms the G*R partial dot
-// products per node, and a reduce-scatter leaves each lane whole sums.
+// children of every node any head kept one level up, each with the bitmask of
+// the heads that kept its parent.  It is split into T contiguous slot ranges,
+// one per CTA of the team (T = 1 for a frontier small enough for one SM).
+// Each CTA streams its nodes' summary rows once (a register prefetch ring per
+// warp) and scores each node for all G heads.  Masses are w = exp(est - M_h)
+// in 2^-40 fixed point (integer sums are exact and do not depend on the order
+// of addition), M_h the maximum over the frontier, and the target is
+// ceil(p * Z_h) of the total Z_h.  Every decision is deterministic:
+//   one CTA, at most SOLO_MAX slots: each slot is ranked exactly against all
+//   others by (estimate descending, node id ascending) and kept while the
+//   mass before it is below the target;
+//   otherwise, round 0 histograms mass and count over buckets of width 1/32
+//   of a log-mass unit below M_h; the bucket where the cumulative mass first
+//   reaches the target holds the cut: every node of a lower bucket is kept,
+//   none of a higher one; when that bucket holds more than CAND_MAX nodes,
+//   rounds 1 and 2 split it 1024-fold again (widths 1/32768 and 1/2^25); the
+//   nodes of the final bucket are ranked exactly as above; a final bucket
+//   still larger than CAND_MAX holds estimates within 2^-25 of each other and
+//   is taken in node-id order.
+// Team barriers separate: the maxima (A), each histogram round (B), the
+// boundary lists (C) and the written segments (D).
+//
+// Code size matters here as much as arithmetic: every function runs once per
+// level on little data, so cold instruction fetch dominates unless the code is
+// short.  Loops that are not hot are kept rolled.
+//
+// Every function here is called by threads 0-255 of a CTA (warps 0-7) and
+// synchronises them with the named barrier of gsync().
 #pragma once
 
 #include "zha_device.cuh"
 #include "zha_internal.cuh"
+#include "zha_sync.cuh"
 
 namespace zha {
 
-template <int HD, int R, int G>
-struct RouteCfg {
-    static constexpr int VEC = HD / 32;
-    static constexpr int NPW = (G * R >= 32) ? 1 : 32 / (G * R);  // nodes per warp pass
-    static constexpr int V = NPW * G * R;                          // partial dots per lane
-    static constexpr int K = V / 32;                               // sums per lane after reduce-scatter
+constexpr int LOC_CAP = 2048;          // local slots held in shared memory
+constexpr int PWIN = LOC_CAP / 2 + 2;  // parents of LOC_CAP consecutive slots (c >= 2)
+constexpr int SOLO_MAX = GT;           // exact ranking for one-CTA levels up to this many slots
+
+enum CutMode : int { CUT_OPEN = 0, CUT_RANK = 1, CUT_ORDER = 2, CUT_ALL = 3, CUT_NONE = 4 };
+
+struct HeadCut {
+    unsigned long long Z, target, C;  // total mass, target, mass strictly above the bucket path
+    float M;                          // maximum estimate
+    uint32_t F;                       // frontier nodes of this head
+    uint32_t nfin;                    // nodes in the last fixed bucket
+    int32_t path[HIST_ROUNDS];        // bucket fixed in each round
+    int rounds;                       // rounds fixed so far
+    int mode;
 };
 
-// Node id, validity and head mask of frontier slot s at level l of KV head kh.
+constexpr int CH_BYTES = 64 * 1024;   // one scoring chunk of summary rows (two are staged)
+constexpr int CH_SLOTS_MAX = 256;     // slots in a chunk at most (R = 1, d = 64)
+constexpr int CH_ROWS_MAX = 256;      // summary rows in a chunk at most (d = 64)
+
+// Shared memory of the routing.  The two scoring chunks share their space
+// with the histogram and boundary lists, which are used only after scoring.
 template <int G>
-__device__ __forceinline__ void slot_info(const Decode &a, int l, int kh, bool top, int64_t S, int64_t s,
-                                          int32_t &node, bool &ok, uint32_t &msk) {
-    if (s >= S) {
-        node = 0; ok = false; msk = 0;
-        return;
+struct RouteSmem {
+    static constexpr size_t off_sc = 0;                                   // [LOC_CAP][G] f32
+    static constexpr size_t off_node = off_sc + (size_t)LOC_CAP * G * 4;  // [LOC_CAP] i32
+    static constexpr size_t off_keep = off_node + (size_t)LOC_CAP * 4;    // [LOC_CAP] u8
+    static constexpr size_t off_u = off_keep + LOC_CAP;                   // union: chunks | cut scratch
+    static constexpr size_t off_chunk = off_u;                            // [2][CH_BYTES]
+    static constexpr size_t off_hc = off_u;                               // [G][NB] u32
+    static constexpr size_t off_hm = off_hc + (size_t)G * NB * 4;         // [G][NB] u64 (solo: [SOLO_MAX][G] masses)
+    static constexpr size_t off_cw = off_hm + (size_t)G * NB * 8;         // [G][CAND_MAX] u64
+    static constexpr size_t off_cs = off_cw + (size_t)G * CAND_MAX * 8;   // [G][CAND_MAX] u32
+    static constexpr size_t off_own = off_cs + (size_t)G * CAND_MAX * 4;  // [G*CAND_MAX] u32
+    static constexpr size_t u_end = off_own + (size_t)G * CAND_MAX * 4 > off_u + 2 * (size_t)CH_BYTES
+                                        ? off_own + (size_t)G * CAND_MAX * 4
+                                        : off_u + 2 * (size_t)CH_BYTES;
+    static constexpr size_t off_pid = u_end;                              // [PWIN] i32
+    static constexpr size_t off_pmk = off_pid + (size_t)PWIN * 4;         // [PWIN] u8
+    static constexpr size_t off_pref = (off_pmk + PWIN + 15) / 16 * 16;   // [SEG_CAP + 1] u32
+    static constexpr size_t off_cut = (off_pref + (SEG_CAP + 1) * 4 + 15) / 16 * 16;  // [G] HeadCut
+    static constexpr size_t off_wm = (off_cut + G * sizeof(HeadCut) + 15) / 16 * 16;  // [8][G] f32 warp maxima
+    static constexpr size_t off_wc = off_wm + 8 * G * 4;                  // [8][G] u32 warp counts
+    static constexpr size_t off_red = (off_wc + 8 * G * 4 + 15) / 16 * 16; // [GT] u64
+    static constexpr size_t off_bar = off_red + GT * 8;                   // [2] u64 chunk barriers
+    static constexpr size_t off_cnode = off_bar + 16;                     // [2][CH_SLOTS_MAX] i32
+    static constexpr size_t off_cmask = off_cnode + 2 * CH_SLOTS_MAX * 4; // [2][CH_SLOTS_MAX] u8
+    static constexpr size_t off_rowres = off_cmask + 2 * CH_SLOTS_MAX;    // [CH_ROWS_MAX][G] f32
+    static constexpr size_t off_misc = off_rowres + (size_t)CH_ROWS_MAX * G * 4;  // u32 counters
+    static constexpr size_t bytes = off_misc + 64;
+    static_assert(SOLO_MAX * G * 8 <= G * NB * 8, "solo masses fit the histogram area");
+    static_assert(off_u % 16 == 0, "bulk copies land on 16-byte boundaries");
+};
+
+// One level of one KV head as seen by one CTA of its team.
+struct Level {
+    int l, kh, T, tr;
+    bool top;
+    int64_t S, s0, n;       // frontier slots, first local slot, local slots
+    int Tp;                 // team size of the parent level
+    int64_t Sp;             // frontier size of the parent level
+    float *sc;              // [n][G] local scores (shared memory, or global when n > LOC_CAP)
+    int32_t *node;          // [n] node of each local slot (-1: no such child)
+    uint8_t *keep;          // [n] heads that keep the slot
+};
+
+struct TeamSync {
+    unsigned *ctr;
+    unsigned *abortw;
+    int32_t *status;
+    int *flag;
+    int T;
+    unsigned epoch;
+    __device__ __forceinline__ bool sync() {
+        if (T == 1) {
+            gsync();
+            return true;
+        }
+        return team_barrier(ctr, T, epoch, abortw, status, flag);
     }
-    if (top) {
-        node = (int32_t)s; ok = true; msk = (1u << G) - 1u;
-        return;
-    }
-    const int c = a.t.c;
-    const int64_t k = a.t.c_log2 >= 0 ? (s >> a.t.c_log2) : s / c;
-    const int o = (int)(s - k * c);
-    const int64_t pbase = (int64_t)kh * a.t.node_cap[l];
-    const int32_t pid = __ldcg(a.kept_ids[l] + pbase + k);
-    node = pid * c + o;
-    ok = node < a.t.n_level[l - 1];
-    msk = ok ? (uint32_t)__ldcg(a.kept_mask[l] + pbase + k) : 0u;
+};
+
+// ---- level bookkeeping ---------------------------------------------------
+
+__device__ __forceinline__ uint32_t *seg_ptr(const Decode &a, int l, int kh) {
+    return a.seg + ((int64_t)(l - 1) * a.t.h_kv + kh) * SEG_CAP;
+}
+__device__ __forceinline__ uint32_t *hseg_ptr(const Decode &a, int l, int kh) {
+    return a.hseg + ((int64_t)(l - 1) * a.t.h_kv + kh) * SEG_CAP * a.t.G;
+}
+__device__ __forceinline__ int32_t *lvl_ptr(const Decode &a, int l, int kh) {
+    return a.lvl + ((int64_t)(l - 1) * a.t.h_kv + kh) * 2;
+}
+// First slot of team rank r's range of a level with S slots and T ranks.
+__device__ __forceinline__ int64_t seg_start(int64_t S, int T, int r) { return S * r / T; }
+
+// Exclusive prefix of level l's per-rank kept counts (T ranks, known to the
+// caller) into pref[0..T] (shared); returns the total.  `scratch`: 8 shared
+// uint32.
+__device__ __noinline__ int64_t load_segments(const Decode &a, int l, int kh, int T, uint32_t *pref,
+                                              uint32_t *scratch) {
+    const uint32_t *sg = seg_ptr(a, l, kh);
+    const uint32_t x = (int)threadIdx.x < T ? __ldcg(sg + threadIdx.x) : 0u;
+    uint32_t total;
+    const uint32_t incl = g_scan_u32(x, scratch, &total);
+    if ((int)threadIdx.x < T) pref[threadIdx.x + 1] = incl;
+    if (threadIdx.x == 0) pref[0] = 0u;
+    gsync();
+    return total;
 }
 
-// Frontier size of KV head kh at level l (every top node, or c children per
-// node kept one level up).
-__device__ __forceinline__ int64_t frontier_size(const Decode &a, int l, int kh) {
-    return (l == a.t.D) ? (int64_t)a.t.n_level[l - 1] : (int64_t)a.t.c * __ldcg(a.kept_cnt + l * a.t.h_kv + kh);
+// Team rank holding kept rank k of a level (pref: exclusive prefix, T ranks).
+__device__ __forceinline__ int seg_find(const uint32_t *pref, int T, int64_t k) {
+    int lo = 0, hi = T - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)pref[mid] <= k) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
 }
 
-// Score the slots of KV head kh handled by this CTA (warp-strided over
-// `nwarps` warps of `ncta` CTAs; this is CTA `bi`), write the scores (-inf
-// where a head does not need the slot) and node ids, and the CTA's maximum
-// per head to pmax[kh][bi].  Called by warps 0-7; `wsm` holds 256 floats.
+// Parents of slots [c0, c1) of level L (ranks [k0, k1]) into the window.
+__device__ __noinline__ void load_parents(const Decode &a, const Level &L, int64_t c0, int64_t c1, const uint32_t *pref,
+                                          int32_t *pid, uint8_t *pmk, int64_t &k0) {
+    const int c = a.t.c, clog = a.t.c_log2;
+    k0 = clog >= 0 ? (c0 >> clog) : c0 / c;
+    const int64_t k1 = clog >= 0 ? ((c1 - 1) >> clog) : (c1 - 1) / c;
+    const int lp = L.l + 1;
+    const int64_t pbase = (int64_t)L.kh * a.slot_cap[lp - 1];
+#pragma unroll 1
+    for (int64_t k = k0 + threadIdx.x; k <= k1; k += GT) {
+        const int r = seg_find(pref, L.Tp, k);
+        const int64_t at = pbase + seg_start(L.Sp, L.Tp, r) + (k - pref[r]);
+        pid[k - k0] = __ldcg(a.kept_ids[lp - 1] + at);
+        pmk[k - k0] = __ldcg(a.kept_mask[lp - 1] + at);
+    }
+}
+
+// ---- scoring ----------------------------------------------------------------
+
+// Sums of the G per-lane partial dots over the warp.  G = 4: a reduce-scatter
+// (xor 16, 8) then a butterfly (xor 4, 2, 1) leaves lane l with the sum of
+// head (l >> 3) & 3.  G = 1: a butterfly.  One fixed order each.
+template <int G>
+__device__ __forceinline__ float head_sum(const float (&v)[G], int lane) {
+    if constexpr (G == 4) {
+        const bool up = (lane & 16) != 0;
+        float s0 = up ? v[2] : v[0], s1 = up ? v[3] : v[1];
+        const float t0 = up ? v[0] : v[2], t1 = up ? v[1] : v[3];
+        s0 += __shfl_xor_sync(FULL, t0, 16);
+        s1 += __shfl_xor_sync(FULL, t1, 16);
+        const bool up8 = (lane & 8) != 0;
+        float k = up8 ? s1 : s0;
+        k += __shfl_xor_sync(FULL, up8 ? s0 : s1, 8);
+        k += __shfl_xor_sync(FULL, k, 4);
+        k += __shfl_xor_sync(FULL, k, 2);
+        k += __shfl_xor_sync(FULL, k, 1);
+        return k;
+    } else {
+        float k = v[0];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) k += __shfl_xor_sync(FULL, k, off);
+        return k;
+    }
+}
+
+template <int HD, int R>
+struct ScoreChunk {
+    static constexpr int NODE_BYTES = R * HD * 4;       // g rows of one node
+    static constexpr int SLOTS = CH_BYTES / NODE_BYTES;  // slots per chunk
+    static constexpr int ROWS = SLOTS * R;               // summary rows per chunk
+    static constexpr int RPW = ROWS / 8;                 // rows per warp per chunk
+    static_assert(SLOTS >= 1 && SLOTS <= CH_SLOTS_MAX && ROWS <= CH_ROWS_MAX, "chunk shape");
+    static_assert(RPW >= 1 && RPW <= 32, "one plane offset per lane");
+};
+
+// Warp 0: node ids of the slots of chunk k and bulk copies of their g rows
+// (one copy per run of consecutive nodes) into chunk buffer k & 1.
 template <int HD, int R, int G>
-__device__ void route_score(const Decode &a, int l, int kh, int bi, int ncta, int64_t S, float *wsm) {
-    using C = RouteCfg<HD, R, G>;
-    constexpr int VEC = C::VEC, NPW = C::NPW, V = C::V, K = C::K;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const bool top = (l == a.t.D);
+__device__ __noinline__ void chunk_issue(const Level &L, int64_t c0, int64_t c1, int64_t k0, int k, const int32_t *pid,
+                                            const uint8_t *pmk, const float *gb, int c, int clog, int32_t nl,
+                                            unsigned char *bufs, uint64_t *bars, int32_t *cnode, uint8_t *cmask,
+                                            int lane) {
+    using C = ScoreChunk<HD, R>;
+    const int buf = k & 1;
+    const int64_t sb = c0 + (int64_t)k * C::SLOTS;
+    const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
+    int32_t *cn = cnode + buf * CH_SLOTS_MAX;
+    uint8_t *cm = cmask + buf * CH_SLOTS_MAX;
+    uint32_t nvalid = 0u;
+#pragma unroll 1
+    for (int i = lane; i < ns; i += 32) {
+        const int s = (int)(sb + i);
+        int nd = s;
+        uint32_t mk = (1u << G) - 1u;
+        if (!L.top) {
+            const int kk = clog >= 0 ? (s >> clog) : (int)((uint32_t)s / (uint32_t)c);
+            nd = pid[kk - (int)k0] * c + (s - kk * c);
+            mk = pmk[kk - (int)k0];
+        }
+        const bool ok = nd < nl;
+        cn[i] = ok ? nd : -1;
+        cm[i] = ok ? (uint8_t)mk : 0;
+        nvalid += ok;
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) nvalid += __shfl_xor_sync(FULL, nvalid, off);
+    __syncwarp();
+    if (lane == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(&bars[buf], nvalid * (uint32_t)C::NODE_BYTES);
+    }
+    __syncwarp();
+    unsigned char *dst = bufs + (size_t)buf * CH_BYTES;
+#pragma unroll 1
+    for (int i = lane; i < ns; i += 32) {
+        const int nd = cn[i];
+        if (nd < 0 || (i > 0 && cn[i - 1] >= 0 && cn[i - 1] + 1 == nd)) continue;
+        int len = 1;
+        while (i + len < ns && cn[i + len] == nd + len) ++len;
+        bulk_g2s(dst + (size_t)i * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES),
+                 &bars[buf]);
+    }
+}
+
+// Score local slots [c0, c1) (global slot ids) of level L.  The slots go in
+// chunks of ScoreChunk::SLOTS through two shared-memory buffers: warp 0
+// bulk-copies the g rows of chunk k + 2 while all warps score chunk k from
+// shared memory (warp w takes rows w, w + 8, ... of the chunk; the plane
+// offsets b of its rows are loaded before the chunk lands).  Parent window:
+// ranks [k0, ...) in pid/pmk.  Writes L.sc / L.node at (s - L.s0) and folds
+// the maxima and counts per head into wm/wc[warp][h].
+template <int HD, int R, int G>
+__device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64_t c0, int64_t c1, int64_t k0,
+                                          const int32_t *pid, const uint8_t *pmk, unsigned char *smem, float *wm,
+                                          uint32_t *wc) {
+    static_assert(G == 1 || G == 4, "query heads per KV head");
+    using C = ScoreChunk<HD, R>;
+    using SM = RouteSmem<G>;
+    constexpr int VEC = HD / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int myh = G == 4 ? ((lane >> 3) & 3) : 0;
+    const bool writer = G == 4 ? ((lane & 7) == 0) : (lane == 0);
+    const int kh = L.kh, l = L.l;
+    unsigned char *bufs = smem + SM::off_chunk;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::off_bar);
+    int32_t *cnode = reinterpret_cast<int32_t *>(smem + SM::off_cnode);
+    uint8_t *cmask = smem + SM::off_cmask;
+    float *rowres = reinterpret_cast<float *>(smem + SM::off_rowres);
     float qs[G][VEC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -75,61 +306,661 @@ __device__ void route_score(const Decode &a, int l, int kh, int bi, int ncta, in
     const int64_t cap = a.t.node_cap[l - 1];
     const float *gb = a.t.g[l - 1] + (int64_t)kh * cap * R * HD;
     const float *bb = a.t.b[l - 1] + (int64_t)kh * cap * R;
-    float *scores = a.scores + (int64_t)kh * a.score_cap * G;
-    int32_t *snode = a.slot_node + (int64_t)kh * a.score_cap;
-    const int idx0 = lane * K;
-    const int my_i = idx0 / (G * R), my_h = (idx0 / R) % G, my_j0 = idx0 % R;
-    float lmax = -INFINITY;
-    const int nwarps = GT / 32;
-    for (int64_t grp = (int64_t)bi * nwarps + warp; grp * NPW < S; grp += (int64_t)ncta * nwarps) {
-        float v[V];
-#pragma unroll
-        for (int i = 0; i < NPW; ++i) {
-            int32_t node; bool ok; uint32_t msk;
-            slot_info<G>(a, l, kh, top, S, grp * NPW + i, node, ok, msk);
-#pragma unroll
-            for (int j = 0; j < R; ++j) {
-                float gs[VEC];
-                if (ok) {
-                    Vec<float, VEC>::load(gb + ((int64_t)node * R + j) * HD + lane * VEC, gs);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < VEC; ++e) gs[e] = 0.f;
-                }
-#pragma unroll
-                for (int h = 0; h < G; ++h) v[(i * G + h) * R + j] = lane_dot<VEC>(qs[h], gs);
+    const int c = a.t.c, clog = a.t.c_log2;
+    const int32_t nl = a.t.n_level[l - 1];
+    const int nch = (int)((c1 - c0 + C::SLOTS - 1) / C::SLOTS);
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_init_fence();
+    }
+    gsync();
+    if (warp == 0) {
+        chunk_issue<HD, R, G>(L, c0, c1, k0, 0, pid, pmk, gb, c, clog, nl, bufs, bars, cnode, cmask, lane);
+        if (nch > 1)
+            chunk_issue<HD, R, G>(L, c0, c1, k0, 1, pid, pmk, gb, c, clog, nl, bufs, bars, cnode, cmask, lane);
+    }
+    gsync();
+    float mloc = -INFINITY;  // this thread's head is tid % G throughout
+    uint32_t cloc = 0u;
+#pragma unroll 1
+    for (int k = 0; k < nch; ++k) {
+        const int buf = k & 1;
+        const int64_t sb = c0 + (int64_t)k * C::SLOTS;
+        const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
+        const int nrows = ns * R;
+        const int32_t *cn = cnode + buf * CH_SLOTS_MAX;
+        const uint8_t *cm = cmask + buf * CH_SLOTS_MAX;
+        // plane offsets of this warp's rows, one per lane
+        float bl = 0.f;
+        {
+            const int r = warp + 8 * lane;
+            if (lane < C::RPW && r < nrows) {
+                const int nd = cn[r / R];
+                if (nd >= 0) bl = __ldg(bb + (size_t)nd * R + r % R);
             }
         }
-        reduce_scatter<V>(v, lane);
-        const int64_t s = grp * NPW + my_i;
-        int32_t node; bool ok; uint32_t msk;
-        slot_info<G>(a, l, kh, top, S, s, node, ok, msk);
-        float est = -INFINITY;
-        if (ok) {
+        if (!mbar_wait(&bars[buf], (uint32_t)((k >> 1) & 1), nullptr)) set_status(a.status, ZHA_TIMEOUT_CODE);
+        const float *cb = reinterpret_cast<const float *>(bufs + (size_t)buf * CH_BYTES);
+#pragma unroll 2
+        for (int t = 0; t < C::RPW; ++t) {
+            const int r = warp + 8 * t;
+            if (r >= nrows) break;
+            float gs[VEC];
+            Vec<float, VEC>::load(cb + (size_t)r * HD + lane * VEC, gs);
+            float v[G];
 #pragma unroll
-            for (int t = 0; t < K; ++t) est = fmaxf(est, __ldg(bb + (int64_t)node * R + my_j0 + t) + v[t]);
+            for (int h = 0; h < G; ++h) v[h] = lane_dot<VEC>(qs[h], gs);
+            const float sum = head_sum<G>(v, lane);
+            const float b = __shfl_sync(FULL, bl, t);
+            if (writer) rowres[r * G + myh] = b + sum;
         }
+        gsync();
+        // rows -> slots: est = max over the node's planes
+#pragma unroll 1
+        for (int idx = tid; idx < ns * G; idx += GT) {
+            const int i = idx / G, h = idx % G;
+            const int nd = cn[i];
+            float est = -INFINITY;
+#pragma unroll 1
+            for (int j = 0; j < R; ++j) est = fmaxf(est, rowres[(i * R + j) * G + h]);
+            const bool need = nd >= 0 && ((cm[i] >> h) & 1u);
+            const int64_t s = sb + i - L.s0;
+            L.sc[s * G + h] = need ? est : -INFINITY;
+            if (h == 0) L.node[s] = nd;
+            if (need) {
+                mloc = fmaxf(mloc, est);
+                cloc += 1u;
+            }
+        }
+        gsync();
+        if (warp == 0 && k + 2 < nch)
+            chunk_issue<HD, R, G>(L, c0, c1, k0, k + 2, pid, pmk, gb, c, clog, nl, bufs, bars, cnode, cmask, lane);
+    }
+    // per-warp maxima and counts of each head (lanes with equal tid % G)
 #pragma unroll
-        for (int off = 1; off < R / K; off <<= 1) est = fmaxf(est, __shfl_xor_sync(FULL, est, off));
-        if (my_j0 == 0 && s < S) {
-            const bool need = ok && ((msk >> my_h) & 1u);
-            scores[s * G + my_h] = need ? est : -INFINITY;
-            if (need) lmax = fmaxf(lmax, est);
-            if (my_h == 0) snode[s] = ok ? node : -1;
+    for (int off = G; off < 32; off <<= 1) {
+        mloc = fmaxf(mloc, __shfl_xor_sync(FULL, mloc, off));
+        cloc += __shfl_xor_sync(FULL, cloc, off);
+    }
+    if (lane < G) {
+        wm[warp * G + lane] = fmaxf(wm[warp * G + lane], mloc);
+        wc[warp * G + lane] += cloc;
+    }
+    gsync();
+}
+
+// ---- the cut ------------------------------------------------------------------
+
+__device__ __forceinline__ int round_bucket(const HeadCut &H, float e, int r) {
+    const float x = H.M - e;
+    float f;
+    if (r == 0) {
+        f = x * 32.f;
+    } else if (r == 1) {
+        f = x * 32768.f - 1024.f * (float)H.path[0];
+    } else {
+        f = x * 33554432.f - 1024.f * (1024.f * (float)H.path[0] + (float)H.path[1]);
+    }
+    if (!(f >= 0.f)) return 0;
+    return f < (float)(NB - 1) ? (int)f : NB - 1;
+}
+
+// -1: above the fixed path (kept), 1: below (dropped), 0: on it.
+__device__ __forceinline__ int path_cmp(const HeadCut &H, float e, int rounds) {
+#pragma unroll 1
+    for (int r = 0; r < rounds; ++r) {
+        const int b = round_bucket(H, e, r);
+        if (b < H.path[r]) return -1;
+        if (b > H.path[r]) return 1;
+    }
+    return 0;
+}
+
+__device__ __forceinline__ unsigned long long target_of(unsigned long long Z, float p) {
+    unsigned long long tg = (unsigned long long)ceil((double)p * (double)Z);
+    if (tg > Z) tg = Z;
+    return tg ? tg : 1ull;
+}
+
+// Exact cut of a one-CTA level with n <= SOLO_MAX slots: thread i ranks slot
+// i against every other slot of each head by (estimate descending, node id
+// ascending) -- the order of the masses, which are monotone in the estimate --
+// and sums the masses before it.  w: shared [SOLO_MAX][G] masses.
+template <int G>
+__device__ __noinline__ void solo_cut(const Level &L, HeadCut *cut, unsigned long long *w, float p) {
+    const int tid = threadIdx.x;
+    const int n = (int)L.n;
+#pragma unroll 1
+    for (int idx = tid; idx < n * G; idx += GT) {
+        const float e = L.sc[idx];
+        w[idx] = (e == -INFINITY) ? 0ull : mass_fx(expf(e - cut[idx % G].M));
+    }
+    gsync();
+    if (tid < G) {
+        unsigned long long Z = 0ull;
+#pragma unroll 1
+        for (int i = 0; i < n; ++i) Z += w[i * G + tid];
+        cut[tid].Z = Z;
+        cut[tid].target = target_of(Z, p);
+    }
+    gsync();
+    if (tid < n) {
+        uint32_t kb = 0u;
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) {
+            const float ei = L.sc[tid * G + h];
+            if (ei == -INFINITY) continue;
+            unsigned long long pre = 0ull;
+#pragma unroll 4
+            for (int j = 0; j < n; ++j) {
+                const float ej = L.sc[j * G + h];
+                if (ej > ei || (ej == ei && j < tid)) pre += w[j * G + h];
+            }
+            if (pre < cut[h].target) kb |= 1u << h;
+        }
+        L.keep[tid] = (uint8_t)kb;
+    }
+    gsync();
+}
+
+// Local histogram of round r over this CTA's slots on the path of every open
+// head, into hc/hm (shared; cleared here).
+template <int G>
+__device__ __noinline__ void local_hist(const Level &L, const HeadCut *cut, int r, uint32_t *hc,
+                                        unsigned long long *hm) {
+#pragma unroll 1
+    for (int i = threadIdx.x; i < G * NB; i += GT) {
+        hc[i] = 0u;
+        hm[i] = 0ull;
+    }
+    gsync();
+#pragma unroll 1
+    for (int64_t idx = threadIdx.x; idx < L.n * G; idx += GT) {
+        const int h = (int)(idx % G);
+        const HeadCut &H = cut[h];
+        if (H.mode != CUT_OPEN || H.rounds != r) continue;
+        const float e = L.sc[idx];
+        if (e == -INFINITY || path_cmp(H, e, r) != 0) continue;
+        const int b = round_bucket(H, e, r);
+        atomicAdd(&hc[h * NB + b], 1u);
+        atomicAdd(&hm[h * NB + b], mass_fx(expf(e - H.M)));
+    }
+    gsync();
+}
+
+// Fix the bucket of round r for every open head from the histogram
+// (cnt/mass: shared, or the team's global one read through L2).
+template <int G>
+__device__ __noinline__ void find_cut(HeadCut *cut, int r, const uint32_t *cnt, const unsigned long long *mass,
+                                      bool global, float p, unsigned long long *red) {
+    constexpr int TPH = GT / G, BPT = NB / TPH;
+    const int tid = threadIdx.x, h = tid / TPH, j = tid % TPH, lane = tid & 31;
+    const bool act = cut[h].mode == CUT_OPEN && cut[h].rounds == r;
+    unsigned long long sum = 0ull;
+#pragma unroll 1
+    for (int i = 0; i < BPT; ++i) {
+        const int b = j * BPT + i;
+        sum += act ? (global ? __ldcg(mass + h * NB + b) : mass[h * NB + b]) : 0ull;
+    }
+    // inclusive scan of the per-thread sums within each head's TPH threads
+    unsigned long long incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long y = __shfl_up_sync(FULL, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) red[tid >> 5] = incl;
+    gsync();
+    unsigned long long base = 0ull, tot = 0ull;
+    const int w0 = (h * TPH) >> 5, w1 = ((h + 1) * TPH) >> 5;
+#pragma unroll 1
+    for (int w = w0; w < w1; ++w) {
+        const unsigned long long s = red[w];
+        if (w < (tid >> 5)) base += s;
+        tot += s;
+    }
+    const unsigned long long excl = base + incl - sum;
+    if (r == 0 && act && j == 0) {
+        HeadCut &H = cut[h];
+        H.Z = tot;
+        H.target = target_of(tot, p);
+        H.C = 0ull;
+    }
+    gsync();
+    if (act) {
+        const HeadCut &H = cut[h];
+        const unsigned long long C = H.C, target = H.target;
+        if (C + excl < target && C + excl + sum >= target) {
+            unsigned long long run = C + excl;
+            int b = j * BPT;
+#pragma unroll 1
+            for (int i = 0; i < BPT; ++i) {
+                const int bi = j * BPT + i;
+                const unsigned long long m = global ? __ldcg(mass + h * NB + bi) : mass[h * NB + bi];
+                if (run + m >= target) {
+                    b = bi;
+                    break;
+                }
+                run += m;
+            }
+            const uint32_t n = global ? __ldcg(cnt + h * NB + b) : cnt[h * NB + b];
+            HeadCut &Hw = cut[h];
+            Hw.path[r] = b;
+            Hw.C = run;
+            Hw.nfin = n;
+            Hw.rounds = r + 1;
+            Hw.mode = (n <= (uint32_t)CAND_MAX) ? CUT_RANK : (r + 1 == HIST_ROUNDS ? CUT_ORDER : CUT_OPEN);
         }
     }
-    // the CTA's maximum per head
-    wsm[threadIdx.x] = (my_j0 == 0) ? lmax : -INFINITY;
     gsync();
-    if (threadIdx.x < G) {
-        float mx = -INFINITY;
-        for (int t = 0; t < GT; ++t) {
-            const int li0 = (t & 31) * K;
-            if (((li0 / R) % G) == (int)threadIdx.x) mx = fmaxf(mx, wsm[t]);
+}
+
+// Set head bit `bit` of keep[i] (byte array, any alignment) atomically.
+__device__ __forceinline__ void keep_or(uint8_t *keep, int64_t i, uint32_t bit) {
+    const uintptr_t at = reinterpret_cast<uintptr_t>(keep + i);
+    atomicOr(reinterpret_cast<uint32_t *>(at & ~(uintptr_t)3), bit << (8 * (at & 3)));
+}
+
+// Classify every local slot for every head: kept above the path, dropped
+// below it, boundary candidate on it.  Writes keep[], appends candidates
+// (CUT_RANK) to the list (global team list or shared list) and to own[],
+// and sums boundary masses (CUT_ORDER) into osum[h] (shared).
+template <int G>
+__device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsigned long long *lw, uint32_t *ls,
+                                      uint32_t *lcnt, uint32_t *own, uint32_t *own_cnt, unsigned long long *osum) {
+    const int lane = threadIdx.x & 31;
+    const int64_t iters = (L.n + GT - 1) / GT;
+#pragma unroll 1
+    for (int64_t it = 0; it < iters; ++it) {
+        const int64_t i = it * GT + threadIdx.x;
+        uint32_t kbits = 0u;
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) {
+            const HeadCut &H = cut[h];
+            const float e = i < L.n ? L.sc[i * G + h] : -INFINITY;
+            bool cand = false;
+            unsigned long long w = 0ull;
+            if (e != -INFINITY) {
+                if (H.mode == CUT_ALL) {
+                    kbits |= 1u << h;
+                } else if (H.mode == CUT_RANK || H.mode == CUT_ORDER) {
+                    const int pc = path_cmp(H, e, H.rounds);
+                    if (pc < 0) kbits |= 1u << h;
+                    else if (pc == 0) {
+                        w = mass_fx(expf(e - H.M));
+                        if (H.mode == CUT_RANK) cand = true;
+                        else atomicAdd(&osum[h], w);
+                    }
+                }
+            }
+            const unsigned bal = __ballot_sync(FULL, cand);
+            if (bal) {
+                const int leader = __ffs(bal) - 1;
+                uint32_t base = 0, obase = 0;
+                if (lane == leader) {
+                    base = atomicAdd(&lcnt[h], (uint32_t)__popc(bal));
+                    obase = atomicAdd(own_cnt, (uint32_t)__popc(bal));
+                }
+                base = __shfl_sync(FULL, base, leader);
+                obase = __shfl_sync(FULL, obase, leader);
+                if (cand) {
+                    const uint32_t rank = __popc(bal & ((1u << lane) - 1u));
+                    const uint32_t at = base + rank;
+                    if (at < (uint32_t)CAND_MAX) {
+                        lw[h * CAND_MAX + at] = w;
+                        ls[h * CAND_MAX + at] = (uint32_t)(L.s0 + i);
+                    }
+                    if (obase + rank < (uint32_t)(G * CAND_MAX)) own[obase + rank] = ((uint32_t)i << 3) | (uint32_t)h;
+                }
+            }
         }
-        a.pmax[((int64_t)kh * a.pmax_cap + bi) * G + threadIdx.x] = mx;
+        if (i < L.n) L.keep[i] = (uint8_t)kbits;
     }
     gsync();
+}
+
+// Rank this CTA's boundary candidates against the whole list (shared cw/cs,
+// counts from cut[h].nfin) and keep those the target still needs.
+template <int G>
+__device__ __noinline__ void rank_own(const Level &L, const HeadCut *cut, const unsigned long long *cw,
+                                      const uint32_t *cs, const uint32_t *own, uint32_t n_own) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll 1
+    for (uint32_t o = warp; o < n_own; o += GT / 32) {
+        const uint32_t code = own[o];
+        const int h = (int)(code & 7u);
+        const int64_t i = (int64_t)(code >> 3);
+        const HeadCut &H = cut[h];
+        const uint32_t nc = H.nfin;
+        const uint32_t slot = (uint32_t)(L.s0 + i);
+        const unsigned long long wi = mass_fx(expf(L.sc[i * G + h] - H.M));
+        unsigned long long pre = 0ull;
+#pragma unroll 1
+        for (uint32_t jj = lane; jj < nc; jj += 32) {
+            const unsigned long long wj = cw[h * CAND_MAX + jj];
+            const uint32_t sj = cs[h * CAND_MAX + jj];
+            if (wj > wi || (wj == wi && sj < slot)) pre += wj;
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) pre += __shfl_xor_sync(FULL, pre, off);
+        if (lane == 0 && H.C + pre < H.target) keep_or(L.keep, i, 1u << h);
+    }
+    gsync();
+}
+
+// Slot-order cut of the boundary for CUT_ORDER heads: `base[h]` is the mass
+// before this CTA's first slot (cut.C plus lower ranks' boundary masses).
+template <int G>
+__device__ __noinline__ void order_own(const Level &L, const HeadCut *cut, const unsigned long long *base,
+                                       unsigned long long *red) {
+    const int64_t per = (L.n + GT - 1) / GT;
+    const int64_t i0 = min(L.n, per * threadIdx.x), i1 = min(L.n, i0 + per);
+#pragma unroll 1
+    for (int h = 0; h < G; ++h) {
+        const HeadCut &H = cut[h];
+        if (H.mode != CUT_ORDER) continue;
+        unsigned long long mine = 0ull;
+#pragma unroll 1
+        for (int64_t i = i0; i < i1; ++i) {
+            const float e = L.sc[i * G + h];
+            if (e != -INFINITY && path_cmp(H, e, H.rounds) == 0) mine += mass_fx(expf(e - H.M));
+        }
+        unsigned long long tot;
+        unsigned long long run = g_scan_u64(mine, red, &tot) - mine + base[h];
+#pragma unroll 1
+        for (int64_t i = i0; i < i1; ++i) {
+            const float e = L.sc[i * G + h];
+            if (e != -INFINITY && path_cmp(H, e, H.rounds) == 0) {
+                if (run < H.target) keep_or(L.keep, i, 1u << h);
+                run += mass_fx(expf(e - H.M));
+            }
+        }
+    }
+    gsync();
+}
+
+// Write this CTA's kept slots (ascending) at the start of its slot range,
+// with per-rank counts.
+template <int G>
+__device__ __noinline__ void write_segment(const Decode &a, const Level &L, uint32_t *red32) {
+    const int64_t per = (L.n + GT - 1) / GT;
+    const int64_t i0 = min(L.n, per * threadIdx.x), i1 = min(L.n, i0 + per);
+    uint32_t mine = 0u;
+    uint32_t hc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) hc[h] = 0u;
+#pragma unroll 1
+    for (int64_t i = i0; i < i1; ++i) {
+        const uint32_t k = L.keep[i];
+        mine += k != 0u;
+#pragma unroll
+        for (int h = 0; h < G; ++h) hc[h] += (k >> h) & 1u;
+    }
+    uint32_t tot;
+    uint32_t at = g_scan_u32(mine, red32, &tot) - mine;
+    const int64_t dst = (int64_t)L.kh * a.slot_cap[L.l - 1] + L.s0;
+    int32_t *ids = a.kept_ids[L.l - 1] + dst;
+    uint8_t *msk = a.kept_mask[L.l - 1] + dst;
+#pragma unroll 1
+    for (int64_t i = i0; i < i1; ++i) {
+        const uint32_t k = L.keep[i];
+        if (k) {
+            ids[at] = L.node[i];
+            msk[at] = (uint8_t)k;
+            ++at;
+        }
+    }
+    // per-head counts: warp sums, then one atomic per warp into shared
+    uint32_t *hs = red32 + 16;
+    if (threadIdx.x < G) hs[threadIdx.x] = 0u;
+    gsync();
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        uint32_t x = hc[h];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+        if ((threadIdx.x & 31) == 0 && x) atomicAdd(&hs[h], x);
+    }
+    gsync();
+    if (threadIdx.x == 0) {
+        seg_ptr(a, L.l, L.kh)[L.tr] = tot;
+        if (L.tr == 0) {
+            int32_t *lv = lvl_ptr(a, L.l, L.kh);
+            lv[0] = L.T;
+            lv[1] = (int32_t)L.S;
+        }
+    }
+    if (threadIdx.x < G) hseg_ptr(a, L.l, L.kh)[(int64_t)L.tr * G + threadIdx.x] = hs[threadIdx.x];
+}
+
+// ---- one level ------------------------------------------------------------------
+
+// The histogram path of the cut (team, or one CTA with more than SOLO_MAX
+// slots): rounds, classification, boundary lists.  false: a barrier gave up.
+template <int G>
+__device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned char *smem, TeamSync &ts) {
+    using SM = RouteSmem<G>;
+    HeadCut *cut = reinterpret_cast<HeadCut *>(smem + SM::off_cut);
+    unsigned long long *red = reinterpret_cast<unsigned long long *>(smem + SM::off_red);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + SM::off_misc);
+    uint32_t *hc = reinterpret_cast<uint32_t *>(smem + SM::off_hc);
+    unsigned long long *hm = reinterpret_cast<unsigned long long *>(smem + SM::off_hm);
+    unsigned long long *cw = reinterpret_cast<unsigned long long *>(smem + SM::off_cw);
+    uint32_t *cs = reinterpret_cast<uint32_t *>(smem + SM::off_cs);
+    uint32_t *own = reinterpret_cast<uint32_t *>(smem + SM::off_own);
+    const int tid = threadIdx.x, kh = L.kh, T = L.T, tr = L.tr;
+    const bool team = T > 1;
+    const int64_t hbase = (int64_t)kh * HIST_ROUNDS * G * NB;
+    int rounds_used = 0;
+#pragma unroll 1
+    for (int r = 0; r < HIST_ROUNDS; ++r) {
+        bool open = false;
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) open |= cut[h].mode == CUT_OPEN;
+        if (!open) break;
+        local_hist<G>(L, cut, r, hc, hm);
+        rounds_used = r + 1;
+        if (team) {
+            uint32_t *gc = a.hist_cnt + hbase + (int64_t)r * G * NB;
+            unsigned long long *gm = a.hist_mass + hbase + (int64_t)r * G * NB;
+#pragma unroll 1
+            for (int i = tid; i < G * NB; i += GT)
+                if (hc[i]) {
+                    atomicAdd(gc + i, hc[i]);
+                    atomicAdd(gm + i, hm[i]);
+                }
+            if (!ts.sync()) return false;  // B
+            // the team's histogram into shared memory: independent loads
+#pragma unroll 8
+            for (int i = tid; i < G * NB; i += GT) {
+                hc[i] = __ldcg(gc + i);
+                hm[i] = __ldcg(gm + i);
+            }
+            gsync();
+            find_cut<G>(cut, r, hc, hm, false, a.p, red);
+        } else {
+            find_cut<G>(cut, r, hc, hm, false, a.p, red);
+        }
+    }
+    // classify, boundary lists
+    unsigned long long *osum = red + 64;
+    if (tid < 8) misc[tid] = 0u;  // [0]: own count, [4 + h]: shared list counters
+    if (tid < G) osum[tid] = 0ull;
+    gsync();
+    uint32_t *lcnt = team ? a.cand_cnt + (int64_t)kh * G : misc + 4;
+    unsigned long long *lw = team ? a.cand_w + (int64_t)kh * G * CAND_MAX : cw;
+    uint32_t *ls = team ? a.cand_slot + (int64_t)kh * G * CAND_MAX : cs;
+    classify<G>(L, cut, lw, ls, lcnt, own, misc, osum);
+    bool any_order = false, any_rank = false;
+#pragma unroll 1
+    for (int h = 0; h < G; ++h) {
+        any_order |= cut[h].mode == CUT_ORDER;
+        any_rank |= cut[h].mode == CUT_RANK;
+    }
+    if (team && any_order && tid < G) a.tsum[((int64_t)kh * SEG_CAP + tr) * G + tid] = osum[tid];
+    if (team) {
+        if (!ts.sync()) return false;  // C
+        // the histograms are consumed: clear this rank's share for the next level
+#pragma unroll 1
+        for (int r = 0; r < rounds_used; ++r) {
+            uint32_t *gc = a.hist_cnt + hbase + (int64_t)r * G * NB;
+            unsigned long long *gm = a.hist_mass + hbase + (int64_t)r * G * NB;
+            const int64_t lo = (int64_t)G * NB * tr / T, hi = (int64_t)G * NB * (tr + 1) / T;
+#pragma unroll 1
+            for (int64_t i = lo + tid; i < hi; i += GT) {
+                gc[i] = 0u;
+                gm[i] = 0ull;
+            }
+        }
+    }
+    const uint32_t n_own = min(misc[0], (uint32_t)(G * CAND_MAX));
+    if (any_rank && n_own > 0) {
+        if (team) {
+            // bring the team's lists into shared memory
+#pragma unroll 1
+            for (int h = 0; h < G; ++h) {
+                if (cut[h].mode != CUT_RANK) continue;
+#pragma unroll 1
+                for (uint32_t j = tid; j < cut[h].nfin; j += GT) {
+                    cw[h * CAND_MAX + j] = __ldcg(lw + h * CAND_MAX + j);
+                    cs[h * CAND_MAX + j] = __ldcg(ls + h * CAND_MAX + j);
+                }
+            }
+            gsync();
+        }
+        rank_own<G>(L, cut, cw, cs, own, n_own);
+    }
+    if (any_order) {
+        unsigned long long *base = red + 72;
+        if (tid < G) {
+            unsigned long long bsum = cut[tid].C;
+            if (team && cut[tid].mode == CUT_ORDER) {
+#pragma unroll 1
+                for (int r = 0; r < tr; ++r) bsum += __ldcg(a.tsum + ((int64_t)kh * SEG_CAP + r) * G + tid);
+            }
+            base[tid] = bsum;
+        }
+        gsync();
+        order_own<G>(L, cut, base, red);
+    }
+    return true;
+}
+
+// Score and cut level l of KV head kh as rank tr of a team of T CTAs (T = 1:
+// this CTA alone).  `S` is the frontier size, `pref`/Tp/Sp the parent level's
+// segments (loaded by the caller).  F[h] receives the frontier counts.
+// Returns false when a team barrier gave up.
+template <int HD, int R, int G>
+__device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, int tr, int64_t S, int Tp, int64_t Sp,
+                                         unsigned char *smem, TeamSync &ts, uint32_t (&F)[G]) {
+    using SM = RouteSmem<G>;
+    HeadCut *cut = reinterpret_cast<HeadCut *>(smem + SM::off_cut);
+    uint32_t *pref = reinterpret_cast<uint32_t *>(smem + SM::off_pref);
+    float *wm = reinterpret_cast<float *>(smem + SM::off_wm);
+    uint32_t *wc = reinterpret_cast<uint32_t *>(smem + SM::off_wc);
+    const int tid = threadIdx.x;
+    Level L;
+    L.l = l;
+    L.kh = kh;
+    L.T = T;
+    L.tr = tr;
+    L.top = (l == a.t.D);
+    L.S = S;
+    L.s0 = seg_start(S, T, tr);
+    L.n = seg_start(S, T, tr + 1) - L.s0;
+    L.Tp = Tp;
+    L.Sp = Sp;
+    if (L.n > LOC_CAP) {
+        const int64_t base = (int64_t)kh * a.score_cap + L.s0;
+        L.sc = a.scores + base * G;
+        L.node = a.slot_node + base;
+        L.keep = a.slot_keep + base;
+    } else {
+        L.sc = reinterpret_cast<float *>(smem + SM::off_sc);
+        L.node = reinterpret_cast<int32_t *>(smem + SM::off_node);
+        L.keep = smem + SM::off_keep;
+    }
+    const bool team = T > 1;
+    // ---- score
+    if (tid < 8 * G) {
+        wm[tid] = -INFINITY;
+        wc[tid] = 0u;
+    }
+    int32_t *pid = reinterpret_cast<int32_t *>(smem + SM::off_pid);
+    uint8_t *pmk = smem + SM::off_pmk;
+#pragma unroll 1
+    for (int64_t c0 = L.s0; c0 < L.s0 + L.n; c0 += LOC_CAP) {
+        const int64_t c1 = min(L.s0 + L.n, c0 + LOC_CAP);
+        int64_t k0 = 0;
+        if (!L.top) load_parents(a, L, c0, c1, pref, pid, pmk, k0);
+        gsync();
+        score_chunks<HD, R, G>(a, L, c0, c1, k0, pid, pmk, smem, wm, wc);
+        gsync();
+    }
+    if (tid < G) {
+        float m = -INFINITY;
+        uint32_t c = 0u;
+#pragma unroll 1
+        for (int w = 0; w < GT / 32; ++w) {
+            m = fmaxf(m, wm[w * G + tid]);
+            c += wc[w * G + tid];
+        }
+        if (team) {
+            a.tmax[((int64_t)kh * SEG_CAP + tr) * G + tid] = m;
+            a.tcnt[((int64_t)kh * SEG_CAP + tr) * G + tid] = c;
+        } else {
+            cut[tid].M = m;
+            cut[tid].F = c;
+        }
+    }
+    if (team && !ts.sync()) return false;  // A
+    if (team && tid < G) {
+        float m = -INFINITY;
+        uint32_t c = 0u;
+#pragma unroll 1
+        for (int r = 0; r < T; ++r) {
+            m = fmaxf(m, __ldcg(a.tmax + ((int64_t)kh * SEG_CAP + r) * G + tid));
+            c += __ldcg(a.tcnt + ((int64_t)kh * SEG_CAP + r) * G + tid);
+        }
+        cut[tid].M = m;
+        cut[tid].F = c;
+    }
+    const bool keep_all = !(a.p < 1.f);
+    gsync();
+    if (tid < G) {
+        HeadCut &H = cut[tid];
+        H.rounds = 0;
+        H.nfin = 0u;
+        H.mode = H.F == 0u ? CUT_NONE : (keep_all ? CUT_ALL : CUT_OPEN);
+    }
+    gsync();
+#pragma unroll
+    for (int h = 0; h < G; ++h) F[h] = cut[h].F;
+    // ---- cut
+    if (keep_all) {
+#pragma unroll 1
+        for (int64_t i = tid; i < L.n; i += GT) {
+            uint32_t kb = 0u;
+#pragma unroll 1
+            for (int h = 0; h < G; ++h) kb |= (L.sc[i * G + h] != -INFINITY ? 1u : 0u) << h;
+            L.keep[i] = (uint8_t)kb;
+        }
+        gsync();
+    } else if (!team && L.n <= SOLO_MAX) {
+        solo_cut<G>(L, cut, reinterpret_cast<unsigned long long *>(smem + SM::off_hm), a.p);
+    } else {
+        if (!hist_cut<G>(a, L, smem, ts)) return false;
+    }
+    write_segment<G>(a, L, reinterpret_cast<uint32_t *>(smem + SM::off_red));
+    if (team) {
+        if (!ts.sync()) return false;  // D
+        // the boundary lists are consumed: rank 0 clears the counters
+        if (tr == 0 && tid < G) a.cand_cnt[(int64_t)kh * G + tid] = 0u;
+    } else {
+        gsync();
+    }
+    return true;
 }
 
 }  // namespace zha

@@ -27,7 +27,7 @@ static __device__ __align__(256) unsigned char g_dense_scratch[ZHA_STATIC_SCRATC
 namespace {
 
 constexpr int DEV_MAX = 64;
-constexpr int STATIC_CTA_CAP = 1024;  // the context path's cap on attention CTAs
+constexpr int STATIC_CTA_CAP = SEG_CAP;  // the context path's cap on attention CTAs
 
 struct DevScratch {
     unsigned char *ptr = nullptr;  // device address of g_dense_scratch on this device
@@ -84,7 +84,7 @@ int zha_dense_decode_static(const zha_config *cfg, const void *d_K, const void *
     // the same grid as the context path: one CTA per SM
     const int n_cta = std::min(STATIC_CTA_CAP, ds.n_sm);
     const int64_t part_bytes = align256((int64_t)n_cta * cfg->h_q * (cfg->d + 4) * 4);
-    const int64_t ticket_bytes = (int64_t)(MAXD + 2) * cfg->h_kv * 4;
+    const int64_t ticket_bytes = (int64_t)cfg->h_kv * 4;
     if (part_bytes + ticket_bytes > (int64_t)ZHA_STATIC_SCRATCH_BYTES) return ZHA_ERR_CAPACITY;
 
     Decode dc{};
@@ -107,12 +107,12 @@ int zha_dense_decode_static(const zha_config *cfg, const void *d_K, const void *
     dc.out = d_out;
     dc.part = reinterpret_cast<float *>(ds.ptr);
     dc.part_cap = n_cta;
-    dc.done = reinterpret_cast<uint32_t *>(ds.ptr + part_bytes);
+    dc.ticket = reinterpret_cast<uint32_t *>(ds.ptr + part_bytes);
     dc.status = d_status;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the merge tickets must start at zero (a call that gave up on a wait can
     // leave them raised); the partials are written before they are read
-    if (cudaMemsetAsync(dc.done, 0, (size_t)ticket_bytes, s) != cudaSuccess) return ZHA_ERR_CUDA;
+    if (cudaMemsetAsync(dc.ticket, 0, (size_t)ticket_bytes, s) != cudaSuccess) return ZHA_ERR_CUDA;
     if (launch_dense(dc, n_cta, s) != cudaSuccess) return ZHA_ERR_CUDA;
     return ZHA_OK;
 }
