@@ -74,6 +74,51 @@ def dist_setup(n_gpus):
     return rank, world, local
 
 
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources: ncu counters stay valid only for the kernels
+    they were taken on."""
+    import glob
+    import hashlib
+
+    csrc = os.path.join(ROOT, "tree_indexed_sparse_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """Per-launch DRAM bytes of k_decode from the committed ncu summary, or
+    None when none was taken for this workload or the kernels changed since."""
+    path = os.path.join(ROOT, "profiles", "k_decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("bytes_per_launch", {}).get(workload)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest value of x over all ranks (the job's time is its slowest
+    rank's); x itself with one rank."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Replicas: every rank decodes its own token stream; whole-job microseconds
+    per decoded token = slowest rank's time over all ranks' tokens."""
+    return ms_max * 1000.0 / (units_per_rank * world)
+
+
 class Clocks:
     """nvidia-smi sampling during the timed region."""
 
@@ -83,7 +128,16 @@ class Clocks:
         vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
         self.index = vis[local].strip() if local < len(vis) else str(local)
 
+    def _lines(self):
+        try:
+            with open(self.path) as f:
+                return sum(1 for line in f if line.count(",") >= 8)
+        except OSError:
+            return 0
+
     def start(self):
+        """Launch the sampler and wait (up to 5 s) for its first sample, so that
+        samples cover the timed region that follows."""
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
@@ -92,13 +146,22 @@ class Clocks:
                  "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                 "--format=csv,noheader,nounits", "-lms", "20"], stdout=self.f, stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while self._lines() < 1 and time.time() - t0 < 5.0 and self.proc.poll() is None:
+                time.sleep(0.01)
+            self.first = self._lines()
         except Exception:
             self.proc = None
 
     def stop(self):
         if not self.proc:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        # one more sample after the timed region, then stop
+        t0 = time.time()
+        n0 = self._lines()
+        while self._lines() <= n0 and time.time() - t0 < 2.0 and self.proc.poll() is None:
+            time.sleep(0.005)
         self.proc.terminate()
         self.proc.wait()
         self.f.close()
@@ -243,7 +306,7 @@ def run_zha(args, rank, world, local):
     stamps = torch.zeros(w.D + 3, dtype=torch.int64, device=dev)
     zha.zha_set_phase_timer(cache.ctx, stamps)
     ea, eb, ec = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-    t_step, t_app, t_route, t_attn, t_merge, t_levels = [], [], [], [], [], []
+    t_step, t_app, t_route, t_attn, t_merge = [], [], [], [], []
     clocks = Clocks(local)
     for i in range(W):
         flush.zero_()
@@ -271,7 +334,6 @@ def run_zha(args, rank, world, local):
         t_route.append(dec - (ns[w.D + 2] - ns[w.D]) * 1e-6)
         t_attn.append((ns[w.D + 1] - ns[w.D]) * 1e-6)
         t_merge.append((ns[w.D + 2] - ns[w.D + 1]) * 1e-6)
-        t_levels.append([(ns[j + 1] - ns[j]) * 1e-6 for j in range(w.D)])
     torch.cuda.synchronize()
     wall = time.time() - wall0
     if world > 1:
@@ -279,12 +341,9 @@ def run_zha(args, rank, world, local):
     clk = clocks.stop()
     same = torch.equal(out, ref_out)
     total_ms = sum(t_step)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / K
-    us_token = ms_step * 1000.0 / world
+    us_token = job_value(K, world, total_ms)
 
     route_b = [s[0] for s in per_step]
     attn_b = [s[1] for s in per_step]
@@ -296,8 +355,7 @@ def run_zha(args, rank, world, local):
         "append": {"us": 1e3 * statistics.mean(t_app), "bytes": statistics.mean(app_b),
                    "gbs": sum(app_b) / (sum(t_app) * 1e-3) / 1e9},
         "route": {"us": 1e3 * statistics.mean(t_route), "bytes": statistics.mean(route_b),
-                  "gbs": sum(route_b) / (sum(t_route) * 1e-3) / 1e9,
-                  "us_per_level_top_down": [1e3 * statistics.mean(x) for x in zip(*t_levels)]},
+                  "gbs": sum(route_b) / (sum(t_route) * 1e-3) / 1e9},
         "attention": {"us": 1e3 * statistics.mean(t_attn), "bytes": statistics.mean(attn_b),
                       "gbs": sum(attn_b) / (sum(t_attn) * 1e-3) / 1e9},
         "merge": {"us": 1e3 * statistics.mean(t_merge)},
@@ -309,7 +367,7 @@ def run_zha(args, rank, world, local):
     achieved = sum(dec_b) / (sum(t_dec) * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": "k_decode", "launches_per_step": 1,
                 "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                "peak_kind": f"{peak_kind} copy bandwidth (burst)", "traffic": None,
+                "peak_kind": f"{peak_kind} copy bandwidth (burst)", "traffic": measured_traffic(w.name),
                 "algorithmic_bytes_per_launch": statistics.mean(dec_b), "us_per_launch": 1e3 * statistics.mean(t_dec)}
 
     # dense flash-decode over the same cache (n_tokens + W + K rows now)
@@ -358,10 +416,7 @@ def run_zha(args, rank, world, local):
     h2d = dq.numel() * 4 + 2 * dk.numel() * dk.element_size()
     d2h = hout.numel() * 4
     e2e_us = 1e3 * sum(t_e2e) / K / world
-    if world > 1:
-        tt = torch.tensor([e2e_us], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        e2e_us = float(tt.item())
+    e2e_us = max_over_ranks(e2e_us, world, dev)
 
     res = {
         "metric": METRIC, "value": us_token, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
@@ -452,6 +507,65 @@ def run_reference(args, rank, world):
             "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+CROSSOVER_N = [16384, 32768, 49152, 65536, 98304, 131072, 196608, 262144, 524288, 1048576]
+
+
+def run_crossover(args, local):
+    """The light workload's settings (chunk 8, R = 1, p = 0.75, mixture keys)
+    at growing context lengths: device time of one routed decode and of one
+    dense decode per length (L2 flushed between calls), and the length at
+    which the two curves cross (linear interpolation)."""
+    import tree_indexed_sparse_b200 as zha
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    base = workloads.WORKLOADS["light_1m"]
+    steps = 32
+    rows = []
+    for n in CROSSOVER_N:
+        D = 1  # deepest tree with at least 4 top nodes, as at 1M (c^D * 4 <= n)
+        while D < base.D and base.c ** (D + 1) * 4 <= n:
+            D += 1
+        w = dataclasses.replace(base.scaled(n, steps=steps), D=D, appends_per_step=0, appends_after=0)
+        inp = workloads.generate(w, dev)
+        dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
+        cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, device=dev)
+        cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
+        out = torch.empty(w.h_q, w.d, dtype=torch.float32, device=dev)
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tz, td = [], []
+        for i in range(3 + steps):
+            q = inp.Q[i % steps]
+            for fn, acc in ((lambda: cache.decode(q, w.p, out=out), tz), (lambda: cache.dense(q, out=out), td)):
+                flush.zero_()
+                torch.cuda._sleep(HOLD_CYCLES)
+                ea.record(stream)
+                fn()
+                eb.record(stream)
+                torch.cuda.synchronize()
+                if i >= 3:
+                    acc.append(ea.elapsed_time(eb) * 1e3)
+        assert cache.status() == 0
+        rows.append({"n_tokens": n, "D": D, "zha_us": statistics.median(tz), "dense_us": statistics.median(td)})
+        del cache, inp
+        torch.cuda.empty_cache()
+    cross = None
+    for a, b in zip(rows, rows[1:]):
+        da, db = a["zha_us"] - a["dense_us"], b["zha_us"] - b["dense_us"]
+        if da >= 0 > db:
+            cross = a["n_tokens"] + (b["n_tokens"] - a["n_tokens"]) * da / (da - db)
+            break
+    if cross is None and rows and rows[0]["zha_us"] < rows[0]["dense_us"]:
+        cross = f"< {rows[0]['n_tokens']}"
+    return {"metric": "crossover context length, routed vs dense decode (light workload settings)",
+            "unit": "tokens", "value": cross, "higher_is_better": False, "n_gpus": 1, "steps": steps,
+            "data": "synthetic", "rows": rows,
+            "config": {"workload": "light_1m settings at each n_tokens (depth: at least 4 top nodes)",
+                       "l2": "256 MiB written before every call"}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -461,9 +575,17 @@ def main():
     ap.add_argument("--workload", choices=workloads.ORDER, default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--crossover", action="store_true",
+                    help="sweep the light workload's settings over context lengths, routed vs dense")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_setup(args.gpus)
+    if args.crossover:
+        if rank == 0:
+            print(json.dumps(run_crossover(args, local)), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
     else:
