@@ -41,44 +41,48 @@ namespace zha {
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr int ACW = 8;                         // consumer warps
 constexpr int A_THREADS = (ACW + 1) * 32;      // + one producer warp
-constexpr int TT = 64;                         // tokens per stage
 constexpr int TW = 16;                         // tokens per consumer warp per stage
-constexpr int CW_STAGE = TT / TW;              // consumer warps per stage (4)
 constexpr int LEAF_WIN = 1024;                 // leaf ids the producer keeps in shared memory
-constexpr size_t STAGE_BUDGET = 176 * 1024;    // shared memory for the stage ring
-static_assert(CW_STAGE * 2 == ACW, "two halves of consumer warps alternate over stages");
+constexpr size_t STAGE_BUDGET = 200 * 1024;    // shared memory for the stage ring
 
 // One partial record: o[HD], max, sum, two pads (16-byte aligned records).
 template <int HD>
 constexpr int prec() { return HD + 4; }
 
-// A stage holds TT tokens as NG groups of GR consecutive tokens.  Each group
-// is filled by bulk copies of whole runs of rows (one copy for a run of GR
-// contiguous rows); groups sit GS bytes apart, 16 bytes more than their rows,
-// so that row w of the eight groups falls in eight different bank groups.
-// Token slot t = GR*group + w sits at row_off(t); K groups first, then V.
+// A stage holds TT tokens as 8 groups of GR consecutive tokens (bf16: 128
+// tokens, groups of 16 rows, 4 KB per copy at d = 128; fp32: 64 tokens, groups
+// of 8).  Each group is filled by bulk copies of whole runs of rows; groups
+// sit GS bytes apart, 16 bytes more than their rows, so that row w of the
+// eight groups falls in eight different bank groups.  Token slot
+// t = GR*group + w sits at row_off(t); K groups first, then V.  The stage goes
+// to CW consumer warps (bf16: all 8; fp32: 4, the two halves alternating).
 template <typename KT, int HD>
 struct StageCfg {
     static constexpr int ES = (int)sizeof(KT);
     static constexpr int RB = HD * ES;                      // row bytes
-    static constexpr int GR = 8;                            // rows per group
-    static constexpr int NG = TT / GR;                      // groups per stage
+    static constexpr int TT = ES == 2 ? 128 : 64;           // tokens per stage
+    static constexpr int NG = 8;                            // groups per stage
+    static constexpr int GR = TT / NG;                      // rows per group
+    static constexpr int GLOG = ES == 2 ? 4 : 3;            // log2(GR)
     static constexpr int GS = GR * RB + 16;                 // group stride
     static constexpr int HALF = NG * GS;                    // K part (V part follows)
     static constexpr int STAGE_BYTES = 2 * HALF;
+    static constexpr int CW = TT / TW;                      // consumer warps per stage
+    static constexpr int HALVES = ACW / CW;                 // consumer halves alternating over stages
     static constexpr int S0 = (int)(STAGE_BUDGET / STAGE_BYTES);
     static constexpr int STAGES = S0 > 6 ? 6 : S0;
     static_assert(STAGES >= 2, "stage ring");
     static_assert(RB % 16 == 0 && GS % 16 == 0, "bulk copies need 16-byte aligned rows");
-    static_assert(NG == 8, "a matrix load takes one row from each of the eight groups");
-    static __device__ __forceinline__ int row_off(int t) { return (t >> 3) * GS + (t & 7) * RB; }
+    static_assert((1 << GLOG) == GR && 2 * CW == GR, "each consumer warp takes two rows of every group");
+    static_assert(HALVES * CW == ACW && TW * CW == TT, "consumer warps cover a stage");
+    static __device__ __forceinline__ int row_off(int t) { return (t >> GLOG) * GS + (t & (GR - 1)) * RB; }
 };
 
 template <typename KT, int HD, int G>
 struct ASmem {
     using C = StageCfg<KT, HD>;
     static constexpr size_t off_meta = (size_t)C::STAGES * C::STAGE_BYTES;
-    static constexpr size_t off_bar = (off_meta + C::STAGES * TT + 15) / 16 * 16;  // full[ST], empty[ST]
+    static constexpr size_t off_bar = (off_meta + C::STAGES * C::TT + 15) / 16 * 16;  // full[ST], empty[ST]
     static constexpr size_t off_abort = off_bar + 2 * C::STAGES * 8;
     static constexpr size_t off_merge = (off_abort + 16 + 15) / 16 * 16;
     static constexpr size_t off_pw = off_merge + (size_t)ACW * G * (HD + 2) * 4;   // FMA consumers' p slots
@@ -160,8 +164,8 @@ struct MmaAttn {
 
     // The 16 tokens of consumer slot wq of a stage: rows w1 = 2 wq and
     // w2 = 2 wq + 1 of each of the 8 groups.  Column n of the first score tile
-    // is token 8n + w1, of the second 8n + w2; the same order is the k order
-    // of p.v.  sK/sV: the stage's K and V parts, msk: its 64 head masks.
+    // is token GR n + w1, of the second GR n + w2; the same order is the k
+    // order of p.v.  sK/sV: the stage's K and V parts, msk: its head masks.
     template <typename SC>
     __device__ void tokens(const unsigned char *sK, const unsigned char *sV, const uint8_t *msk, int wq, int lane) {
         const int g = lane >> 2, c4 = lane & 3;
@@ -182,10 +186,11 @@ struct MmaAttn {
         }
         const uint32_t hb = g < G ? (1u << g) : 0u;
         float x[4];
-        x[0] = (msk[16 * c4 + w1] & hb) ? s0[0] + s0[2] : -INFINITY;
-        x[1] = (msk[16 * c4 + 8 + w1] & hb) ? s0[1] + s0[3] : -INFINITY;
-        x[2] = (msk[16 * c4 + w2] & hb) ? s1[0] + s1[2] : -INFINITY;
-        x[3] = (msk[16 * c4 + 8 + w2] & hb) ? s1[1] + s1[3] : -INFINITY;
+        constexpr int GR = SC::GR;
+        x[0] = (msk[GR * (2 * c4) + w1] & hb) ? s0[0] + s0[2] : -INFINITY;
+        x[1] = (msk[GR * (2 * c4 + 1) + w1] & hb) ? s0[1] + s0[3] : -INFINITY;
+        x[2] = (msk[GR * (2 * c4) + w2] & hb) ? s1[0] + s1[2] : -INFINITY;
+        x[3] = (msk[GR * (2 * c4 + 1) + w2] & hb) ? s1[1] + s1[3] : -INFINITY;
         float mt = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
         mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 1));
         mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
@@ -289,7 +294,7 @@ struct FmaAttn {
     }
 
     // The warp's TW tokens (token i of consumer slot wq is stage slot
-    // 8 (i % 8) + 2 wq + i / 8), in passes of SUBT.
+    // GR (i % 8) + 2 wq + i / 8), in passes of SUBT.
     template <typename SC>
     __device__ void tokens(const unsigned char *sK, const unsigned char *sV, const uint8_t *msk, int wq, float *pw,
                            int lane) {
@@ -307,7 +312,7 @@ struct FmaAttn {
 #pragma unroll
         for (int r = 0; r < C::RPB; ++r) {
             const int i = i0 + r * C::RPL + grp;
-            const int t = 8 * (i & 7) + 2 * wq + (i >> 3);
+            const int t = SC::GR * (i & 7) + 2 * wq + (i >> 3);
             off[r] = SC::row_off(t);
             mr[r] = msk[t];
             float k[C::EPL];
@@ -480,19 +485,23 @@ struct StageMap {
 
 // Fill the stage map; all threads of the CTA call it, then it is valid after
 // the __syncthreads inside.  Gather: the level-1 segments written by routing.
-template <bool DENSE>
+template <bool DENSE, int TT>
 __device__ void stage_map_init(const Decode &a, StageMap &map) {
     const int h_kv = a.t.h_kv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if ((int)threadIdx.x < h_kv) {  // level 1's team and frontier sizes, in parallel
+        const int kh = threadIdx.x;
+        map.T1[kh] = DENSE ? 1 : __ldcg(a.lvl + (int64_t)kh * 2);
+        map.S1[kh] = DENSE ? 0 : __ldcg(a.lvl + (int64_t)kh * 2 + 1);
+    }
+    __syncthreads();
     if (threadIdx.x == 0) {
         map.h_kv = h_kv;
         int off = 0;
+#pragma unroll 1
         for (int kh = 0; kh < h_kv; ++kh) {
-            const int T = DENSE ? 1 : __ldcg(a.lvl + (int64_t)kh * 2);
-            map.T1[kh] = T;
-            map.S1[kh] = DENSE ? 0 : __ldcg(a.lvl + (int64_t)kh * 2 + 1);
             map.soff[kh] = off;
-            off += T + 1;
+            off += map.T1[kh] + 1;
         }
         map.soff[h_kv] = off;
     }
@@ -540,7 +549,7 @@ template <typename KT, int HD, int G, bool DENSE>
 __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char *smem, int b, int nb) {
     using C = StageCfg<KT, HD>;
     using SM = ASmem<KT, HD, G>;
-    constexpr int ST = C::STAGES, RB = C::RB, GR = C::GR;
+    constexpr int ST = C::STAGES, RB = C::RB, GR = C::GR, TT = C::TT;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int h_kv = a.t.h_kv, c = a.t.c, clog = a.t.c_log2;
     uint8_t *meta = smem + SM::off_meta;
@@ -548,11 +557,11 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
     uint64_t *empty = full + ST;
     volatile int *abort = reinterpret_cast<volatile int *>(smem + SM::off_abort);
     float *merge = reinterpret_cast<float *>(smem + SM::off_merge);
-    const int64_t N = a.t.n_tokens;
+    const int N = (int)a.t.n_tokens;  // rows per KV head < 2^31
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], CW_STAGE);
+            mbar_init(&empty[s], C::CW);
         }
         *abort = 0;
         mbar_init_fence();
@@ -560,42 +569,51 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
     __syncthreads();
     const int64_t U = map.pref[h_kv];
     const int64_t u0 = U * b / nb, u1 = U * (b + 1) / nb;
-    const int64_t n = u1 - u0;
+    const int n = (int)(u1 - u0);
 
     if (warp == ACW) {
         // ---------------- producer warp ----------------
         int32_t *win_ids = reinterpret_cast<int32_t *>(smem + SM::off_win);
         uint8_t *win_msk = smem + SM::off_win + (size_t)LEAF_WIN * 4;
-        int win_kh = -1;
-        int64_t win_k0 = 0;
-        int64_t issued = 0;
-        for (int64_t j = 0; j < n; ++j) {
-            const int slot = (int)(j % ST);
+        int win_kh = -1, win_k0 = 0;
+        int issued = 0;
+        int kh;
+        int64_t st64;
+        map.locate(u0, kh, st64);
+        int st = (int)st64;
+        // lane gi < 8: K rows of group gi; lane 8 + gi: V rows of group gi
+        const int gi = lane & 7;
+        const bool act = lane < 16;
+        const bool isV = lane >= 8;
+#pragma unroll 1
+        for (int j = 0; j < n; ++j, ++st) {
+            while (kh + 1 < h_kv && u0 + j >= map.pref[kh + 1]) {
+                ++kh;
+                st = 0;
+            }
+            const int slot = j % ST;
             const uint32_t round = (uint32_t)(j / ST);
             if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1u, abort)) {
                 set_status(a.status, ZHA_TIMEOUT_CODE);
                 *abort = 1;
                 break;
             }
-            int kh;
-            int64_t st;
-            map.locate(u0 + j, kh, st);
-            const unsigned char *Kh = reinterpret_cast<const unsigned char *>(a.t.K) + (int64_t)kh * a.t.kv_cap * C::RB;
-            const unsigned char *Vh = reinterpret_cast<const unsigned char *>(a.t.V) + (int64_t)kh * a.t.kv_cap * C::RB;
+            const unsigned char *Kh = reinterpret_cast<const unsigned char *>(a.t.K) + (int64_t)kh * a.t.kv_cap * RB;
+            const unsigned char *Vh = reinterpret_cast<const unsigned char *>(a.t.V) + (int64_t)kh * a.t.kv_cap * RB;
             unsigned char *sK = smem + (size_t)slot * C::STAGE_BYTES;
             uint8_t *mt = meta + slot * TT;
-            const int64_t t0 = st * TT;
-            int64_t L = 0;
+            const int t0 = st * TT;
+            int L = 0;
             if (!DENSE) {
-                L = map.cnt[kh];
-                const int64_t kf = (int64_t)div_c((uint32_t)t0, c, clog);
-                const int64_t kl = min(L - 1, (int64_t)div_c((uint32_t)(t0 + TT - 1), c, clog));
+                L = (int)map.cnt[kh];
+                const int kf = (int)div_c((uint32_t)t0, c, clog);
+                const int kl = min(L - 1, (int)div_c((uint32_t)(t0 + TT - 1), c, clog));
                 if (kh != win_kh || kl >= win_k0 + LEAF_WIN || kf < win_k0) {
                     // refill the window from leaf rank kf up to the last leaf
                     // this CTA needs in this KV head: independent loads
-                    const int64_t jl = min(u1, map.pref[kh + 1]) - 1 - map.pref[kh];
-                    const int64_t klast = min(L - 1, (int64_t)div_c((uint32_t)(jl * TT + TT - 1), c, clog));
-                    const int nwin = (int)min((int64_t)LEAF_WIN, klast - kf + 1);
+                    const int jl = (int)(min(u1, map.pref[kh + 1]) - 1 - map.pref[kh]);
+                    const int klast = min(L - 1, (int)div_c((uint32_t)(jl * TT + TT - 1), c, clog));
+                    const int nwin = min(LEAF_WIN, klast - kf + 1);
                     win_kh = kh;
                     win_k0 = kf;
                     const int64_t kbase = (int64_t)kh * a.slot_cap[0];
@@ -608,47 +626,49 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                     __syncwarp();
                 }
             }
-            // lane gi < 8: K rows of group gi; lane 8 + gi: V rows of group gi
-            const int gi = lane & 7;
-            const bool act = lane < 16;
-            const bool isV = lane >= 8;
-            int64_t row[GR];
+            // rows of this lane's group: flattened positions ug .. ug + GR - 1
+            const int ug = t0 + gi * GR;
+            int row[GR];
             uint32_t nvalid = 0u;
+            if (DENSE) {
 #pragma unroll
-            for (int w = 0; w < GR; ++w) {
-                const int64_t u = t0 + gi * GR + w;
-                int64_t r = -1;
-                uint32_t mk = 0u;
-                if (act) {
-                    if (DENSE) {
-                        if (u < N) {
-                            r = u;
-                            mk = 0xffu;
-                        }
-                    } else {
-                        const int64_t k = div_c((uint32_t)u, c, clog);
-                        if (k < L) {
-                            const int64_t rr = (int64_t)win_ids[k - win_k0] * c + (u - k * c);
-                            if (rr < N) {
-                                r = rr;
-                                mk = win_msk[k - win_k0];
-                            }
+                for (int w = 0; w < GR; ++w) {
+                    row[w] = (act && ug + w < N) ? ug + w : -1;
+                    if (act && !isV) mt[gi * GR + w] = row[w] >= 0 ? 0xffu : 0u;
+                }
+            } else {
+                int k = (int)div_c((uint32_t)ug, c, clog), off = ug - k * c;
+#pragma unroll
+                for (int w = 0; w < GR; ++w) {
+                    if (off == c) {
+                        ++k;
+                        off = 0;
+                    }
+                    int r = -1;
+                    uint32_t mk = 0u;
+                    if (act && k < L) {
+                        const int rr = win_ids[k - win_k0] * c + off;
+                        if (rr < N) {
+                            r = rr;
+                            mk = win_msk[k - win_k0];
                         }
                     }
+                    row[w] = r;
+                    if (act && !isV) mt[gi * GR + w] = (uint8_t)mk;
+                    ++off;
                 }
-                row[w] = r;
-                nvalid += r >= 0;
-                if (act && !isV) mt[gi * GR + w] = (uint8_t)mk;
             }
+#pragma unroll
+            for (int w = 0; w < GR; ++w) nvalid += row[w] >= 0;
             uint32_t bytes = nvalid * RB;
 #pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) bytes += __shfl_xor_sync(FULL, bytes, off);
+            for (int o = 16; o >= 1; o >>= 1) bytes += __shfl_xor_sync(FULL, bytes, o);
             unsigned char *dst = sK + (isV ? C::HALF : 0) + gi * C::GS;
             // rows without a token: zeros, so that 0 * row stays 0 in the
             // products (the fence orders these generic stores before later
             // bulk copies into the same rows)
             if (act && nvalid < (uint32_t)GR) {
-#pragma unroll
+#pragma unroll 1
                 for (int w = 0; w < GR; ++w) {
                     if (row[w] >= 0) continue;
                     uint4 *z = reinterpret_cast<uint4 *>(dst + w * RB);
@@ -668,7 +688,8 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                     const bool brk = (w == GR) || row[w] < 0 || row[w - 1] < 0 || row[w] != row[w - 1] + 1;
                     if (brk) {
                         if (row[w0] >= 0)
-                            bulk_g2s(dst + w0 * RB, src + row[w0] * RB, (uint32_t)((w - w0) * RB), &full[slot]);
+                            bulk_g2s(dst + w0 * RB, src + (size_t)row[w0] * RB, (uint32_t)((w - w0) * RB),
+                                     &full[slot]);
                         w0 = w;
                     }
                 }
@@ -677,7 +698,7 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
         }
         // on an abort, wait (bounded) for the copies already in flight
         if (*abort) {
-            for (int64_t j = (issued > ST ? issued - ST : 0); j < issued; ++j)
+            for (int j = (issued > ST ? issued - ST : 0); j < issued; ++j)
                 mbar_wait(&full[j % ST], (uint32_t)((j / ST) & 1), nullptr);
         }
     } else {
@@ -687,13 +708,13 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
         gsync();
         typename Consumer<KT, HD, G>::T st;
         st.init();
-        const int half = warp / CW_STAGE, wq = warp % CW_STAGE;
+        const int half = warp / C::CW, wq = warp % C::CW;
         const float qscale = a.t.scale * LOG2E;
-        int kh_cur = -1;
-        for (int64_t j = 0; j < n; ++j) {
-            int kh;
-            int64_t stage_in_kh;
-            map.locate(u0 + j, kh, stage_in_kh);
+        int kh_cur = -1, kh = 0;
+        while (kh + 1 < h_kv && u0 >= map.pref[kh + 1]) ++kh;
+#pragma unroll 1
+        for (int j = 0; j < n; ++j) {
+            while (kh + 1 < h_kv && u0 + j >= map.pref[kh + 1]) ++kh;
             if (kh != kh_cur) {
                 // every consumer warp sees every stage's KV head, so the
                 // named barriers inside the flushes match
@@ -705,8 +726,8 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                 st.init();
                 st.load_q(a.q, kh, qscale, lane);
             }
-            if ((int)(j & 1) != half) continue;
-            const int slot = (int)(j % ST);
+            if (j % C::HALVES != half) continue;
+            const int slot = j % ST;
             const uint32_t round = (uint32_t)(j / ST);
             const bool ok = mbar_wait(&full[slot], round & 1u, abort);
             if (!ok) {

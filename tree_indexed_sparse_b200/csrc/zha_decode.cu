@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__
     unsigned gepoch = 0;
     if (s_ok && grid_barrier(words + h_kv, nb, gepoch, abortw, a.status, &s_flag)) {
         stamp(a, a.t.D);
-        stage_map_init<false>(a, map);
+        stage_map_init<false, StageCfg<KT, HD>::TT>(a, map);
         if (router && warp < ACW) write_lists<G>(a, kh, tr);
         attn_stages<KT, HD, G, false>(a, map, smem, b, nb);
         stamp(a, a.t.D + 1);

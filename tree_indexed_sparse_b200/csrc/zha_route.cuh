@@ -261,14 +261,21 @@ __device__ __noinline__ void chunk_issue(const Level &L, int64_t c0, int64_t c1,
     }
     __syncwarp();
     unsigned char *dst = bufs + (size_t)buf * CH_BYTES;
+    // one copy per run of consecutive nodes inside each group of 32 slots:
+    // a run starts where the node does not follow its left neighbour's
 #pragma unroll 1
-    for (int i = lane; i < ns; i += 32) {
-        const int nd = cn[i];
-        if (nd < 0 || (i > 0 && cn[i - 1] >= 0 && cn[i - 1] + 1 == nd)) continue;
-        int len = 1;
-        while (i + len < ns && cn[i + len] == nd + len) ++len;
-        bulk_g2s(dst + (size_t)i * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES),
-                 &bars[buf]);
+    for (int i0 = 0; i0 < ns; i0 += 32) {
+        const int i = i0 + lane;
+        const int nd = i < ns ? cn[i] : -1;
+        const int left = __shfl_up_sync(FULL, nd, 1);
+        const bool start = nd >= 0 && (lane == 0 || left < 0 || left + 1 != nd);
+        const unsigned brk = __ballot_sync(FULL, start || nd < 0);  // where runs end
+        if (start) {
+            const unsigned after = lane == 31 ? 0u : (brk >> (lane + 1));
+            const int len = after ? __ffs(after) : 32 - lane;
+            bulk_g2s(dst + (size_t)i * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES),
+                     &bars[buf]);
+        }
     }
 }
 
@@ -833,11 +840,22 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
     }
     if (any_order) {
         unsigned long long *base = red + 72;
+        // mass of the boundary before this rank: lower ranks' sums (parallel
+        // loads, reduced per head in a fixed order)
+        unsigned long long x = 0ull;
+        if (team) {
+#pragma unroll 1
+            for (int t = tid; t < tr * G; t += GT) x += __ldcg(a.tsum + (int64_t)kh * SEG_CAP * G + t);
+        }
+#pragma unroll
+        for (int off = G; off < 32; off <<= 1) x += __shfl_xor_sync(FULL, x, off);
+        if ((tid & 31) < G) red[128 + (tid >> 5) * G + (tid & 31)] = x;
+        gsync();
         if (tid < G) {
             unsigned long long bsum = cut[tid].C;
-            if (team && cut[tid].mode == CUT_ORDER) {
+            if (cut[tid].mode == CUT_ORDER) {
 #pragma unroll 1
-                for (int r = 0; r < tr; ++r) bsum += __ldcg(a.tsum + ((int64_t)kh * SEG_CAP + r) * G + tid);
+                for (int w = 0; w < GT / 32; ++w) bsum += red[128 + w * G + tid];
             }
             base[tid] = bsum;
         }
@@ -915,16 +933,37 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
         }
     }
     if (team && !ts.sync()) return false;  // A
-    if (team && tid < G) {
+    if (team) {
+        // thread t < T*G loads rank t/G's (max, count) of head t%G; then a
+        // reduction over threads with equal t%G (fixed order)
         float m = -INFINITY;
         uint32_t c = 0u;
 #pragma unroll 1
-        for (int r = 0; r < T; ++r) {
-            m = fmaxf(m, __ldcg(a.tmax + ((int64_t)kh * SEG_CAP + r) * G + tid));
-            c += __ldcg(a.tcnt + ((int64_t)kh * SEG_CAP + r) * G + tid);
+        for (int t = tid; t < T * G; t += GT) {  // GT is a multiple of G: t % G == tid % G
+            m = fmaxf(m, __ldcg(a.tmax + (int64_t)kh * SEG_CAP * G + t));
+            c += __ldcg(a.tcnt + (int64_t)kh * SEG_CAP * G + t);
         }
-        cut[tid].M = m;
-        cut[tid].F = c;
+#pragma unroll
+        for (int off = G; off < 32; off <<= 1) {
+            m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+            c += __shfl_xor_sync(FULL, c, off);
+        }
+        if ((tid & 31) < G) {
+            wm[(tid >> 5) * G + (tid & 31)] = m;
+            wc[(tid >> 5) * G + (tid & 31)] = c;
+        }
+        gsync();
+        if (tid < G) {
+            float mm = -INFINITY;
+            uint32_t cc = 0u;
+#pragma unroll 1
+            for (int w = 0; w < GT / 32; ++w) {
+                mm = fmaxf(mm, wm[w * G + tid]);
+                cc += wc[w * G + tid];
+            }
+            cut[tid].M = mm;
+            cut[tid].F = cc;
+        }
     }
     const bool keep_all = !(a.p < 1.f);
     gsync();
