@@ -119,7 +119,8 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
 #pragma unroll 1
                 for (;;) {
                     uint32_t F[G];
-                    route_level<HD, R, G>(a, l, kh, 1, 0, S, Tp, Sp, smem, solo, F);
+                    int Tout;
+                    route_level<HD, R, G>(a, l, kh, 1, 0, S, Tp, Sp, smem, solo, F, Tout);
 #pragma unroll
                     for (int h = 0; h < G; ++h) vis[h] += F[h];
                     Tp = 1;
@@ -143,10 +144,11 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
             }
         } else {
             uint32_t F[G];
-            if (!route_level<HD, R, G>(a, l, kh, T, tr, S, Tp, Sp, smem, ts, F)) return false;
+            int Tout;
+            if (!route_level<HD, R, G>(a, l, kh, T, tr, S, Tp, Sp, smem, ts, F, Tout)) return false;
 #pragma unroll
             for (int h = 0; h < G; ++h) vis[h] += F[h];
-            Tp = T;
+            Tp = Tout;
             Sp = S;
             --l;
             if (l >= 1) S = load_segments(a, l + 1, kh, Tp, pref, scratch) * a.t.c;

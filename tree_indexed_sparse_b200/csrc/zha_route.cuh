@@ -279,30 +279,51 @@ __device__ __noinline__ void chunk_issue(const Level &L, int64_t c0, int64_t c1,
     }
 }
 
+// Sums over the warp of 8 rows x G heads of per-lane partial dots, v[row*G + h].
+// Afterwards lane l holds the sum of (row (l / G) % 8, head l % G): G = 4 is a
+// reduce-scatter of 32 values; G = 1 reduce-scatters 8 values over 8 lanes and
+// finishes with a butterfly over the groups of 8.  One fixed order each.
+template <int G>
+__device__ __forceinline__ float batch_sum(float (&v)[8 * G], int lane) {
+    if constexpr (G == 4) {
+        reduce_scatter<32>(v, lane);
+        return v[0];
+    } else {
+        reduce_scatter<8, 8>(v, lane);
+        float k = v[0];
+        k += __shfl_xor_sync(FULL, k, 8);
+        k += __shfl_xor_sync(FULL, k, 16);
+        return k;
+    }
+}
+
 // Score local slots [c0, c1) (global slot ids) of level L.  The slots go in
 // chunks of ScoreChunk::SLOTS through two shared-memory buffers: warp 0
 // bulk-copies the g rows of chunk k + 2 while all warps score chunk k from
-// shared memory (warp w takes rows w, w + 8, ... of the chunk; the plane
-// offsets b of its rows are loaded before the chunk lands).  Parent window:
-// ranks [k0, ...) in pid/pmk.  Writes L.sc / L.node at (s - L.s0) and folds
-// the maxima and counts per head into wm/wc[warp][h].
+// shared memory.  Warp w scores slots w, w + 8, ... of the chunk, 8 summary
+// rows at a time (one reduce-scatter per 8 rows), and keeps each node's
+// maximum over its planes in registers; the plane offsets b of its rows are
+// loaded before the chunk lands.  Parent window: ranks [k0, ...) in pid/pmk.
+// Writes L.sc / L.node at (s - L.s0) and folds the maxima and counts per head
+// into wm/wc[warp][h].
 template <int HD, int R, int G>
 __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64_t c0, int64_t c1, int64_t k0,
                                           const int32_t *pid, const uint8_t *pmk, unsigned char *smem, float *wm,
                                           uint32_t *wc) {
     static_assert(G == 1 || G == 4, "query heads per KV head");
+    static_assert(R == 1 || R % 8 == 0, "planes per node: 1 or a multiple of 8");
     using C = ScoreChunk<HD, R>;
     using SM = RouteSmem<G>;
     constexpr int VEC = HD / 32;
+    constexpr int SPW = C::SLOTS / 8;                    // slots per warp per chunk
+    constexpr int RPWC = SPW * R;                        // rows per warp per chunk
+    static_assert(C::SLOTS % 8 == 0 && RPWC % 8 == 0 && RPWC <= 32, "rows per warp");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int myh = G == 4 ? ((lane >> 3) & 3) : 0;
-    const bool writer = G == 4 ? ((lane & 7) == 0) : (lane == 0);
     const int kh = L.kh, l = L.l;
     unsigned char *bufs = smem + SM::off_chunk;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::off_bar);
     int32_t *cnode = reinterpret_cast<int32_t *>(smem + SM::off_cnode);
     uint8_t *cmask = smem + SM::off_cmask;
-    float *rowres = reinterpret_cast<float *>(smem + SM::off_rowres);
     float qs[G][VEC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -328,71 +349,100 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
             chunk_issue<HD, R, G>(L, c0, c1, k0, 1, pid, pmk, gb, c, clog, nl, bufs, bars, cnode, cmask, lane);
     }
     gsync();
-    float mloc = -INFINITY;  // this thread's head is tid % G throughout
-    uint32_t cloc = 0u;
+    const int hl = lane % G;             // head of this lane's sum
+    const int rl = (lane / G) % 8;       // row of this lane's sum within the batch
+    float mymax = -INFINITY;             // this lane's head's maximum (lanes < G report)
+    uint32_t mycnt = 0u;
 #pragma unroll 1
     for (int k = 0; k < nch; ++k) {
         const int buf = k & 1;
         const int64_t sb = c0 + (int64_t)k * C::SLOTS;
         const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
-        const int nrows = ns * R;
         const int32_t *cn = cnode + buf * CH_SLOTS_MAX;
         const uint8_t *cm = cmask + buf * CH_SLOTS_MAX;
-        // plane offsets of this warp's rows, one per lane
+        // plane offset of this warp's row `lane`: slot warp + 8 (lane / R), plane lane % R
         float bl = 0.f;
-        {
-            const int r = warp + 8 * lane;
-            if (lane < C::RPW && r < nrows) {
-                const int nd = cn[r / R];
-                if (nd >= 0) bl = __ldg(bb + (size_t)nd * R + r % R);
+        if (lane < RPWC) {
+            const int i = warp + 8 * (lane / R);
+            if (i < ns) {
+                const int nd = cn[i];
+                if (nd >= 0) bl = __ldg(bb + (size_t)nd * R + lane % R);
             }
         }
         if (!mbar_wait(&bars[buf], (uint32_t)((k >> 1) & 1), nullptr)) set_status(a.status, ZHA_TIMEOUT_CODE);
         const float *cb = reinterpret_cast<const float *>(bufs + (size_t)buf * CH_BYTES);
-#pragma unroll 2
-        for (int t = 0; t < C::RPW; ++t) {
-            const int r = warp + 8 * t;
-            if (r >= nrows) break;
-            float gs[VEC];
-            Vec<float, VEC>::load(cb + (size_t)r * HD + lane * VEC, gs);
-            float v[G];
+        float est = -INFINITY;
+#pragma unroll 1
+        for (int r0 = 0; r0 < RPWC; r0 += 8) {
+            // rows r0 .. r0 + 7 of this warp: slot warp + 8 (r / R), plane r % R
+            float v[8 * G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) v[h] = lane_dot<VEC>(qs[h], gs);
-            const float sum = head_sum<G>(v, lane);
-            const float b = __shfl_sync(FULL, bl, t);
-            if (writer) rowres[r * G + myh] = b + sum;
-        }
-        gsync();
-        // rows -> slots: est = max over the node's planes
-#pragma unroll 1
-        for (int idx = tid; idx < ns * G; idx += GT) {
-            const int i = idx / G, h = idx % G;
-            const int nd = cn[i];
-            float est = -INFINITY;
-#pragma unroll 1
-            for (int j = 0; j < R; ++j) est = fmaxf(est, rowres[(i * R + j) * G + h]);
-            const bool need = nd >= 0 && ((cm[i] >> h) & 1u);
-            const int64_t s = sb + i - L.s0;
-            L.sc[s * G + h] = need ? est : -INFINITY;
-            if (h == 0) L.node[s] = nd;
-            if (need) {
-                mloc = fmaxf(mloc, est);
-                cloc += 1u;
+            for (int q = 0; q < 8; ++q) {
+                const int r = r0 + q;
+                const int i = warp + 8 * (r / R);
+                float gs[VEC];
+                if (i < ns) {
+                    Vec<float, VEC>::load(cb + ((size_t)i * R + r % R) * HD + lane * VEC, gs);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) gs[e] = 0.f;
+                }
+#pragma unroll
+                for (int h = 0; h < G; ++h) v[q * G + h] = lane_dot<VEC>(qs[h], gs);
+            }
+            const float sum = batch_sum<G>(v, lane);
+            const int r = r0 + rl;
+            const float e = __shfl_sync(FULL, bl, r) + sum;
+            if constexpr (R == 1) {
+                // every row is its own slot
+                const int i = warp + 8 * r;
+                if (i < ns && (G == 4 || lane < 8)) {
+                    const int nd = cn[i];
+                    const bool need = nd >= 0 && ((cm[i] >> hl) & 1u);
+                    const int64_t s = sb + i - L.s0;
+                    L.sc[s * G + hl] = need ? e : -INFINITY;
+                    if (hl == 0) L.node[s] = nd;
+                    if (need) {
+                        mymax = fmaxf(mymax, e);
+                        mycnt += 1u;
+                    }
+                }
+            } else {
+                // the 8 rows belong to one slot: max over them, then over batches
+                float m8 = e;
+#pragma unroll
+                for (int off = G; off < 8 * G; off <<= 1) m8 = fmaxf(m8, __shfl_xor_sync(FULL, m8, off));
+                est = fmaxf(est, m8);
+                if ((r0 + 8) % R == 0) {
+                    const int i = warp + 8 * (r0 / R);
+                    if (i < ns && lane < G) {
+                        const int nd = cn[i];
+                        const bool need = nd >= 0 && ((cm[i] >> hl) & 1u);
+                        const int64_t s = sb + i - L.s0;
+                        L.sc[s * G + hl] = need ? est : -INFINITY;
+                        if (hl == 0) L.node[s] = nd;
+                        if (need) {
+                            mymax = fmaxf(mymax, est);
+                            mycnt += 1u;
+                        }
+                    }
+                    est = -INFINITY;
+                }
             }
         }
-        gsync();
+        gsync();  // chunk k's buffer is free
         if (warp == 0 && k + 2 < nch)
             chunk_issue<HD, R, G>(L, c0, c1, k0, k + 2, pid, pmk, gb, c, clog, nl, bufs, bars, cnode, cmask, lane);
     }
-    // per-warp maxima and counts of each head (lanes with equal tid % G)
+    // per-warp maxima and counts of each head: lanes with equal head
 #pragma unroll
     for (int off = G; off < 32; off <<= 1) {
-        mloc = fmaxf(mloc, __shfl_xor_sync(FULL, mloc, off));
-        cloc += __shfl_xor_sync(FULL, cloc, off);
+        mymax = fmaxf(mymax, __shfl_xor_sync(FULL, mymax, off));
+        mycnt += __shfl_xor_sync(FULL, mycnt, off);
     }
     if (lane < G) {
-        wm[warp * G + lane] = fmaxf(wm[warp * G + lane], mloc);
-        wc[warp * G + lane] += cloc;
+        wm[warp * G + lane] = fmaxf(wm[warp * G + lane], mymax);
+        wc[warp * G + lane] += mycnt;
     }
     gsync();
 }
@@ -871,7 +921,7 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
 // Returns false when a team barrier gave up.
 template <int HD, int R, int G>
 __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, int tr, int64_t S, int Tp, int64_t Sp,
-                                         unsigned char *smem, TeamSync &ts, uint32_t (&F)[G]) {
+                                         unsigned char *smem, TeamSync &ts, uint32_t (&F)[G], int &Tout) {
     using SM = RouteSmem<G>;
     HeadCut *cut = reinterpret_cast<HeadCut *>(smem + SM::off_cut);
     uint32_t *pref = reinterpret_cast<uint32_t *>(smem + SM::off_pref);
@@ -889,6 +939,7 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
     L.n = seg_start(S, T, tr + 1) - L.s0;
     L.Tp = Tp;
     L.Sp = Sp;
+    Tout = T;
     if (L.n > LOC_CAP) {
         const int64_t base = (int64_t)kh * a.score_cap + L.s0;
         L.sc = a.scores + base * G;
@@ -966,6 +1017,7 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
         }
     }
     const bool keep_all = !(a.p < 1.f);
+    const bool solo = L.T == 1;
     gsync();
     if (tid < G) {
         HeadCut &H = cut[tid];
@@ -986,7 +1038,7 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
             L.keep[i] = (uint8_t)kb;
         }
         gsync();
-    } else if (!team && L.n <= SOLO_MAX) {
+    } else if (solo && L.n <= SOLO_MAX) {
         solo_cut<G>(L, cut, reinterpret_cast<unsigned long long *>(smem + SM::off_hm), a.p);
     } else {
         if (!hist_cut<G>(a, L, smem, ts)) return false;
