@@ -196,6 +196,7 @@ def step_bytes(w, trace_ids, trace_cnt, n_tokens):
     route = 0
     attn = 0
     slots_total = 0
+    slots_level = [0] * (D + 1)
     for kh in range(w.h_kv):
         heads = range(kh * G, (kh + 1) * G)
         for level in range(D, 0, -1):
@@ -209,6 +210,7 @@ def step_bytes(w, trace_ids, trace_cnt, n_tokens):
                 nodes = sum(min(c, nb - k * c) for k in kept)
             route += nodes * node
             slots_total += nodes
+            slots_level[level] += nodes
         leaves = set()
         sink = False
         for h in heads:
@@ -219,7 +221,7 @@ def step_bytes(w, trace_ids, trace_cnt, n_tokens):
         toks = sum(min(c, n_tokens - lf * c) for lf in leaves) + (1 if sink and 0 not in leaves else 0)
         attn += toks * 2 * d * e
     qo = w.h_q * d * 8
-    return route, attn + qo, slots_total
+    return route, attn + qo, slots_total, slots_level
 
 
 def append_bytes(w, n_after):
@@ -294,8 +296,8 @@ def run_zha(args, rank, world, local):
             ids = tr_ids.cpu().numpy()
             cnt = tr_cnt.cpu().numpy()
             n_now = w.n_tokens + i + 1
-            rb, ab, slots = step_bytes(w, ids, cnt, n_now)
-            per_step.append((rb, ab, append_bytes(w, n_now), slots, n_now))
+            rb, ab, slots, slots_level = step_bytes(w, ids, cnt, n_now)
+            per_step.append((rb, ab, append_bytes(w, n_now), slots, n_now, slots_level))
             leaves_per_head.append(n_leaf.float().mean().item())
             vis_per_head.append(visited.float().mean().item())
     ref_out = out.clone()
@@ -306,7 +308,7 @@ def run_zha(args, rank, world, local):
     stamps = torch.zeros(w.D + 3, dtype=torch.int64, device=dev)
     zha.zha_set_phase_timer(cache.ctx, stamps)
     ea, eb, ec = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-    t_step, t_app, t_route, t_attn, t_merge = [], [], [], [], []
+    t_step, t_app, t_route, t_attn, t_merge, t_lvl = [], [], [], [], [], []
     clocks = Clocks(local)
     for i in range(W):
         flush.zero_()
@@ -334,6 +336,9 @@ def run_zha(args, rank, world, local):
         t_route.append(dec - (ns[w.D + 2] - ns[w.D]) * 1e-6)
         t_attn.append((ns[w.D + 1] - ns[w.D]) * 1e-6)
         t_merge.append((ns[w.D + 2] - ns[w.D + 1]) * 1e-6)
+        # levels D .. 1 as seen by the first CTA of KV head 0 (kernel start to
+        # the end of level D, ..., end of level 2 to the end of the routing)
+        t_lvl.append([(ns[i + 1] - ns[i]) * 1e-3 for i in range(w.D)])
     torch.cuda.synchronize()
     wall = time.time() - wall0
     if world > 1:
@@ -359,6 +364,7 @@ def run_zha(args, rank, world, local):
         "attention": {"us": 1e3 * statistics.mean(t_attn), "bytes": statistics.mean(attn_b),
                       "gbs": sum(attn_b) / (sum(t_attn) * 1e-3) / 1e9},
         "merge": {"us": 1e3 * statistics.mean(t_merge)},
+        "route_levels_us": {f"level_{w.D - i}": statistics.mean(x[i] for x in t_lvl) for i in range(w.D)},
     }
     # the decode is one kernel (routing levels + attention + merge): its
     # algorithmic bytes over its event-timed duration
@@ -438,6 +444,8 @@ def run_zha(args, rank, world, local):
                     "nodes_visited_per_head": statistics.mean(vis_per_head),
                     "keys_touched_frac": statistics.mean(leaves_per_head) * w.c / w.n_tokens,
                     "union_slots_per_step": statistics.mean(s[3] for s in per_step),
+                    "union_slots_per_level": {f"level_{lv}": statistics.mean(s[5][lv] for s in per_step)
+                                              for lv in range(w.D, 0, -1)},
                     "timed_pass_reproduces_traced": bool(same)},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk,

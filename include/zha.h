@@ -212,10 +212,11 @@ int zha_device_status(zha_ctx *ctx, int32_t *out_status, void *stream);
  * Profiling hook: zha_decode runs as one kernel; when a buffer is set, the
  * kernel writes the GPU global timer (nanoseconds) at its phase boundaries:
  *   d_ns  caller-owned device buffer of D + 3 int64 (8-byte aligned), kept
- *         alive while set; NULL clears.  d_ns[0] = start, d_ns[D] = end of
- *         the routing (every level), d_ns[D + 1] = end of this CTA's share of
- *         the attention over the kept tokens, d_ns[D + 2] = end of the merge;
- *         d_ns[1 .. D-1] are not written.
+ *         alive while set; NULL clears.  d_ns[0] = start, d_ns[i] for
+ *         i = 1 .. D-1 = end of routing level D - i + 1 as seen by the first
+ *         CTA of KV head 0, d_ns[D] = end of the routing (every level, every
+ *         KV head), d_ns[D + 1] = end of that CTA's share of the attention
+ *         over the kept tokens, d_ns[D + 2] = end of the merge.
  * No effect on results.
  */
 int zha_set_phase_timer(zha_ctx *ctx, int64_t *d_ns);

@@ -123,6 +123,7 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
                     route_level<HD, R, G>(a, l, kh, 1, 0, S, Tp, Sp, smem, solo, F, Tout);
 #pragma unroll
                     for (int h = 0; h < G; ++h) vis[h] += F[h];
+                    if (l > 1) stamp(a, D - l + 1);
                     Tp = 1;
                     Sp = S;
                     --l;
@@ -148,6 +149,7 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
             if (!route_level<HD, R, G>(a, l, kh, T, tr, S, Tp, Sp, smem, ts, F, Tout)) return false;
 #pragma unroll
             for (int h = 0; h < G; ++h) vis[h] += F[h];
+            if (l > 1) stamp(a, D - l + 1);
             Tp = Tout;
             Sp = S;
             --l;

@@ -737,6 +737,12 @@ __device__ __noinline__ void order_own(const Level &L, const HeadCut *cut, const
     gsync();
 }
 
+// Keep bits of local slot i.  Bits set by atomics live at L2 when the slots
+// overflow shared memory, so global keep bits are read around L1.
+__device__ __forceinline__ uint32_t keep_at(const Level &L, int64_t i) {
+    return L.n > LOC_CAP ? (uint32_t)__ldcg(L.keep + i) : (uint32_t)L.keep[i];
+}
+
 // Write this CTA's kept slots (ascending) at the start of its slot range,
 // with per-rank counts.
 template <int G>
@@ -749,7 +755,7 @@ __device__ __noinline__ void write_segment(const Decode &a, const Level &L, uint
     for (int h = 0; h < G; ++h) hc[h] = 0u;
 #pragma unroll 1
     for (int64_t i = i0; i < i1; ++i) {
-        const uint32_t k = L.keep[i];
+        const uint32_t k = keep_at(L, i);
         mine += k != 0u;
 #pragma unroll
         for (int h = 0; h < G; ++h) hc[h] += (k >> h) & 1u;
@@ -761,7 +767,7 @@ __device__ __noinline__ void write_segment(const Decode &a, const Level &L, uint
     uint8_t *msk = a.kept_mask[L.l - 1] + dst;
 #pragma unroll 1
     for (int64_t i = i0; i < i1; ++i) {
-        const uint32_t k = L.keep[i];
+        const uint32_t k = keep_at(L, i);
         if (k) {
             ids[at] = L.node[i];
             msk[at] = (uint8_t)k;
