@@ -275,41 +275,189 @@ __global__ void __launch_bounds__(BUILD_THREADS) k_build_parents(Tree t, int lev
     }
 }
 
-// One warp per KV head: store the new row, then recompute the leaf holding it
-// and every ancestor.  t.n_tokens and t.n_level already count the new token.
+// Append, one plane at a time: warp j of the KV head's CTA recomputes plane
+// j (reference query r_j) of the leaf holding the new row and of every
+// ancestor.  Each plane of a node depends only on that plane's reference
+// query and on the children's rows, so the planes are independent; every sum
+// below takes the same order as in LeafOps / ParentOps (a dot product is a
+// per-lane fmaf chain and a 32-lane butterfly, here as a reduce-scatter of 32
+// dot products; log-sum-exp and weighted sums run over tokens / children in
+// order), so the appended tree is bit-identical to a build.
 template <typename KT, int HD, int R>
-__global__ void __launch_bounds__(32) k_append(Tree t, const KT *__restrict__ knew, const KT *__restrict__ vnew) {
+struct PlaneOps {
+    static constexpr int VEC = HD / 32;
+
+    // Leaf n of this head, plane j: tokens [tok0, tok0 + ntok).  sh: warp-
+    // private shared scratch of ntok floats.
+    static __device__ void leaf(const KT *__restrict__ Kh, int64_t tok0, int ntok, const float (&r)[VEC], int j,
+                                float scale, float *__restrict__ gL, float *__restrict__ bL, float *__restrict__ mL,
+                                int64_t n, float *sh, int lane) {
+        for (int i0 = 0; i0 < ntok; i0 += 32) {
+            float v[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                float k[VEC];
+                if (i0 + t < ntok) {
+                    Vec<KT, VEC>::load(Kh + (tok0 + i0 + t) * HD + lane * VEC, k);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) k[e] = 0.f;
+                }
+                v[t] = lane_dot<VEC>(r, k);
+            }
+            reduce_scatter<32>(v, lane);
+            if (i0 + lane < ntok) sh[i0 + lane] = v[0] * scale;
+        }
+        __syncwarp();
+        float m = 0.f;
+        if (lane == 0) {
+            float mx = -INFINITY;
+            for (int i = 0; i < ntok; ++i) mx = fmaxf(mx, sh[i]);
+            float sum = 0.f;
+            for (int i = 0; i < ntok; ++i) sum += expf(sh[i] - mx);
+            m = mx + logf(sum);
+            mL[n * R + j] = m;
+        }
+        m = __shfl_sync(FULL, m, 0);
+        __syncwarp();
+        for (int i = lane; i < ntok; i += 32) sh[i] = expf(sh[i] - m);
+        __syncwarp();
+        float acc[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+        for (int i = 0; i < ntok; ++i) {
+            float k[VEC];
+            Vec<KT, VEC>::load(Kh + (tok0 + i) * HD + lane * VEC, k);
+            const float w = sh[i];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] = fmaf(w, k[e], acc[e]);
+        }
+        float *dst = gL + (n * R + j) * HD + lane * VEC;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) dst[e] = acc[e];
+        const float dot = warp_sum(lane_dot<VEC>(r, acc));
+        if (lane == 0) bL[n * R + j] = m - scale * dot;
+        __syncwarp();
+    }
+
+    // Node n of this level, plane j, from its nch children (rows ch0 ..
+    // ch0 + nch - 1 of the level below).  sh: warp-private scratch of nch floats.
+    static __device__ void parent(const float *__restrict__ gC, const float *__restrict__ bC, int64_t ch0, int nch,
+                                  const float (&r)[VEC], int j, float scale, float *__restrict__ gP,
+                                  float *__restrict__ bP, float *__restrict__ mP, int64_t n, float *sh, int lane) {
+        // child estimates at r_j: max over the child's planes j'
+        constexpr int CPB = 32 / R;  // children per batch of 32 dot products
+        for (int c0 = 0; c0 < nch; c0 += CPB) {
+            float v[32];
+#pragma unroll
+            for (int t = 0; t < CPB; ++t) {
+#pragma unroll
+                for (int jp = 0; jp < R; ++jp) {
+                    float gs[VEC];
+                    if (c0 + t < nch) {
+                        Vec<float, VEC>::load(gC + ((ch0 + c0 + t) * R + jp) * HD + lane * VEC, gs);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < VEC; ++e) gs[e] = 0.f;
+                    }
+                    v[t * R + jp] = lane_dot<VEC>(r, gs);
+                }
+            }
+            reduce_scatter<32>(v, lane);
+            const int t = lane / R, jp = lane % R;
+            float val = -INFINITY;
+            if (c0 + t < nch) val = bC[(ch0 + c0 + t) * R + jp] + scale * v[0];
+#pragma unroll
+            for (int off = 1; off < R; off <<= 1) val = fmaxf(val, __shfl_xor_sync(FULL, val, off));
+            if (jp == 0 && c0 + t < nch) sh[c0 + t] = val;
+        }
+        __syncwarp();
+        float m = 0.f;
+        if (lane == 0) {
+            float mx = -INFINITY;
+            for (int ch = 0; ch < nch; ++ch) mx = fmaxf(mx, sh[ch]);
+            float sum = 0.f;
+            for (int ch = 0; ch < nch; ++ch) sum += expf(sh[ch] - mx);
+            m = mx + logf(sum);
+            for (int ch = 0; ch < nch; ++ch) sh[ch] = expf(sh[ch] - m);
+            mP[n * R + j] = m;
+        }
+        m = __shfl_sync(FULL, m, 0);
+        __syncwarp();
+        float acc[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+        for (int ch = 0; ch < nch; ++ch) {
+            float gs[VEC];
+            Vec<float, VEC>::load(gC + ((ch0 + ch) * R + j) * HD + lane * VEC, gs);
+            const float w = sh[ch];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] = fmaf(w, gs[e], acc[e]);
+        }
+        float *dst = gP + (n * R + j) * HD + lane * VEC;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) dst[e] = acc[e];
+        const float dot = warp_sum(lane_dot<VEC>(r, acc));
+        if (lane == 0) bP[n * R + j] = m - scale * dot;
+        __syncwarp();
+    }
+};
+
+// One CTA per KV head, one warp per plane: store the new row, prefetch every
+// ancestor's children into L2, then recompute the leaf holding the row and
+// every ancestor, a level at a time.  t.n_tokens and t.n_level already count
+// the new token.
+template <typename KT, int HD, int R>
+__global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict__ knew, const KT *__restrict__ vnew) {
     extern __shared__ __align__(16) float bsm[];
     constexpr int VEC = HD / 32;
-    const int lane = threadIdx.x;
+    const int lane = threadIdx.x & 31, j = threadIdx.x >> 5;
     const int kh = blockIdx.x;
     const int64_t pos = t.n_tokens - 1;
     KT *Kh = const_cast<KT *>(reinterpret_cast<const KT *>(t.K)) + (int64_t)kh * t.kv_cap * HD;
     KT *Vh = const_cast<KT *>(reinterpret_cast<const KT *>(t.V)) + (int64_t)kh * t.kv_cap * HD;
-    for (int e = lane; e < HD; e += 32) {
-        Kh[pos * HD + e] = knew[kh * HD + e];
-        Vh[pos * HD + e] = vnew[kh * HD + e];
+    if (j == 0) {
+        for (int e = lane; e < HD; e += 32) {
+            Kh[pos * HD + e] = knew[kh * HD + e];
+            Vh[pos * HD + e] = vnew[kh * HD + e];
+        }
     }
-    __syncwarp();
-    float rj[R][VEC];
-    load_ref<HD, R>(t.ref + (int64_t)kh * R * HD, rj, lane);
+    // the children of every ancestor: 128-byte lines into L2
+    {
+        int64_t n = pos / t.c;
+        for (int level = 2; level <= t.D; ++level) {
+            n /= t.c;
+            const int64_t ch0 = n * t.c;
+            const int nch = (int)min((int64_t)t.c, (int64_t)t.n_level[level - 2] - ch0);
+            const float *g = t.g[level - 2] + ((int64_t)kh * t.node_cap[level - 2] + ch0) * R * HD;
+            const int64_t lines = ((int64_t)nch * R * HD * 4 + 127) / 128;
+            for (int64_t i = threadIdx.x; i < lines; i += blockDim.x)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<const char *>(g) + i * 128));
+        }
+    }
+    __syncthreads();
+    float r[VEC];
+    Vec<float, VEC>::load(t.ref + ((int64_t)kh * R + j) * HD + lane * VEC, r);
+    float *sh = bsm + j * (t.c > 32 ? t.c : 32);
     int64_t n = pos / t.c;
     {
         const int64_t tok0 = n * t.c;
         const int ntok = (int)(t.n_tokens - tok0);
         const int64_t nc = t.node_cap[0];
-        LeafOps<KT, HD, R>::tile(Kh, tok0, ntok, t.c, rj, t.scale, t.g[0] + (int64_t)kh * nc * R * HD,
-                                 t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, bsm, lane);
+        PlaneOps<KT, HD, R>::leaf(Kh, tok0, ntok, r, j, t.scale, t.g[0] + (int64_t)kh * nc * R * HD,
+                                  t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, n, sh, lane);
     }
+    __syncthreads();
     for (int level = 2; level <= t.D; ++level) {
         n /= t.c;
         const int64_t ch0 = n * t.c;
         const int nch = (int)min((int64_t)t.c, (int64_t)t.n_level[level - 2] - ch0);
         const int64_t capP = t.node_cap[level - 1], capC = t.node_cap[level - 2];
-        ParentOps<HD, R>::node(t.g[level - 2] + (int64_t)kh * capC * R * HD, t.b[level - 2] + (int64_t)kh * capC * R,
-                               ch0, nch, rj, t.scale, t.g[level - 1] + (int64_t)kh * capP * R * HD,
-                               t.b[level - 1] + (int64_t)kh * capP * R, t.m[level - 1] + (int64_t)kh * capP * R,
-                               n, bsm, lane);
+        PlaneOps<KT, HD, R>::parent(t.g[level - 2] + (int64_t)kh * capC * R * HD, t.b[level - 2] + (int64_t)kh * capC * R,
+                                    ch0, nch, r, j, t.scale, t.g[level - 1] + (int64_t)kh * capP * R * HD,
+                                    t.b[level - 1] + (int64_t)kh * capP * R, t.m[level - 1] + (int64_t)kh * capP * R, n,
+                                    sh, lane);
+        __syncthreads();
     }
 }
 
@@ -350,18 +498,15 @@ static cudaError_t build_impl(const Tree &t, cudaStream_t s, int n_sm) {
 
 template <typename KT, int HD, int R>
 static cudaError_t append_impl(const Tree &t, const void *k, const void *v, cudaStream_t s) {
-    const int tt = leaf_tile_tokens(t.c, R);
-    const int rows = tt > t.c ? tt : t.c;
-    size_t smem = (size_t)(rows * R + (rows / t.c + 1) * R) * sizeof(float);
-    const size_t psmem = (size_t)(t.c * R + R) * sizeof(float);
-    if (psmem > smem) smem = psmem;
+    // per plane warp: one score per token of a leaf, or one estimate per child
+    const size_t smem = (size_t)R * (t.c > 32 ? t.c : 32) * sizeof(float);
     static size_t attr = 0;
     if (smem > attr) {
         cudaError_t err = cudaFuncSetAttribute(k_append<KT, HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
         attr = smem;
     }
-    k_append<KT, HD, R><<<t.h_kv, 32, smem, s>>>(t, reinterpret_cast<const KT *>(k), reinterpret_cast<const KT *>(v));
+    k_append<KT, HD, R><<<t.h_kv, 32 * R, smem, s>>>(t, reinterpret_cast<const KT *>(k), reinterpret_cast<const KT *>(v));
     return cudaGetLastError();
 }
 
