@@ -93,8 +93,8 @@ struct RouteSmem {
     static constexpr size_t off_bar = off_red + GT * 8;                   // [2] u64 chunk barriers
     static constexpr size_t off_cnode = off_bar + 16;                     // [2][CH_SLOTS_MAX] i32
     static constexpr size_t off_cmask = off_cnode + 2 * CH_SLOTS_MAX * 4; // [2][CH_SLOTS_MAX] u8
-    static constexpr size_t off_rowres = off_cmask + 2 * CH_SLOTS_MAX;    // [CH_ROWS_MAX][G] f32
-    static constexpr size_t off_misc = off_rowres + (size_t)CH_ROWS_MAX * G * 4;  // u32 counters
+    static constexpr size_t off_bpl = (off_cmask + 2 * CH_SLOTS_MAX + 15) / 16 * 16;  // [2][CH_ROWS_MAX] f32 plane offsets
+    static constexpr size_t off_misc = off_bpl + (size_t)2 * CH_ROWS_MAX * 4;  // u32 counters
     static constexpr size_t bytes = off_misc + 64;
     static_assert(SOLO_MAX * G * 8 <= G * NB * 8, "solo masses fit the histogram area");
     static_assert(off_u % 16 == 0, "bulk copies land on 16-byte boundaries");
@@ -227,9 +227,9 @@ struct ScoreChunk {
 // (one copy per run of consecutive nodes) into chunk buffer k & 1.
 template <int HD, int R, int G>
 __device__ __noinline__ void chunk_issue(const Level &L, int64_t c0, int64_t c1, int64_t k0, int k, const int32_t *pid,
-                                            const uint8_t *pmk, const float *gb, int c, int clog, int32_t nl,
-                                            unsigned char *bufs, uint64_t *bars, int32_t *cnode, uint8_t *cmask,
-                                            int lane) {
+                                            const uint8_t *pmk, const float *gb, const float *bb, int c, int clog,
+                                            int32_t nl, unsigned char *bufs, uint64_t *bars, int32_t *cnode,
+                                            uint8_t *cmask, float *bpl, int lane) {
     using C = ScoreChunk<HD, R>;
     const int buf = k & 1;
     const int64_t sb = c0 + (int64_t)k * C::SLOTS;
@@ -276,7 +276,19 @@ __device__ __noinline__ void chunk_issue(const Level &L, int64_t c0, int64_t c1,
             bulk_g2s(dst + (size_t)i * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES),
                      &bars[buf]);
         }
+        // the slot's plane offsets, asynchronously, completing on the same barrier
+        if (nd >= 0) {
+            float *pb = bpl + buf * CH_ROWS_MAX + (size_t)i * R;
+            if constexpr (R % 4 == 0) {
+#pragma unroll
+                for (int j = 0; j < R; j += 4) cp_async16(pb + j, bb + (size_t)nd * R + j);
+            } else {
+#pragma unroll
+                for (int j = 0; j < R; ++j) cp_async4(pb + j, bb + (size_t)nd * R + j);
+            }
+        }
     }
+    cp_async_arrive_noinc(&bars[buf]);
 }
 
 // Sums over the warp of 8 rows x G heads of per-lane partial dots, v[row*G + h].
@@ -337,16 +349,18 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
     const int c = a.t.c, clog = a.t.c_log2;
     const int32_t nl = a.t.n_level[l - 1];
     const int nch = (int)((c1 - c0 + C::SLOTS - 1) / C::SLOTS);
+    float *bpl = reinterpret_cast<float *>(smem + SM::off_bpl);
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        // the expect-tx arrive plus one cp.async arrive per lane of warp 0
+        mbar_init(&bars[0], 1 + 32);
+        mbar_init(&bars[1], 1 + 32);
         mbar_init_fence();
     }
     gsync();
     if (warp == 0) {
-        chunk_issue<HD, R, G>(L, c0, c1, k0, 0, pid, pmk, gb, c, clog, nl, bufs, bars, cnode, cmask, lane);
+        chunk_issue<HD, R, G>(L, c0, c1, k0, 0, pid, pmk, gb, bb, c, clog, nl, bufs, bars, cnode, cmask, bpl, lane);
         if (nch > 1)
-            chunk_issue<HD, R, G>(L, c0, c1, k0, 1, pid, pmk, gb, c, clog, nl, bufs, bars, cnode, cmask, lane);
+            chunk_issue<HD, R, G>(L, c0, c1, k0, 1, pid, pmk, gb, bb, c, clog, nl, bufs, bars, cnode, cmask, bpl, lane);
     }
     gsync();
     const int hl = lane % G;             // head of this lane's sum
@@ -360,16 +374,13 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
         const int32_t *cn = cnode + buf * CH_SLOTS_MAX;
         const uint8_t *cm = cmask + buf * CH_SLOTS_MAX;
+        if (!mbar_wait(&bars[buf], (uint32_t)((k >> 1) & 1), nullptr)) set_status(a.status, ZHA_TIMEOUT_CODE);
         // plane offset of this warp's row `lane`: slot warp + 8 (lane / R), plane lane % R
         float bl = 0.f;
         if (lane < RPWC) {
             const int i = warp + 8 * (lane / R);
-            if (i < ns) {
-                const int nd = cn[i];
-                if (nd >= 0) bl = __ldg(bb + (size_t)nd * R + lane % R);
-            }
+            if (i < ns && cn[i] >= 0) bl = bpl[buf * CH_ROWS_MAX + i * R + lane % R];
         }
-        if (!mbar_wait(&bars[buf], (uint32_t)((k >> 1) & 1), nullptr)) set_status(a.status, ZHA_TIMEOUT_CODE);
         const float *cb = reinterpret_cast<const float *>(bufs + (size_t)buf * CH_BYTES);
         float est = -INFINITY;
 #pragma unroll 1
@@ -432,7 +443,8 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         }
         gsync();  // chunk k's buffer is free
         if (warp == 0 && k + 2 < nch)
-            chunk_issue<HD, R, G>(L, c0, c1, k0, k + 2, pid, pmk, gb, c, clog, nl, bufs, bars, cnode, cmask, lane);
+            chunk_issue<HD, R, G>(L, c0, c1, k0, k + 2, pid, pmk, gb, bb, c, clog, nl, bufs, bars, cnode, cmask, bpl,
+                                  lane);
     }
     // per-warp maxima and counts of each head: lanes with equal head
 #pragma unroll
@@ -532,16 +544,24 @@ __device__ __noinline__ void local_hist(const Level &L, const HeadCut *cut, int 
         hm[i] = 0ull;
     }
     gsync();
+    // GT is a multiple of G: every entry this thread visits belongs to head tid % G
+    const int h = (int)(threadIdx.x % G);
+    const HeadCut &H = cut[h];
+    if (H.mode == CUT_OPEN && H.rounds == r) {
+        const int64_t total = L.n * G;
 #pragma unroll 1
-    for (int64_t idx = threadIdx.x; idx < L.n * G; idx += GT) {
-        const int h = (int)(idx % G);
-        const HeadCut &H = cut[h];
-        if (H.mode != CUT_OPEN || H.rounds != r) continue;
-        const float e = L.sc[idx];
-        if (e == -INFINITY || path_cmp(H, e, r) != 0) continue;
-        const int b = round_bucket(H, e, r);
-        atomicAdd(&hc[h * NB + b], 1u);
-        atomicAdd(&hm[h * NB + b], mass_fx(expf(e - H.M)));
+        for (int64_t i0 = threadIdx.x; i0 < total; i0 += 4 * GT) {
+            float e[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) e[u] = i0 + u * GT < total ? L.sc[i0 + u * GT] : -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (e[u] == -INFINITY || path_cmp(H, e[u], r) != 0) continue;
+                const int b = round_bucket(H, e[u], r);
+                atomicAdd(&hc[h * NB + b], 1u);
+                atomicAdd(&hm[h * NB + b], mass_fx(expf(e[u] - H.M)));
+            }
+        }
     }
     gsync();
 }
@@ -632,10 +652,13 @@ __device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsign
     for (int64_t it = 0; it < iters; ++it) {
         const int64_t i = it * GT + threadIdx.x;
         uint32_t kbits = 0u;
-#pragma unroll 1
+        float ev[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) ev[h] = i < L.n ? L.sc[i * G + h] : -INFINITY;
+#pragma unroll
         for (int h = 0; h < G; ++h) {
             const HeadCut &H = cut[h];
-            const float e = i < L.n ? L.sc[i * G + h] : -INFINITY;
+            const float e = ev[h];
             bool cand = false;
             unsigned long long w = 0ull;
             if (e != -INFINITY) {
@@ -718,7 +741,7 @@ __device__ __noinline__ void order_own(const Level &L, const HeadCut *cut, const
         const HeadCut &H = cut[h];
         if (H.mode != CUT_ORDER) continue;
         unsigned long long mine = 0ull;
-#pragma unroll 1
+#pragma unroll 4
         for (int64_t i = i0; i < i1; ++i) {
             const float e = L.sc[i * G + h];
             if (e != -INFINITY && path_cmp(H, e, H.rounds) == 0) mine += mass_fx(expf(e - H.M));
@@ -753,7 +776,7 @@ __device__ __noinline__ void write_segment(const Decode &a, const Level &L, uint
     uint32_t hc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) hc[h] = 0u;
-#pragma unroll 1
+#pragma unroll 4
     for (int64_t i = i0; i < i1; ++i) {
         const uint32_t k = keep_at(L, i);
         mine += k != 0u;
@@ -765,7 +788,7 @@ __device__ __noinline__ void write_segment(const Decode &a, const Level &L, uint
     const int64_t dst = (int64_t)L.kh * a.slot_cap[L.l - 1] + L.s0;
     int32_t *ids = a.kept_ids[L.l - 1] + dst;
     uint8_t *msk = a.kept_mask[L.l - 1] + dst;
-#pragma unroll 1
+#pragma unroll 4
     for (int64_t i = i0; i < i1; ++i) {
         const uint32_t k = keep_at(L, i);
         if (k) {
