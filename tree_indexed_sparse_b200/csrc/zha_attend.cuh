@@ -481,6 +481,14 @@ struct StageMap {
         }
         return (int64_t)S1[kh] * lo / T + (k - p[lo]);
     }
+    // The same for a rank k not below the one `r` was found for: advance r
+    // (the segment holding the last rank looked up) and return the position.
+    __device__ int64_t leaf_at_from(int kh, int64_t k, int &r) const {
+        const uint32_t *p = spref + soff[kh];
+        const int T = T1[kh];
+        while (r + 1 < T && (int64_t)p[r + 1] <= k) ++r;
+        return (int64_t)S1[kh] * r / T + (k - p[r]);
+    }
 };
 
 // Fill the stage map; all threads of the CTA call it, then it is valid after
@@ -617,9 +625,11 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                     win_kh = kh;
                     win_k0 = kf;
                     const int64_t kbase = (int64_t)kh * a.slot_cap[0];
+                    // ranks kf + lane, + 32, ...: the segment only moves forward
+                    int rseg = 0;
 #pragma unroll 4
                     for (int i = lane; i < nwin; i += 32) {
-                        const int64_t at = kbase + map.leaf_at(kh, kf + i);
+                        const int64_t at = kbase + map.leaf_at_from(kh, kf + i, rseg);
                         win_ids[i] = __ldcg(a.kept_ids[0] + at);
                         win_msk[i] = __ldcg(a.kept_mask[0] + at);
                     }
@@ -628,49 +638,54 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
             }
             // rows of this lane's group: flattened positions ug .. ug + GR - 1
             const int ug = t0 + gi * GR;
-            int row[GR];
-            uint32_t nvalid = 0u;
+            const unsigned char *src = isV ? Vh : Kh;
+            unsigned char *dst = sK + (isV ? C::HALF : 0) + gi * C::GS;
+            uint32_t nvalid = 0u;  // the group's token slots that hold a row: a prefix of the group
             if (DENSE) {
+                nvalid = act ? (uint32_t)max(0, min(GR, N - ug)) : 0u;
+                if (act && !isV) {
 #pragma unroll
-                for (int w = 0; w < GR; ++w) {
-                    row[w] = (act && ug + w < N) ? ug + w : -1;
-                    if (act && !isV) mt[gi * GR + w] = row[w] >= 0 ? 0xffu : 0u;
+                    for (int w = 0; w < GR; w += 4)
+                        *reinterpret_cast<uint32_t *>(mt + gi * GR + w) =
+                            (w + 0 < (int)nvalid ? 0xffu : 0u) | (w + 1 < (int)nvalid ? 0xff00u : 0u) |
+                            (w + 2 < (int)nvalid ? 0xff0000u : 0u) | (w + 3 < (int)nvalid ? 0xff000000u : 0u);
                 }
-            } else {
-                int k = (int)div_c((uint32_t)ug, c, clog), off = ug - k * c;
-#pragma unroll
-                for (int w = 0; w < GR; ++w) {
-                    if (off == c) {
-                        ++k;
-                        off = 0;
-                    }
-                    int r = -1;
-                    uint32_t mk = 0u;
-                    if (act && k < L) {
-                        const int rr = win_ids[k - win_k0] * c + off;
-                        if (rr < N) {
-                            r = rr;
-                            mk = win_msk[k - win_k0];
+            } else if (act) {
+                // the group's slots, one leaf at a time: leaf k covers slots
+                // [k c, (k + 1) c) of the flattened list, rows id_k c + (0 .. c-1)
+                int u = ug, k = (int)div_c((uint32_t)ug, c, clog), off = ug - k * c;
+                while (u < ug + GR && k < L) {
+                    const int id = win_ids[k - win_k0];
+                    const uint32_t mk = win_msk[k - win_k0];
+                    const int len = min(c - off, ug + GR - u);
+                    const int vlen = max(0, min(len, N - (id * c + off)));
+                    if (!isV) {
+                        const int w0 = u - ug;
+                        if (((w0 | vlen) & 3) == 0) {
+                            const uint32_t m4 = mk * 0x01010101u;
+                            for (int w = 0; w < vlen; w += 4) *reinterpret_cast<uint32_t *>(mt + gi * GR + w0 + w) = m4;
+                        } else {
+                            for (int w = 0; w < vlen; ++w) mt[gi * GR + w0 + w] = (uint8_t)mk;
                         }
                     }
-                    row[w] = r;
-                    if (act && !isV) mt[gi * GR + w] = (uint8_t)mk;
-                    ++off;
+                    nvalid += (uint32_t)vlen;
+                    if (vlen < len) break;  // the sequence's last, partial leaf
+                    u += len;
+                    ++k;
+                    off = 0;
                 }
+                if (!isV)
+                    for (int w = (int)nvalid; w < GR; ++w) mt[gi * GR + w] = 0u;
             }
-#pragma unroll
-            for (int w = 0; w < GR; ++w) nvalid += row[w] >= 0;
             uint32_t bytes = nvalid * RB;
 #pragma unroll
             for (int o = 16; o >= 1; o >>= 1) bytes += __shfl_xor_sync(FULL, bytes, o);
-            unsigned char *dst = sK + (isV ? C::HALF : 0) + gi * C::GS;
             // rows without a token: zeros, so that 0 * row stays 0 in the
             // products (the fence orders these generic stores before later
             // bulk copies into the same rows)
             if (act && nvalid < (uint32_t)GR) {
 #pragma unroll 1
-                for (int w = 0; w < GR; ++w) {
-                    if (row[w] >= 0) continue;
+                for (int w = (int)nvalid; w < GR; ++w) {
                     uint4 *z = reinterpret_cast<uint4 *>(dst + w * RB);
                     for (int i = 0; i < RB / 16; ++i) z[i] = make_uint4(0u, 0u, 0u, 0u);
                 }
@@ -679,19 +694,31 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
             __syncwarp();
             if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
             __syncwarp();
-            if (act) {
-                // one copy per run of consecutive rows
-                const unsigned char *src = isV ? Vh : Kh;
-                int w0 = 0;
-#pragma unroll
-                for (int w = 1; w <= GR; ++w) {
-                    const bool brk = (w == GR) || row[w] < 0 || row[w - 1] < 0 || row[w] != row[w - 1] + 1;
-                    if (brk) {
-                        if (row[w0] >= 0)
-                            bulk_g2s(dst + w0 * RB, src + (size_t)row[w0] * RB, (uint32_t)((w - w0) * RB),
-                                     &full[slot]);
-                        w0 = w;
+            if (act && nvalid > 0u) {
+                if (DENSE) {
+                    bulk_g2s(dst, src + (size_t)ug * RB, nvalid * RB, &full[slot]);
+                } else {
+                    // one copy per run of consecutive rows: adjacent leaves merge
+                    int u = ug, k = (int)div_c((uint32_t)ug, c, clog), off = ug - k * c;
+                    int run_w = 0, run_row = -1, run_len = 0;
+                    while (u < ug + (int)nvalid) {
+                        const int r0 = win_ids[k - win_k0] * c + off;
+                        const int len = min(c - off, ug + (int)nvalid - u);
+                        if (run_len > 0 && r0 == run_row + run_len) {
+                            run_len += len;
+                        } else {
+                            if (run_len > 0)
+                                bulk_g2s(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB),
+                                         &full[slot]);
+                            run_w = u - ug;
+                            run_row = r0;
+                            run_len = len;
+                        }
+                        u += len;
+                        ++k;
+                        off = 0;
                     }
+                    bulk_g2s(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB), &full[slot]);
                 }
             }
             issued = j + 1;
