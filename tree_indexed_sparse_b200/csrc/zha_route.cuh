@@ -48,7 +48,8 @@ namespace zha {
 
 constexpr int LOC_CAP = 2048;          // local slots held in shared memory
 constexpr int PWIN = LOC_CAP / 2 + 2;  // parents of LOC_CAP consecutive slots (c >= 2)
-constexpr int SOLO_MAX = GT;           // exact ranking for one-CTA levels up to this many slots
+constexpr int SOLO_MAX = GT;           // one-CTA levels up to this many slots
+constexpr int RANK_MAX = 32;           // ... ranked slot against slot up to this many; the histogram cut above
 
 enum CutMode : int { CUT_OPEN = 0, CUT_RANK = 1, CUT_ORDER = 2, CUT_ALL = 3, CUT_NONE = 4 };
 
@@ -874,10 +875,29 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
     if (tid < 8) misc[tid] = 0u;  // [0]: own count, [4 + h]: shared list counters
     if (tid < G) osum[tid] = 0ull;
     gsync();
-    uint32_t *lcnt = team ? a.cand_cnt + (int64_t)kh * G : misc + 4;
+    // candidates go to shared lists first (shared counters); a team then
+    // reserves room in its global lists with one atomic per head
+    classify<G>(L, cut, cw, cs, misc + 4, own, misc, osum);
     unsigned long long *lw = team ? a.cand_w + (int64_t)kh * G * CAND_MAX : cw;
     uint32_t *ls = team ? a.cand_slot + (int64_t)kh * G * CAND_MAX : cs;
-    classify<G>(L, cut, lw, ls, lcnt, own, misc, osum);
+    if (team) {
+        uint32_t *gbase = misc + 8;
+        if (tid < G) {
+            const uint32_t nh = min(misc[4 + tid], (uint32_t)CAND_MAX);
+            gbase[tid] = nh ? atomicAdd(a.cand_cnt + (int64_t)kh * G + tid, nh) : 0u;
+        }
+        gsync();
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) {
+            const uint32_t nh = min(misc[4 + h], (uint32_t)CAND_MAX), base = gbase[h];
+            for (uint32_t j = tid; j < nh; j += GT) {
+                if (base + j < (uint32_t)CAND_MAX) {
+                    lw[h * CAND_MAX + base + j] = cw[h * CAND_MAX + j];
+                    ls[h * CAND_MAX + base + j] = cs[h * CAND_MAX + j];
+                }
+            }
+        }
+    }
     bool any_order = false, any_rank = false;
 #pragma unroll 1
     for (int h = 0; h < G; ++h) {
@@ -1067,7 +1087,7 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
             L.keep[i] = (uint8_t)kb;
         }
         gsync();
-    } else if (solo && L.n <= SOLO_MAX) {
+    } else if (solo && L.n <= RANK_MAX) {
         solo_cut<G>(L, cut, reinterpret_cast<unsigned long long *>(smem + SM::off_hm), a.p);
     } else {
         if (!hist_cut<G>(a, L, smem, ts)) return false;
