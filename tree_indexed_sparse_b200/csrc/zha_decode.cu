@@ -110,6 +110,7 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
     int64_t Sp = 0;
     int64_t S = a.t.n_level[D - 1];
     auto small = [&](int64_t s) { return T == 1 || (s <= SOLO_MAX && s * node_bytes <= SMALL_BYTES); };
+    stages_init<G>(smem);
 #pragma unroll 1
     while (l >= 1) {
         if (small(S)) {
@@ -156,6 +157,7 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
             if (l >= 1) S = load_segments(a, l + 1, kh, Tp, pref, scratch) * a.t.c;
         }
     }
+    stages_inval<G>(smem);
     if (tr == 0 && threadIdx.x < G && a.visited) {
 #pragma unroll
         for (int h = 0; h < G; ++h)

@@ -13,12 +13,13 @@
 // children of every node any head kept one level up, each with the bitmask of
 // the heads that kept its parent.  It is split into T contiguous slot ranges,
 // one per CTA of the team (T = 1 for a frontier small enough for one SM).
-// Each CTA streams its nodes' summary rows once (a register prefetch ring per
-// warp) and scores each node for all G heads.  Masses are w = exp(est - M_h)
-// in 2^-40 fixed point (integer sums are exact and do not depend on the order
-// of addition), M_h the maximum over the frontier, and the target is
-// ceil(p * Z_h) of the total Z_h.  Every decision is deterministic:
-//   one CTA, at most SOLO_MAX slots: each slot is ranked exactly against all
+// Each CTA streams its nodes' summary rows once (bulk copies into per-warp
+// shared-memory stages) and scores each node for all G heads.  Masses are
+// w = exp(est - M_h) in 2^-40 fixed point (integer sums are exact and do not
+// depend on the order of addition), M_h the maximum over the frontier, and
+// the target is ceil(p * Z_h) of the total Z_h.  Every decision is
+// deterministic:
+//   one CTA, at most RANK_MAX slots: each slot is ranked exactly against all
 //   others by (estimate descending, node id ascending) and kept while the
 //   mass before it is below the target;
 //   otherwise, round 0 histograms mass and count over buckets of width 1/32
@@ -63,9 +64,10 @@ struct HeadCut {
     int mode;
 };
 
-constexpr int CH_BYTES = 64 * 1024;   // one scoring chunk of summary rows (two are staged)
-constexpr int CH_SLOTS_MAX = 256;     // slots in a chunk at most (R = 1, d = 64)
-constexpr int CH_ROWS_MAX = 256;      // summary rows in a chunk at most (d = 64)
+constexpr int SW_STAGES = 2;            // scoring stages per warp
+constexpr int SW_BYTES = 8 * 1024;      // one stage of summary rows
+constexpr int SW_ROWS_MAX = 32;         // summary rows (and slots) in a stage at most
+constexpr int SW_N = (GT / 32) * SW_STAGES;  // stages of the CTA
 
 // Shared memory of the routing.  The two scoring chunks share their space
 // with the histogram and boundary lists, which are used only after scoring.
@@ -75,15 +77,15 @@ struct RouteSmem {
     static constexpr size_t off_node = off_sc + (size_t)LOC_CAP * G * 4;  // [LOC_CAP] i32
     static constexpr size_t off_keep = off_node + (size_t)LOC_CAP * 4;    // [LOC_CAP] u8
     static constexpr size_t off_u = off_keep + LOC_CAP;                   // union: chunks | cut scratch
-    static constexpr size_t off_chunk = off_u;                            // [2][CH_BYTES]
+    static constexpr size_t off_chunk = off_u;                            // [8 warps][SW_STAGES][SW_BYTES]
     static constexpr size_t off_hc = off_u;                               // [G][NB] u32
     static constexpr size_t off_hm = off_hc + (size_t)G * NB * 4;         // [G][NB] u64 (solo: [SOLO_MAX][G] masses)
     static constexpr size_t off_cw = off_hm + (size_t)G * NB * 8;         // [G][CAND_MAX] u64
     static constexpr size_t off_cs = off_cw + (size_t)G * CAND_MAX * 8;   // [G][CAND_MAX] u32
     static constexpr size_t off_own = off_cs + (size_t)G * CAND_MAX * 4;  // [G*CAND_MAX] u32
-    static constexpr size_t u_end = off_own + (size_t)G * CAND_MAX * 4 > off_u + 2 * (size_t)CH_BYTES
+    static constexpr size_t u_end = off_own + (size_t)G * CAND_MAX * 4 > off_u + (size_t)SW_N * SW_BYTES
                                         ? off_own + (size_t)G * CAND_MAX * 4
-                                        : off_u + 2 * (size_t)CH_BYTES;
+                                        : off_u + (size_t)SW_N * SW_BYTES;
     static constexpr size_t off_pid = u_end;                              // [PWIN] i32
     static constexpr size_t off_pmk = off_pid + (size_t)PWIN * 4;         // [PWIN] u8
     static constexpr size_t off_pref = (off_pmk + PWIN + 15) / 16 * 16;   // [SEG_CAP + 1] u32
@@ -91,11 +93,11 @@ struct RouteSmem {
     static constexpr size_t off_wm = (off_cut + G * sizeof(HeadCut) + 15) / 16 * 16;  // [8][G] f32 warp maxima
     static constexpr size_t off_wc = off_wm + 8 * G * 4;                  // [8][G] u32 warp counts
     static constexpr size_t off_red = (off_wc + 8 * G * 4 + 15) / 16 * 16; // [GT] u64
-    static constexpr size_t off_bar = off_red + GT * 8;                   // [2] u64 chunk barriers
-    static constexpr size_t off_cnode = off_bar + 16;                     // [2][CH_SLOTS_MAX] i32
-    static constexpr size_t off_cmask = off_cnode + 2 * CH_SLOTS_MAX * 4; // [2][CH_SLOTS_MAX] u8
-    static constexpr size_t off_bpl = (off_cmask + 2 * CH_SLOTS_MAX + 15) / 16 * 16;  // [2][CH_ROWS_MAX] f32 plane offsets
-    static constexpr size_t off_misc = off_bpl + (size_t)2 * CH_ROWS_MAX * 4;  // u32 counters
+    static constexpr size_t off_bar = off_red + GT * 8;                   // [SW_N] u64 stage barriers
+    static constexpr size_t off_uses = off_bar + SW_N * 8;               // [SW_N] u32 completed phases
+    static constexpr size_t off_cnode = off_uses + SW_N * 4;              // [SW_N][SW_ROWS_MAX] i32
+    static constexpr size_t off_cmask = off_cnode + (size_t)SW_N * SW_ROWS_MAX * 4;  // [SW_N][SW_ROWS_MAX] u8
+    static constexpr size_t off_misc = (off_cmask + (size_t)SW_N * SW_ROWS_MAX + 15) / 16 * 16;  // u32 counters
     static constexpr size_t bytes = off_misc + 64;
     static_assert(SOLO_MAX * G * 8 <= G * NB * 8, "solo masses fit the histogram area");
     static_assert(off_u % 16 == 0, "bulk copies land on 16-byte boundaries");
@@ -215,81 +217,59 @@ __device__ __forceinline__ float head_sum(const float (&v)[G], int lane) {
 }
 
 template <int HD, int R>
-struct ScoreChunk {
-    static constexpr int NODE_BYTES = R * HD * 4;       // g rows of one node
-    static constexpr int SLOTS = CH_BYTES / NODE_BYTES;  // slots per chunk
-    static constexpr int ROWS = SLOTS * R;               // summary rows per chunk
-    static constexpr int RPW = ROWS / 8;                 // rows per warp per chunk
-    static_assert(SLOTS >= 1 && SLOTS <= CH_SLOTS_MAX && ROWS <= CH_ROWS_MAX, "chunk shape");
-    static_assert(RPW >= 1 && RPW <= 32, "one plane offset per lane");
+struct ScoreStage {
+    static constexpr int NODE_BYTES = R * HD * 4;                    // g rows of one node
+    static constexpr int SLOTS = SW_BYTES / NODE_BYTES < SW_ROWS_MAX / R ? SW_BYTES / NODE_BYTES
+                                                                          : SW_ROWS_MAX / R;  // slots per stage
+    static constexpr int ROWS = SLOTS * R;                           // summary rows per stage
+    static_assert(SLOTS >= 1 && ROWS % 8 == 0 && ROWS <= SW_ROWS_MAX, "stage shape");
 };
 
-// Warp 0: node ids of the slots of chunk k and bulk copies of their g rows
-// (one copy per run of consecutive nodes) into chunk buffer k & 1.
+// One warp: node ids of the slots of unit u (SLOTS consecutive local slots
+// from c0) and bulk copies of their g rows (one copy per run of consecutive
+// nodes) into this warp's stage buffer `dst`, completing on the stage barrier
+// `bar`.  Returns the plane offset of row `lane` (slot lane / R, plane
+// lane % R; 0 past the unit): a register load whose latency the copy hides.
 template <int HD, int R, int G>
-__device__ __noinline__ void chunk_issue(const Level &L, int64_t c0, int64_t c1, int64_t k0, int k, const int32_t *pid,
-                                            const uint8_t *pmk, const float *gb, const float *bb, int c, int clog,
-                                            int32_t nl, unsigned char *bufs, uint64_t *bars, int32_t *cnode,
-                                            uint8_t *cmask, float *bpl, int lane) {
-    using C = ScoreChunk<HD, R>;
-    const int buf = k & 1;
-    const int64_t sb = c0 + (int64_t)k * C::SLOTS;
+__device__ __forceinline__ float stage_issue(const Level &L, int64_t c0, int64_t c1, int64_t k0, int64_t u,
+                                             const int32_t *pid, const uint8_t *pmk, const float *gb, const float *bb,
+                                             int c, int clog, int32_t nl, unsigned char *dst, uint64_t *bar,
+                                             int32_t *cn, uint8_t *cm, int lane) {
+    using C = ScoreStage<HD, R>;
+    const int64_t sb = c0 + u * C::SLOTS;
     const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
-    int32_t *cn = cnode + buf * CH_SLOTS_MAX;
-    uint8_t *cm = cmask + buf * CH_SLOTS_MAX;
-    uint32_t nvalid = 0u;
-#pragma unroll 1
-    for (int i = lane; i < ns; i += 32) {
-        const int s = (int)(sb + i);
-        int nd = s;
+    int nd = -1;
+    if (lane < ns) {
+        const int s = (int)(sb + lane);
+        nd = s;
         uint32_t mk = (1u << G) - 1u;
         if (!L.top) {
             const int kk = clog >= 0 ? (s >> clog) : (int)((uint32_t)s / (uint32_t)c);
             nd = pid[kk - (int)k0] * c + (s - kk * c);
             mk = pmk[kk - (int)k0];
         }
-        const bool ok = nd < nl;
-        cn[i] = ok ? nd : -1;
-        cm[i] = ok ? (uint8_t)mk : 0;
-        nvalid += ok;
+        if (nd >= nl) nd = -1;
+        cn[lane] = nd;
+        cm[lane] = nd >= 0 ? (uint8_t)mk : 0;
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) nvalid += __shfl_xor_sync(FULL, nvalid, off);
-    __syncwarp();
+    const uint32_t nvalid = __popc(__ballot_sync(FULL, nd >= 0));
     if (lane == 0) {
+        // the stage was read through the generic proxy; the copies write it
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(&bars[buf], nvalid * (uint32_t)C::NODE_BYTES);
+        mbar_arrive_expect_tx(bar, nvalid * (uint32_t)C::NODE_BYTES);
     }
     __syncwarp();
-    unsigned char *dst = bufs + (size_t)buf * CH_BYTES;
-    // one copy per run of consecutive nodes inside each group of 32 slots:
     // a run starts where the node does not follow its left neighbour's
-#pragma unroll 1
-    for (int i0 = 0; i0 < ns; i0 += 32) {
-        const int i = i0 + lane;
-        const int nd = i < ns ? cn[i] : -1;
-        const int left = __shfl_up_sync(FULL, nd, 1);
-        const bool start = nd >= 0 && (lane == 0 || left < 0 || left + 1 != nd);
-        const unsigned brk = __ballot_sync(FULL, start || nd < 0);  // where runs end
-        if (start) {
-            const unsigned after = lane == 31 ? 0u : (brk >> (lane + 1));
-            const int len = after ? __ffs(after) : 32 - lane;
-            bulk_g2s(dst + (size_t)i * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES),
-                     &bars[buf]);
-        }
-        // the slot's plane offsets, asynchronously, completing on the same barrier
-        if (nd >= 0) {
-            float *pb = bpl + buf * CH_ROWS_MAX + (size_t)i * R;
-            if constexpr (R % 4 == 0) {
-#pragma unroll
-                for (int j = 0; j < R; j += 4) cp_async16(pb + j, bb + (size_t)nd * R + j);
-            } else {
-#pragma unroll
-                for (int j = 0; j < R; ++j) cp_async4(pb + j, bb + (size_t)nd * R + j);
-            }
-        }
+    const int left = __shfl_up_sync(FULL, nd, 1);
+    const bool start = nd >= 0 && (lane == 0 || left < 0 || left + 1 != nd);
+    const unsigned brk = __ballot_sync(FULL, start || nd < 0);
+    if (start) {
+        const unsigned after = lane == 31 ? 0u : (brk >> (lane + 1));
+        const int len = after ? __ffs(after) : 32 - lane;
+        bulk_g2s(dst + (size_t)lane * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES), bar);
     }
-    cp_async_arrive_noinc(&bars[buf]);
+    const int ndr = __shfl_sync(FULL, nd, (lane / R) & 31);
+    return (lane < C::ROWS && ndr >= 0) ? __ldg(bb + (size_t)ndr * R + lane % R) : 0.f;
 }
 
 // Sums over the warp of 8 rows x G heads of per-lane partial dots, v[row*G + h].
@@ -310,33 +290,65 @@ __device__ __forceinline__ float batch_sum(float (&v)[8 * G], int lane) {
     }
 }
 
+// The scoring stage barriers of every warp: initialised once before the
+// first level (one arrival per phase: the expect-tx arrive of the issuing
+// lane) with their phase counts, and invalidated after the last level, so
+// that the memory can serve other purposes.  Warps 0-7, each its own.
+template <int G>
+__device__ __forceinline__ void stages_init(unsigned char *smem) {
+    using SM = RouteSmem<G>;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::off_bar) + warp * SW_STAGES;
+        uint32_t *uses = reinterpret_cast<uint32_t *>(smem + SM::off_uses) + warp * SW_STAGES;
+#pragma unroll
+        for (int st = 0; st < SW_STAGES; ++st) {
+            mbar_init(&bars[st], 1);
+            uses[st] = 0u;
+        }
+        mbar_init_fence();
+    }
+    __syncwarp();
+}
+
+template <int G>
+__device__ __forceinline__ void stages_inval(unsigned char *smem) {
+    using SM = RouteSmem<G>;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncwarp();
+    if (lane == 0) {
+        uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::off_bar) + warp * SW_STAGES;
+#pragma unroll
+        for (int st = 0; st < SW_STAGES; ++st) mbar_inval(&bars[st]);
+    }
+    __syncwarp();
+}
+
 // Score local slots [c0, c1) (global slot ids) of level L.  The slots go in
-// chunks of ScoreChunk::SLOTS through two shared-memory buffers: warp 0
-// bulk-copies the g rows of chunk k + 2 while all warps score chunk k from
-// shared memory.  Warp w scores slots w, w + 8, ... of the chunk, 8 summary
-// rows at a time (one reduce-scatter per 8 rows), and keeps each node's
-// maximum over its planes in registers; the plane offsets b of its rows are
-// loaded before the chunk lands.  Parent window: ranks [k0, ...) in pid/pmk.
-// Writes L.sc / L.node at (s - L.s0) and folds the maxima and counts per head
-// into wm/wc[warp][h].
+// units of ScoreStage::SLOTS consecutive slots, unit u to warp u % 8; each
+// warp streams its own units through SW_STAGES shared-memory stages with
+// their own barriers (bulk copies of unit j + SW_STAGES are issued as soon as
+// the warp has scored unit j), so no warp waits for another while scoring.
+// A warp scores 8 summary rows at a time (one reduce-scatter per 8 rows) and
+// keeps each node's maximum over its planes in registers.  Parent window:
+// ranks [k0, ...) in pid/pmk.  Writes L.sc / L.node at (s - L.s0) and folds
+// the maxima and counts per head into wm/wc[warp][h].
 template <int HD, int R, int G>
 __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64_t c0, int64_t c1, int64_t k0,
                                           const int32_t *pid, const uint8_t *pmk, unsigned char *smem, float *wm,
                                           uint32_t *wc) {
     static_assert(G == 1 || G == 4, "query heads per KV head");
     static_assert(R == 1 || R % 8 == 0, "planes per node: 1 or a multiple of 8");
-    using C = ScoreChunk<HD, R>;
+    using C = ScoreStage<HD, R>;
     using SM = RouteSmem<G>;
     constexpr int VEC = HD / 32;
-    constexpr int SPW = C::SLOTS / 8;                    // slots per warp per chunk
-    constexpr int RPWC = SPW * R;                        // rows per warp per chunk
-    static_assert(C::SLOTS % 8 == 0 && RPWC % 8 == 0 && RPWC <= 32, "rows per warp");
+    constexpr int NW = GT / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kh = L.kh, l = L.l;
-    unsigned char *bufs = smem + SM::off_chunk;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::off_bar);
-    int32_t *cnode = reinterpret_cast<int32_t *>(smem + SM::off_cnode);
-    uint8_t *cmask = smem + SM::off_cmask;
+    unsigned char *bufs = smem + SM::off_chunk + (size_t)warp * SW_STAGES * SW_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::off_bar) + warp * SW_STAGES;
+    int32_t *cnode = reinterpret_cast<int32_t *>(smem + SM::off_cnode) + warp * SW_STAGES * SW_ROWS_MAX;
+    uint8_t *cmask = smem + SM::off_cmask + warp * SW_STAGES * SW_ROWS_MAX;
     float qs[G][VEC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -349,52 +361,46 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
     const float *bb = a.t.b[l - 1] + (int64_t)kh * cap * R;
     const int c = a.t.c, clog = a.t.c_log2;
     const int32_t nl = a.t.n_level[l - 1];
-    const int nch = (int)((c1 - c0 + C::SLOTS - 1) / C::SLOTS);
-    float *bpl = reinterpret_cast<float *>(smem + SM::off_bpl);
-    if (tid == 0) {
-        // the expect-tx arrive plus one cp.async arrive per lane of warp 0
-        mbar_init(&bars[0], 1 + 32);
-        mbar_init(&bars[1], 1 + 32);
-        mbar_init_fence();
-    }
-    gsync();
-    if (warp == 0) {
-        chunk_issue<HD, R, G>(L, c0, c1, k0, 0, pid, pmk, gb, bb, c, clog, nl, bufs, bars, cnode, cmask, bpl, lane);
-        if (nch > 1)
-            chunk_issue<HD, R, G>(L, c0, c1, k0, 1, pid, pmk, gb, bb, c, clog, nl, bufs, bars, cnode, cmask, bpl, lane);
-    }
-    gsync();
+    const int64_t nu = (c1 - c0 + C::SLOTS - 1) / C::SLOTS;  // units
+    const int nmine = nu > warp ? (int)((nu - 1 - warp) / NW + 1) : 0;
+    static_assert(SW_STAGES == 2, "two stages: plane offsets in b0 / b1");
+    // phases each stage barrier has completed before this call
+    uint32_t *uses = reinterpret_cast<uint32_t *>(smem + SM::off_uses) + warp * SW_STAGES;
+    const uint32_t u0 = uses[0], u1 = uses[1];
+    float b0 = 0.f, b1 = 0.f;  // plane offsets of row `lane` of stages 0 and 1
+    if (nmine > 0)
+        b0 = stage_issue<HD, R, G>(L, c0, c1, k0, warp, pid, pmk, gb, bb, c, clog, nl, bufs, &bars[0], cnode,
+                                   cmask, lane);
+    if (nmine > 1)
+        b1 = stage_issue<HD, R, G>(L, c0, c1, k0, warp + NW, pid, pmk, gb, bb, c, clog, nl, bufs + SW_BYTES,
+                                   &bars[1], cnode + SW_ROWS_MAX, cmask + SW_ROWS_MAX, lane);
     const int hl = lane % G;             // head of this lane's sum
     const int rl = (lane / G) % 8;       // row of this lane's sum within the batch
     float mymax = -INFINITY;             // this lane's head's maximum (lanes < G report)
     uint32_t mycnt = 0u;
 #pragma unroll 1
-    for (int k = 0; k < nch; ++k) {
-        const int buf = k & 1;
-        const int64_t sb = c0 + (int64_t)k * C::SLOTS;
+    for (int j = 0; j < nmine; ++j) {
+        const int st = j % SW_STAGES;
+        const int64_t u = warp + (int64_t)j * NW;
+        const int64_t sb = c0 + u * C::SLOTS;
         const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
-        const int32_t *cn = cnode + buf * CH_SLOTS_MAX;
-        const uint8_t *cm = cmask + buf * CH_SLOTS_MAX;
-        if (!mbar_wait(&bars[buf], (uint32_t)((k >> 1) & 1), nullptr)) set_status(a.status, ZHA_TIMEOUT_CODE);
-        // plane offset of this warp's row `lane`: slot warp + 8 (lane / R), plane lane % R
-        float bl = 0.f;
-        if (lane < RPWC) {
-            const int i = warp + 8 * (lane / R);
-            if (i < ns && cn[i] >= 0) bl = bpl[buf * CH_ROWS_MAX + i * R + lane % R];
-        }
-        const float *cb = reinterpret_cast<const float *>(bufs + (size_t)buf * CH_BYTES);
+        const int32_t *cn = cnode + st * SW_ROWS_MAX;
+        const uint8_t *cm = cmask + st * SW_ROWS_MAX;
+        if (!mbar_wait(&bars[st], ((st ? u1 : u0) + (uint32_t)(j / SW_STAGES)) & 1u, nullptr))
+            set_status(a.status, ZHA_TIMEOUT_CODE);
+        const float bl = st ? b1 : b0;  // plane offset of row `lane`
+        const float *cb = reinterpret_cast<const float *>(bufs + (size_t)st * SW_BYTES);
         float est = -INFINITY;
 #pragma unroll 1
-        for (int r0 = 0; r0 < RPWC; r0 += 8) {
-            // rows r0 .. r0 + 7 of this warp: slot warp + 8 (r / R), plane r % R
+        for (int r0 = 0; r0 < C::ROWS; r0 += 8) {
+            // rows r0 .. r0 + 7: slot r / R, plane r % R
             float v[8 * G];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const int r = r0 + q;
-                const int i = warp + 8 * (r / R);
                 float gs[VEC];
-                if (i < ns) {
-                    Vec<float, VEC>::load(cb + ((size_t)i * R + r % R) * HD + lane * VEC, gs);
+                if (r / R < ns) {
+                    Vec<float, VEC>::load(cb + (size_t)r * HD + lane * VEC, gs);
                 } else {
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) gs[e] = 0.f;
@@ -407,7 +413,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
             const float e = __shfl_sync(FULL, bl, r) + sum;
             if constexpr (R == 1) {
                 // every row is its own slot
-                const int i = warp + 8 * r;
+                const int i = r;
                 if (i < ns && (G == 4 || lane < 8)) {
                     const int nd = cn[i];
                     const bool need = nd >= 0 && ((cm[i] >> hl) & 1u);
@@ -426,7 +432,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
                 for (int off = G; off < 8 * G; off <<= 1) m8 = fmaxf(m8, __shfl_xor_sync(FULL, m8, off));
                 est = fmaxf(est, m8);
                 if ((r0 + 8) % R == 0) {
-                    const int i = warp + 8 * (r0 / R);
+                    const int i = r0 / R;
                     if (i < ns && lane < G) {
                         const int nd = cn[i];
                         const bool need = nd >= 0 && ((cm[i] >> hl) & 1u);
@@ -442,10 +448,19 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
                 }
             }
         }
-        gsync();  // chunk k's buffer is free
-        if (warp == 0 && k + 2 < nch)
-            chunk_issue<HD, R, G>(L, c0, c1, k0, k + 2, pid, pmk, gb, bb, c, clog, nl, bufs, bars, cnode, cmask, bpl,
-                                  lane);
+        __syncwarp();  // stage st is free
+        if (j + SW_STAGES < nmine) {
+            const float bn = stage_issue<HD, R, G>(L, c0, c1, k0, u + (int64_t)SW_STAGES * NW, pid, pmk, gb, bb, c,
+                                                   clog, nl, bufs + (size_t)st * SW_BYTES, &bars[st],
+                                                   cnode + st * SW_ROWS_MAX, cmask + st * SW_ROWS_MAX, lane);
+            if (st) b1 = bn;
+            else b0 = bn;
+        }
+    }
+    __syncwarp();
+    if (lane == 0) {
+        uses[0] = u0 + (uint32_t)(nmine + 1) / 2;
+        uses[1] = u1 + (uint32_t)nmine / 2;
     }
     // per-warp maxima and counts of each head: lanes with equal head
 #pragma unroll
@@ -567,19 +582,23 @@ __device__ __noinline__ void local_hist(const Level &L, const HeadCut *cut, int 
     gsync();
 }
 
-// Fix the bucket of round r for every open head from the histogram
-// (cnt/mass: shared, or the team's global one read through L2).
+// Fix the bucket of round r for every open head from the histogram (masses
+// in shared memory; counts in shared memory, or the team's global counts
+// `gcnt` read through L2 when not null: only the chosen bucket's is read).
 template <int G>
-__device__ __noinline__ void find_cut(HeadCut *cut, int r, const uint32_t *cnt, const unsigned long long *mass,
-                                      bool global, float p, unsigned long long *red) {
+__device__ __noinline__ void find_cut(HeadCut *cut, int r, const uint32_t *cnt, const uint32_t *gcnt,
+                                      const unsigned long long *mass, float p, unsigned long long *red) {
     constexpr int TPH = GT / G, BPT = NB / TPH;
+    static_assert((BPT & (BPT - 1)) == 0, "buckets per thread: a power of two");
     const int tid = threadIdx.x, h = tid / TPH, j = tid % TPH, lane = tid & 31;
     const bool act = cut[h].mode == CUT_OPEN && cut[h].rounds == r;
     unsigned long long sum = 0ull;
-#pragma unroll 1
+    // each thread sums its run of BPT buckets starting at a lane-dependent
+    // offset, so that the lanes of a warp read different banks
+#pragma unroll 4
     for (int i = 0; i < BPT; ++i) {
-        const int b = j * BPT + i;
-        sum += act ? (global ? __ldcg(mass + h * NB + b) : mass[h * NB + b]) : 0ull;
+        const int b = j * BPT + ((i + lane) & (BPT - 1));
+        sum += act ? mass[h * NB + b] : 0ull;
     }
     // inclusive scan of the per-thread sums within each head's TPH threads
     unsigned long long incl = sum;
@@ -615,14 +634,14 @@ __device__ __noinline__ void find_cut(HeadCut *cut, int r, const uint32_t *cnt, 
 #pragma unroll 1
             for (int i = 0; i < BPT; ++i) {
                 const int bi = j * BPT + i;
-                const unsigned long long m = global ? __ldcg(mass + h * NB + bi) : mass[h * NB + bi];
+                const unsigned long long m = mass[h * NB + bi];
                 if (run + m >= target) {
                     b = bi;
                     break;
                 }
                 run += m;
             }
-            const uint32_t n = global ? __ldcg(cnt + h * NB + b) : cnt[h * NB + b];
+            const uint32_t n = gcnt ? __ldcg(gcnt + h * NB + b) : cnt[h * NB + b];
             HeadCut &Hw = cut[h];
             Hw.path[r] = b;
             Hw.C = run;
@@ -858,16 +877,13 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
                     atomicAdd(gm + i, hm[i]);
                 }
             if (!ts.sync()) return false;  // B
-            // the team's histogram into shared memory: independent loads
-#pragma unroll 8
-            for (int i = tid; i < G * NB; i += GT) {
-                hc[i] = __ldcg(gc + i);
-                hm[i] = __ldcg(gm + i);
-            }
+            // the team's bucket masses into shared memory: independent loads
+#pragma unroll 16
+            for (int i = tid; i < G * NB; i += GT) hm[i] = __ldcg(gm + i);
             gsync();
-            find_cut<G>(cut, r, hc, hm, false, a.p, red);
+            find_cut<G>(cut, r, hc, gc, hm, a.p, red);
         } else {
-            find_cut<G>(cut, r, hc, hm, false, a.p, red);
+            find_cut<G>(cut, r, hc, nullptr, hm, a.p, red);
         }
     }
     // classify, boundary lists

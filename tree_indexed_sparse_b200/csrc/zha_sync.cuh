@@ -22,11 +22,13 @@
 
 namespace zha {
 
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p) {
+__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned *p) {
     unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ void red_release_add_u32(unsigned *p, unsigned v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -37,8 +39,14 @@ __device__ __noinline__ bool counter_arrive_wait(unsigned *ctr, unsigned target,
     red_release_add_u32(ctr, 1u);
     const long long t0 = clock64();
     for (;;) {
-        if (ld_acquire_u32(ctr) >= target) return true;
-        if (ld_acquire_u32(abortw)) return false;
+        // two independent relaxed polls per round trip; the fence after the
+        // counter is seen makes the pair an acquire of every arrival
+        const unsigned c = ld_relaxed_u32(ctr), ab = ld_relaxed_u32(abortw);
+        if (c >= target) {
+            fence_acq_rel_gpu();
+            return true;
+        }
+        if (ab) return false;
         if (clock64() - t0 > WAIT_BUDGET_CYCLES) {
             set_status(status, ZHA_TIMEOUT_CODE);
             atomicExch(abortw, 1u);

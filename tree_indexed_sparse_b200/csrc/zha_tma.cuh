@@ -25,6 +25,10 @@ __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }
 
+__device__ __forceinline__ void mbar_inval(uint64_t *bar) {
+    asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 // Make barrier initialisation visible to the async (TMA) proxy.
 __device__ __forceinline__ void mbar_init_fence() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -63,22 +67,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         if (abort && *abort) return false;
         if (clock64() - t0 > WAIT_BUDGET_CYCLES) return false;
     }
-}
-
-// Asynchronous 4- and 16-byte copies global -> shared (cp.async); their
-// completion is tracked on an mbarrier by cp_async_arrive_noinc.
-__device__ __forceinline__ void cp_async4(void *dst_smem, const void *src_gmem) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst_smem)), "l"(src_gmem) : "memory");
-}
-
-__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src_gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)), "l"(src_gmem) : "memory");
-}
-
-// Arrive on `bar` once every cp.async this thread has issued so far is
-// complete; the barrier's expected arrival count includes this arrival.
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 // 1-D bulk copy of `bytes` from global to shared memory; completion is
