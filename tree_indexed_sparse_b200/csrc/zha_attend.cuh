@@ -11,14 +11,16 @@
 // The union leaf list of each KV head (every leaf any of its G query heads
 // kept, with the head bitmask) is flattened into stages of TT tokens; the
 // grid's CTAs take contiguous ranges of stages over all KV heads.  In each CTA
-// one producer warp (warp 8) maps a stage's tokens to K/V rows, writes the
-// per-token head masks and issues one cp.async.bulk per K row and per V row
-// into a ring of shared-memory stages guarded by mbarriers.  Rows land at a
+// one producer warp (warp 8) maps a stage's tokens to K/V rows a leaf at a
+// time, writes the per-token head masks and issues one cp.async.bulk per run
+// of consecutive K rows (and V rows) inside each group of the stage, into a
+// ring of shared-memory stages guarded by mbarriers.  Rows land at a
 // padded stride (16 bytes past the row for bf16) so that the consumers'
 // 8-row matrix loads hit eight different bank groups.  Every K and V row
 // crosses HBM once and serves all G heads of its group (GQA sharing).
 //
-// Consumers, warps 0-7, 16 tokens each; stage j goes to warps 4(j%2)..+3:
+// Consumers, warps 0-7, 16 tokens each (bf16: every stage to all 8 warps;
+// fp32: stage j to warps 4(j%2)..+3):
 //   bf16 K/V: tensor cores (mma.sync m16n8k16, fp32 accumulate).  The queries
 //     and the probabilities are split into bf16 high and low parts (x = hi +
 //     lo to ~2^-16 relative), rows h and 8+h of the A operand, so that the
