@@ -587,6 +587,7 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
         uint8_t *win_msk = smem + SM::off_win + (size_t)LEAF_WIN * 4;
         int win_kh = -1, win_k0 = 0;
         int issued = 0;
+        const uint64_t pol = l2_evict_first();  // K/V rows are read once
         int kh;
         int64_t st64;
         map.locate(u0, kh, st64);
@@ -698,7 +699,7 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
             __syncwarp();
             if (act && nvalid > 0u) {
                 if (DENSE) {
-                    bulk_g2s(dst, src + (size_t)ug * RB, nvalid * RB, &full[slot]);
+                    bulk_g2s_hint(dst, src + (size_t)ug * RB, nvalid * RB, &full[slot], pol);
                 } else {
                     // one copy per run of consecutive rows: adjacent leaves merge
                     int u = ug, k = (int)div_c((uint32_t)ug, c, clog), off = ug - k * c;
@@ -710,8 +711,8 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                             run_len += len;
                         } else {
                             if (run_len > 0)
-                                bulk_g2s(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB),
-                                         &full[slot]);
+                                bulk_g2s_hint(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB),
+                                              &full[slot], pol);
                             run_w = u - ug;
                             run_row = r0;
                             run_len = len;
@@ -720,7 +721,8 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                         ++k;
                         off = 0;
                     }
-                    bulk_g2s(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB), &full[slot]);
+                    bulk_g2s_hint(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB), &full[slot],
+                                  pol);
                 }
             }
             issued = j + 1;
@@ -786,30 +788,38 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
 
 // Merge the partials of CTAs [b0, b1) for the G heads of KV head kh, add the
 // sink token (gather: unless leaf 0 is in the head's set) and write the
-// outputs.  Threads 0-255; every partial's (max, sum) is loaded at once, then
-// each thread sweeps four output columns over the partials in a fixed order.
-// `sm` holds 2*G*(b1-b0) + 4*G floats.
+// outputs.  Threads 0-255, one gsync: thread t takes (head, four output
+// columns) q = t % NQ and the contiguous part t / NQ of the partials, and
+// merges its part online (running max, rescaled sum and columns), eight
+// partials' loads in flight; meanwhile warps 0..G-1 compute the sink scores.
+// Then threads q < NQ add the parts in order and the sink.  `sm` holds
+// 4 * GT + G floats.
 template <typename KT, int HD, int G>
 __device__ __noinline__ void combine_kvh(const Decode &a, const StageMap &map, int kh, int b0, int b1, bool gather,
                                          float *sm) {
+    constexpr int NQ = G * (HD / 4);  // (head, column quad) pairs
+    constexpr int NS = GT / NQ;       // parts of the partial range
+    static_assert(NS >= 1 && NS * NQ == GT, "threads cover (head, quad, part)");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n = max(0, b1 - b0);
-    float *wv = sm;              // [G][n]: max, then weight
-    float *lv = sm + G * n;      // [G][n]: sums
-    float *hd = lv + G * n;      // [G] L, [G] sink weight, [G] sink score
+    float4 *racc = reinterpret_cast<float4 *>(sm);  // [GT] part columns
+    float *rml = sm + 4 * GT;                          // [GT] part max, [GT] part sum
+    float *hs0 = rml + 2 * GT;                         // [G] sink scores
     const int h_kv = a.t.h_kv;
-    for (int i = tid; i < n * G; i += GT) {
-        const int bb = i / G, h = i % G;
-        const float *pb = a.part + (((int64_t)(b0 + bb) * h_kv + kh) * G + h) * prec<HD>();
-        wv[h * n + bb] = __ldcg(pb + HD);
-        lv[h * n + bb] = __ldcg(pb + HD + 1);
-    }
     const KT *Kh = reinterpret_cast<const KT *>(a.t.K) + (int64_t)kh * a.t.kv_cap * HD;
     const KT *Vh = reinterpret_cast<const KT *>(a.t.V) + (int64_t)kh * a.t.kv_cap * HD;
-    const float qscale = a.t.scale * LOG2E;
     if (warp < G) {
         // sink score of head `warp` (-inf when it is not added)
         const int h = warp;
+        constexpr int CPL = HD / 32;
+        const float qscale = a.t.scale * LOG2E;
+        float k0[CPL], qh[CPL];
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) {
+            qh[e] = a.q[(int64_t)(kh * G + h) * HD + lane * CPL + e] * qscale;
+            if constexpr (sizeof(KT) == 2) k0[e] = __uint_as_float(((uint32_t)Kh[lane * CPL + e]) << 16);
+            else k0[e] = Kh[lane * CPL + e];
+        }
         bool add = false;
         if (gather) {
             bool has0 = false;
@@ -819,60 +829,81 @@ __device__ __noinline__ void combine_kvh(const Decode &a, const StageMap &map, i
             }
             add = !has0;
         }
-        float s0 = -INFINITY;
-        if (add) {
-            constexpr int CPL = HD / 32;
-            float k0[CPL], qh[CPL];
-#pragma unroll
-            for (int e = 0; e < CPL; ++e) {
-                qh[e] = a.q[(int64_t)(kh * G + h) * HD + lane * CPL + e] * qscale;
-                if constexpr (sizeof(KT) == 2) k0[e] = __uint_as_float(((uint32_t)Kh[lane * CPL + e]) << 16);
-                else k0[e] = Kh[lane * CPL + e];
-            }
-            s0 = warp_sum(lane_dot<CPL>(qh, k0));
-        }
-        if (lane == 0) hd[2 * G + h] = s0;
+        const float s0 = warp_sum(lane_dot<CPL>(qh, k0));
+        if (lane == 0) hs0[h] = add ? s0 : -INFINITY;
     }
-    gsync();
-    if (warp < G) {
-        const int h = warp;
-        const float s0 = hd[2 * G + h];
-        float M = s0;
-        for (int i = lane; i < n; i += 32) M = fmaxf(M, wv[h * n + i]);
-        M = warp_max(M);
-        __syncwarp();
-        float L = 0.f;
-        for (int i = lane; i < n; i += 32) {
-            const float m = wv[h * n + i];
-            const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
-            wv[h * n + i] = w;
-            L = fmaf(w, lv[h * n + i], L);
-        }
-        L = warp_sum(L);
-        const float ws = (s0 == -INFINITY) ? 0.f : exp2f(s0 - M);
-        if (lane == 0) {
-            hd[h] = L + ws;
-            hd[G + h] = ws;
-        }
-    }
-    gsync();
-    // outputs: thread -> (head, four columns)
-    for (int idx = tid; idx < G * (HD / 4); idx += GT) {
-        const int h = idx / (HD / 4), e4 = (idx % (HD / 4)) * 4;
+    {
+        const int q = tid % NQ, sp = tid / NQ;
+        const int h = q / (HD / 4), e4 = (q % (HD / 4)) * 4;
+        const int i0 = n * sp / NS, i1 = n * (sp + 1) / NS;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int i = 0; i < n; ++i) {
-            const float w = wv[h * n + i];
-            if (w == 0.f) continue;
-            const float4 o = __ldcg(reinterpret_cast<const float4 *>(
-                a.part + (((int64_t)(b0 + i) * h_kv + kh) * G + h) * prec<HD>() + e4));
-            acc.x = fmaf(w, o.x, acc.x);
-            acc.y = fmaf(w, o.y, acc.y);
-            acc.z = fmaf(w, o.z, acc.z);
-            acc.w = fmaf(w, o.w, acc.w);
+        float M = -INFINITY, L = 0.f;
+        constexpr int CB = 8;  // partials loaded per batch
+#pragma unroll 1
+        for (int i = i0; i < i1; i += CB) {
+            float m[CB], l[CB];
+            float4 o[CB];
+#pragma unroll
+            for (int u = 0; u < CB; ++u) {
+                if (i + u < i1) {
+                    const float *pb = a.part + (((int64_t)(b0 + i + u) * h_kv + kh) * G + h) * prec<HD>();
+                    m[u] = __ldcg(pb + HD);
+                    l[u] = __ldcg(pb + HD + 1);
+                    o[u] = __ldcg(reinterpret_cast<const float4 *>(pb + e4));
+                } else {
+                    m[u] = -INFINITY;
+                    l[u] = 0.f;
+                    o[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < CB; ++u) {
+                // a part with no token of head h has max -inf and is skipped
+                if (m[u] == -INFINITY) continue;
+                if (m[u] > M) {
+                    const float r = exp2f(M - m[u]);
+                    acc.x *= r;
+                    acc.y *= r;
+                    acc.z *= r;
+                    acc.w *= r;
+                    L *= r;
+                    M = m[u];
+                }
+                const float w = exp2f(m[u] - M);
+                acc.x = fmaf(w, o[u].x, acc.x);
+                acc.y = fmaf(w, o[u].y, acc.y);
+                acc.z = fmaf(w, o[u].z, acc.z);
+                acc.w = fmaf(w, o[u].w, acc.w);
+                L = fmaf(w, l[u], L);
+            }
         }
-        const float ws = hd[G + h];
-        if (ws != 0.f) {
+        racc[tid] = acc;
+        rml[tid] = M;
+        rml[GT + tid] = L;
+    }
+    gsync();
+    if (tid < NQ) {
+        const int h = tid / (HD / 4), e4 = (tid % (HD / 4)) * 4;
+        const float s0 = hs0[h];
+        float M = s0;
+#pragma unroll 1
+        for (int sp = 0; sp < NS; ++sp) M = fmaxf(M, rml[sp * NQ + tid]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float L = 0.f;
+#pragma unroll 1
+        for (int sp = 0; sp < NS; ++sp) {
+            const float m = rml[sp * NQ + tid];
+            if (m == -INFINITY) continue;
+            const float r = exp2f(m - M);
+            const float4 x = racc[sp * NQ + tid];
+            acc.x = fmaf(r, x.x, acc.x);
+            acc.y = fmaf(r, x.y, acc.y);
+            acc.z = fmaf(r, x.z, acc.z);
+            acc.w = fmaf(r, x.w, acc.w);
+            L = fmaf(r, rml[GT + sp * NQ + tid], L);
+        }
+        if (s0 != -INFINITY) {
+            const float ws = exp2f(s0 - M);
             float v0[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -883,8 +914,9 @@ __device__ __noinline__ void combine_kvh(const Decode &a, const StageMap &map, i
             acc.y = fmaf(ws, v0[1], acc.y);
             acc.z = fmaf(ws, v0[2], acc.z);
             acc.w = fmaf(ws, v0[3], acc.w);
+            L += ws;
         }
-        const float inv = 1.f / hd[h];
+        const float inv = 1.f / L;
         float4 r = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
         *reinterpret_cast<float4 *>(a.out + (int64_t)(kh * G + h) * HD + e4) = r;
     }

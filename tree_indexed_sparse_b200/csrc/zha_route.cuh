@@ -266,7 +266,8 @@ __device__ __forceinline__ float stage_issue(const Level &L, int64_t c0, int64_t
     if (start) {
         const unsigned after = lane == 31 ? 0u : (brk >> (lane + 1));
         const int len = after ? __ffs(after) : 32 - lane;
-        bulk_g2s(dst + (size_t)lane * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES), bar);
+        bulk_g2s_hint(dst + (size_t)lane * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES),
+                      bar, l2_evict_first());
     }
     const int ndr = __shfl_sync(FULL, nd, (lane / R) & 31);
     return (lane < C::ROWS && ndr >= 0) ? __ldg(bb + (size_t)ndr * R + lane % R) : 0.f;
