@@ -24,6 +24,7 @@
 
 #include "zha_device.cuh"
 #include "zha_internal.cuh"
+#include "zha_tma.cuh"
 
 namespace zha {
 
@@ -414,6 +415,8 @@ __global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict_
     const int lane = threadIdx.x & 31, j = threadIdx.x >> 5;
     const int kh = blockIdx.x;
     const int64_t pos = t.n_tokens - 1;
+    // a decode launched next may start its launch now (it waits for this grid)
+    griddep_launch_dependents();
     KT *Kh = const_cast<KT *>(reinterpret_cast<const KT *>(t.K)) + (int64_t)kh * t.kv_cap * HD;
     KT *Vh = const_cast<KT *>(reinterpret_cast<const KT *>(t.V)) + (int64_t)kh * t.kv_cap * HD;
     if (j == 0) {

@@ -178,6 +178,9 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__
     const int nbk = nb / h_kv;  // CTAs per KV head team
     unsigned *words = a.sync;
     unsigned *abortw = words + h_kv + 2;
+    // launched as a programmatic dependent of the previous kernel on the
+    // stream (an append, typically): nothing is read before it completes
+    griddep_wait();
     stamp(a, 0);
     const bool router = b < nbk * h_kv;
     const int kh = router ? b / nbk : 0, tr = router ? b % nbk : 0;
@@ -242,10 +245,21 @@ static cudaError_t decode_impl(const Decode &dc, int n_cta, cudaStream_t s) {
         if (err != cudaSuccess) return err;
         attr = smem;
     }
-    Decode arg = dc;
-    void *args[] = {&arg};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(k_decode<KT, HD, R, G>), dim3(n_cta),
-                                       dim3(A_THREADS), args, smem, s);
+    // cooperative (the CTAs meet at barriers), and a programmatic dependent
+    // of the previous kernel so that its launch overlaps that kernel's tail
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)n_cta);
+    cfg.blockDim = dim3(A_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, k_decode<KT, HD, R, G>, dc);
 }
 
 template <typename KT, int HD, int R, int G>

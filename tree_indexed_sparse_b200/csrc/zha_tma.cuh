@@ -79,6 +79,16 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
         : "memory");
 }
 
+// Programmatic dependent launch: let the next kernel on the stream begin its
+// launch now; it waits for this grid's completion in griddep_wait.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Wait until the grids this one depends on have completed and their memory
+// operations are visible (a no-op for a launch without that dependency).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // L2 policy for data read once per decode (summaries and K/V rows streamed
 // through shared memory): evicted first, so that the streams do not push the
 // kernel's code and its small scratch (lists, partials, counters) out of L2.
