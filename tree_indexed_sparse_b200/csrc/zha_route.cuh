@@ -51,6 +51,7 @@ constexpr int LOC_CAP = 2048;          // local slots held in shared memory
 constexpr int PWIN = LOC_CAP / 2 + 2;  // parents of LOC_CAP consecutive slots (c >= 2)
 constexpr int SOLO_MAX = GT;           // one-CTA levels up to this many slots
 constexpr int RANK_MAX = 32;           // ... ranked slot against slot up to this many; the histogram cut above
+constexpr int RC_MAX = 512;            // team levels up to this many slots: cut by each CTA on its own
 
 enum CutMode : int { CUT_OPEN = 0, CUT_RANK = 1, CUT_ORDER = 2, CUT_ALL = 3, CUT_NONE = 4 };
 
@@ -73,7 +74,10 @@ constexpr int SW_N = (GT / 32) * SW_STAGES;  // stages of the CTA
 // with the histogram and boundary lists, which are used only after scoring.
 template <int G>
 struct RouteSmem {
-    static constexpr size_t off_sc = 0;                                   // [LOC_CAP][G] f32
+    // [LOC_CAP][G] f32 local scores; on a redundantly cut team level
+    // (at most RC_MAX slots) every score of the level, [S][G]
+    static constexpr size_t off_sc = 0;
+    static_assert(RC_MAX <= LOC_CAP, "a redundantly cut level fits the local score array");
     static constexpr size_t off_node = off_sc + (size_t)LOC_CAP * G * 4;  // [LOC_CAP] i32
     static constexpr size_t off_keep = off_node + (size_t)LOC_CAP * 4;    // [LOC_CAP] u8
     static constexpr size_t off_u = off_keep + LOC_CAP;                   // union: chunks | cut scratch
@@ -981,6 +985,127 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
     return true;
 }
 
+// Classification of a redundantly cut level (every score in shared memory,
+// LA: all S slots): every slot is visited for the boundary lists and for the
+// boundary mass before this CTA's range (CUT_ORDER heads, into obefore[h]);
+// keep bits and own[] entries are written for this CTA's slots [s0, s0 + n)
+// only (keep: L's local array).
+template <int G>
+__device__ __noinline__ void classify_rc(const Level &LA, int64_t s0, int64_t n, uint8_t *keep, const HeadCut *cut,
+                                         unsigned long long *lw, uint32_t *ls, uint32_t *lcnt, uint32_t *own,
+                                         uint32_t *own_cnt, unsigned long long *obefore) {
+    const int lane = threadIdx.x & 31;
+    const int64_t iters = (LA.n + GT - 1) / GT;
+#pragma unroll 1
+    for (int64_t it = 0; it < iters; ++it) {
+        const int64_t s = it * GT + threadIdx.x;
+        const bool mine = s >= s0 && s < s0 + n;
+        uint32_t kbits = 0u;
+        float ev[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) ev[h] = s < LA.n ? LA.sc[s * G + h] : -INFINITY;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const HeadCut &H = cut[h];
+            const float e = ev[h];
+            bool cand = false;
+            unsigned long long w = 0ull;
+            if (e != -INFINITY) {
+                if (H.mode == CUT_ALL) {
+                    kbits |= 1u << h;
+                } else if (H.mode == CUT_RANK || H.mode == CUT_ORDER) {
+                    const int pc = path_cmp(H, e, H.rounds);
+                    if (pc < 0) kbits |= 1u << h;
+                    else if (pc == 0) {
+                        w = mass_fx(expf(e - H.M));
+                        if (H.mode == CUT_RANK) cand = true;
+                        else if (s < s0) atomicAdd(&obefore[h], w);
+                    }
+                }
+            }
+            const unsigned bal = __ballot_sync(FULL, cand);
+            if (bal) {
+                const unsigned bown = __ballot_sync(FULL, cand && mine);
+                const int leader = __ffs(bal) - 1;
+                uint32_t base = 0, obase = 0;
+                if (lane == leader) {
+                    base = atomicAdd(&lcnt[h], (uint32_t)__popc(bal));
+                    if (bown) obase = atomicAdd(own_cnt, (uint32_t)__popc(bown));
+                }
+                base = __shfl_sync(FULL, base, leader);
+                obase = __shfl_sync(FULL, obase, leader);
+                if (cand) {
+                    const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
+                    if (at < (uint32_t)CAND_MAX) {
+                        lw[h * CAND_MAX + at] = w;
+                        ls[h * CAND_MAX + at] = (uint32_t)s;
+                    }
+                    if (mine) {
+                        const uint32_t o = obase + __popc(bown & ((1u << lane) - 1u));
+                        if (o < (uint32_t)(G * CAND_MAX)) own[o] = ((uint32_t)(s - s0) << 3) | (uint32_t)h;
+                    }
+                }
+            }
+        }
+        if (mine) keep[s - s0] = (uint8_t)kbits;
+    }
+    gsync();
+}
+
+// The cut of a small team level (S <= RC_MAX; every score fits the local
+// score array): after the maxima barrier each CTA copies the team's
+// scores in and cuts the whole frontier by itself (the same integer
+// histograms as the team's, hence the same decisions), then keeps its own
+// slots.  No histogram atomics and no barriers B and C.  L.sc points at this
+// CTA's first slot inside the shared copy.
+template <int G>
+__device__ __noinline__ void rc_cut(const Decode &a, const Level &L, unsigned char *smem) {
+    using SM = RouteSmem<G>;
+    HeadCut *cut = reinterpret_cast<HeadCut *>(smem + SM::off_cut);
+    unsigned long long *red = reinterpret_cast<unsigned long long *>(smem + SM::off_red);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + SM::off_misc);
+    uint32_t *hc = reinterpret_cast<uint32_t *>(smem + SM::off_hc);
+    unsigned long long *hm = reinterpret_cast<unsigned long long *>(smem + SM::off_hm);
+    unsigned long long *cw = reinterpret_cast<unsigned long long *>(smem + SM::off_cw);
+    uint32_t *cs = reinterpret_cast<uint32_t *>(smem + SM::off_cs);
+    uint32_t *own = reinterpret_cast<uint32_t *>(smem + SM::off_own);
+    const int tid = threadIdx.x;
+    Level LA = L;
+    LA.s0 = 0;
+    LA.n = L.S;
+    LA.T = 1;
+    LA.tr = 0;
+    LA.sc = reinterpret_cast<float *>(smem + SM::off_sc);
+#pragma unroll 1
+    for (int r = 0; r < HIST_ROUNDS; ++r) {
+        bool open = false;
+#pragma unroll 1
+        for (int h = 0; h < G; ++h) open |= cut[h].mode == CUT_OPEN;
+        if (!open) break;
+        local_hist<G>(LA, cut, r, hc, hm);
+        find_cut<G>(cut, r, hc, nullptr, hm, a.p, red);
+    }
+    unsigned long long *obefore = red + 64;
+    if (tid < 8) misc[tid] = 0u;  // [0]: own count, [4 + h]: list counters
+    if (tid < G) obefore[tid] = 0ull;
+    gsync();
+    classify_rc<G>(LA, L.s0, L.n, L.keep, cut, cw, cs, misc + 4, own, misc, obefore);
+    bool any_order = false, any_rank = false;
+#pragma unroll 1
+    for (int h = 0; h < G; ++h) {
+        any_order |= cut[h].mode == CUT_ORDER;
+        any_rank |= cut[h].mode == CUT_RANK;
+    }
+    const uint32_t n_own = min(misc[0], (uint32_t)(G * CAND_MAX));
+    if (any_rank && n_own > 0) rank_own<G>(L, cut, cw, cs, own, n_own);
+    if (any_order) {
+        unsigned long long *base = red + 72;
+        if (tid < G) base[tid] = cut[tid].C + obefore[tid];
+        gsync();
+        order_own<G>(L, cut, base, red);
+    }
+}
+
 // Score and cut level l of KV head kh as rank tr of a team of T CTAs (T = 1:
 // this CTA alone).  `S` is the frontier size, `pref`/Tp/Sp the parent level's
 // segments (loaded by the caller).  F[h] receives the frontier counts.
@@ -1006,17 +1131,20 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
     L.Tp = Tp;
     L.Sp = Sp;
     Tout = T;
+    const bool team = T > 1;
+    // a team level whose scores all fit shared memory is cut by every CTA
+    // on its own copy of them (rc_cut); the scores go out through global
+    const bool rc = team && S <= RC_MAX;
     if (L.n > LOC_CAP) {
         const int64_t base = (int64_t)kh * a.score_cap + L.s0;
         L.sc = a.scores + base * G;
         L.node = a.slot_node + base;
         L.keep = a.slot_keep + base;
     } else {
-        L.sc = reinterpret_cast<float *>(smem + SM::off_sc);
+        L.sc = rc ? a.scores + ((int64_t)kh * a.score_cap + L.s0) * G : reinterpret_cast<float *>(smem + SM::off_sc);
         L.node = reinterpret_cast<int32_t *>(smem + SM::off_node);
         L.keep = smem + SM::off_keep;
     }
-    const bool team = T > 1;
     // ---- score
     if (tid < 8 * G) {
         wm[tid] = -INFINITY;
@@ -1106,6 +1234,22 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
         gsync();
     } else if (solo && L.n <= RANK_MAX) {
         solo_cut<G>(L, cut, reinterpret_cast<unsigned long long *>(smem + SM::off_hm), a.p);
+    } else if (rc) {
+        // every score of the team into shared memory (written before barrier A)
+        float *alls = reinterpret_cast<float *>(smem + SM::off_sc);
+        const float *src = a.scores + (int64_t)kh * a.score_cap * G;
+        if constexpr (G == 4) {
+            const float4 *s4 = reinterpret_cast<const float4 *>(src);
+            float4 *d4 = reinterpret_cast<float4 *>(alls);
+#pragma unroll 8
+            for (int64_t i = tid; i < S; i += GT) d4[i] = __ldcg(s4 + i);
+        } else {
+#pragma unroll 8
+            for (int64_t i = tid; i < S * G; i += GT) alls[i] = __ldcg(src + i);
+        }
+        gsync();
+        L.sc = alls + L.s0 * G;
+        rc_cut<G>(a, L, smem);
     } else {
         if (!hist_cut<G>(a, L, smem, ts)) return false;
     }
