@@ -290,7 +290,8 @@ struct PlaneOps {
 
     // Leaf n of this head, plane j: tokens [tok0, tok0 + ntok).  sh: warp-
     // private shared scratch of ntok floats.
-    static __device__ void leaf(const KT *__restrict__ Kh, int64_t tok0, int ntok, const float (&r)[VEC], int j,
+    // Kr: the leaf's rows, row i at Kr + i * HD (the cache, or a shared copy).
+    static __device__ void leaf(const KT *Kr, int ntok, const float (&r)[VEC], int j,
                                 float scale, float *__restrict__ gL, float *__restrict__ bL, float *__restrict__ mL,
                                 int64_t n, float *sh, int lane) {
         for (int i0 = 0; i0 < ntok; i0 += 32) {
@@ -299,7 +300,7 @@ struct PlaneOps {
             for (int t = 0; t < 32; ++t) {
                 float k[VEC];
                 if (i0 + t < ntok) {
-                    Vec<KT, VEC>::load(Kh + (tok0 + i0 + t) * HD + lane * VEC, k);
+                    Vec<KT, VEC>::load(Kr + (int64_t)(i0 + t) * HD + lane * VEC, k);
                 } else {
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) k[e] = 0.f;
@@ -328,7 +329,7 @@ struct PlaneOps {
         for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
         for (int i = 0; i < ntok; ++i) {
             float k[VEC];
-            Vec<KT, VEC>::load(Kh + (tok0 + i) * HD + lane * VEC, k);
+            Vec<KT, VEC>::load(Kr + (int64_t)i * HD + lane * VEC, k);
             const float w = sh[i];
 #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] = fmaf(w, k[e], acc[e]);
@@ -343,7 +344,9 @@ struct PlaneOps {
 
     // Node n of this level, plane j, from its nch children (rows ch0 ..
     // ch0 + nch - 1 of the level below).  sh: warp-private scratch of nch floats.
-    static __device__ void parent(const float *__restrict__ gC, const float *__restrict__ bC, int64_t ch0, int nch,
+    // gr: the children's g rows, child i's plane j' at gr + (i * R + j') * HD
+    // (the store, or a shared copy); bC: the level's plane offsets.
+    static __device__ void parent(const float *gr, const float *__restrict__ bC, int64_t ch0, int nch,
                                   const float (&r)[VEC], int j, float scale, float *__restrict__ gP,
                                   float *__restrict__ bP, float *__restrict__ mP, int64_t n, float *sh, int lane) {
         // child estimates at r_j: max over the child's planes j'
@@ -356,7 +359,7 @@ struct PlaneOps {
                 for (int jp = 0; jp < R; ++jp) {
                     float gs[VEC];
                     if (c0 + t < nch) {
-                        Vec<float, VEC>::load(gC + ((ch0 + c0 + t) * R + jp) * HD + lane * VEC, gs);
+                        Vec<float, VEC>::load(gr + ((int64_t)(c0 + t) * R + jp) * HD + lane * VEC, gs);
                     } else {
 #pragma unroll
                         for (int e = 0; e < VEC; ++e) gs[e] = 0.f;
@@ -390,7 +393,7 @@ struct PlaneOps {
         for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
         for (int ch = 0; ch < nch; ++ch) {
             float gs[VEC];
-            Vec<float, VEC>::load(gC + ((ch0 + ch) * R + j) * HD + lane * VEC, gs);
+            Vec<float, VEC>::load(gr + ((int64_t)ch * R + j) * HD + lane * VEC, gs);
             const float w = sh[ch];
 #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] = fmaf(w, gs[e], acc[e]);
@@ -403,6 +406,34 @@ struct PlaneOps {
         __syncwarp();
     }
 };
+
+constexpr int64_t APPEND_STAGE = 64 * 1024;  // shared copy of the rows every plane reads
+
+// Bytes of that copy for a tree (0: planes read the rows from global memory):
+// a full leaf's keys or a full node's children, whichever is larger, each
+// only when it fits APPEND_STAGE.  The kernel stages a level's rows when they
+// fit this size.
+template <typename KT, int HD, int R>
+__host__ __device__ __forceinline__ int64_t append_stage_bytes(int c, int D) {
+    if (R == 1) return 0;
+    const int64_t leaf_bytes = (int64_t)c * HD * (int64_t)sizeof(KT);
+    const int64_t child_bytes = D > 1 ? (int64_t)c * R * HD * 4 : 0;
+    int64_t need = 0;
+    if (leaf_bytes <= APPEND_STAGE) need = leaf_bytes;
+    if (child_bytes <= APPEND_STAGE && child_bytes > need) need = child_bytes;
+    return need;
+}
+
+// Copy `bytes` (a multiple of 16, both ends 16-byte aligned) from global to
+// shared memory with every thread of the CTA, all loads of a thread in flight
+// at once.  Coherent loads: the rows may have been written by this CTA.
+__device__ __forceinline__ void stage_copy(void *dst, const void *src, int64_t bytes) {
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+    const int64_t n = bytes / 16;
+#pragma unroll 8
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) d[i] = __ldcg(s + i);
+}
 
 // One CTA per KV head, one warp per plane: store the new row, prefetch every
 // ancestor's children into L2, then recompute the leaf holding the row and
@@ -442,12 +473,23 @@ __global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict_
     float r[VEC];
     Vec<float, VEC>::load(t.ref + ((int64_t)kh * R + j) * HD + lane * VEC, r);
     float *sh = bsm + j * (t.c > 32 ? t.c : 32);
+    // rows every plane's warp reads (the leaf's keys, then each level's
+    // children) go to shared memory once when they fit the staged copy
+    unsigned char *stg = reinterpret_cast<unsigned char *>(bsm + R * (t.c > 32 ? t.c : 32));
+    const int64_t stage_cap = append_stage_bytes<KT, HD, R>(t.c, t.D);
     int64_t n = pos / t.c;
     {
         const int64_t tok0 = n * t.c;
         const int ntok = (int)(t.n_tokens - tok0);
         const int64_t nc = t.node_cap[0];
-        PlaneOps<KT, HD, R>::leaf(Kh, tok0, ntok, r, j, t.scale, t.g[0] + (int64_t)kh * nc * R * HD,
+        const KT *Kr = Kh + tok0 * HD;
+        const int64_t bytes = (int64_t)ntok * HD * sizeof(KT);
+        if (bytes <= stage_cap) {
+            stage_copy(stg, Kr, bytes);
+            __syncthreads();
+            Kr = reinterpret_cast<const KT *>(stg);
+        }
+        PlaneOps<KT, HD, R>::leaf(Kr, ntok, r, j, t.scale, t.g[0] + (int64_t)kh * nc * R * HD,
                                   t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, n, sh, lane);
     }
     __syncthreads();
@@ -456,10 +498,16 @@ __global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict_
         const int64_t ch0 = n * t.c;
         const int nch = (int)min((int64_t)t.c, (int64_t)t.n_level[level - 2] - ch0);
         const int64_t capP = t.node_cap[level - 1], capC = t.node_cap[level - 2];
-        PlaneOps<KT, HD, R>::parent(t.g[level - 2] + (int64_t)kh * capC * R * HD, t.b[level - 2] + (int64_t)kh * capC * R,
-                                    ch0, nch, r, j, t.scale, t.g[level - 1] + (int64_t)kh * capP * R * HD,
-                                    t.b[level - 1] + (int64_t)kh * capP * R, t.m[level - 1] + (int64_t)kh * capP * R, n,
-                                    sh, lane);
+        const float *gr = t.g[level - 2] + ((int64_t)kh * capC + ch0) * R * HD;
+        const int64_t bytes = (int64_t)nch * R * HD * 4;
+        if (bytes <= stage_cap) {
+            stage_copy(stg, gr, bytes);
+            __syncthreads();
+            gr = reinterpret_cast<const float *>(stg);
+        }
+        PlaneOps<KT, HD, R>::parent(gr, t.b[level - 2] + (int64_t)kh * capC * R, ch0, nch, r, j, t.scale,
+                                    t.g[level - 1] + (int64_t)kh * capP * R * HD, t.b[level - 1] + (int64_t)kh * capP * R,
+                                    t.m[level - 1] + (int64_t)kh * capP * R, n, sh, lane);
         __syncthreads();
     }
 }
@@ -502,7 +550,8 @@ static cudaError_t build_impl(const Tree &t, cudaStream_t s, int n_sm) {
 template <typename KT, int HD, int R>
 static cudaError_t append_impl(const Tree &t, const void *k, const void *v, cudaStream_t s) {
     // per plane warp: one score per token of a leaf, or one estimate per child
-    const size_t smem = (size_t)R * (t.c > 32 ? t.c : 32) * sizeof(float);
+    size_t smem = (size_t)R * (t.c > 32 ? t.c : 32) * sizeof(float);
+    smem += (size_t)append_stage_bytes<KT, HD, R>(t.c, t.D);  // the shared copy of the rows every plane reads
     static size_t attr = 0;
     if (smem > attr) {
         cudaError_t err = cudaFuncSetAttribute(k_append<KT, HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
