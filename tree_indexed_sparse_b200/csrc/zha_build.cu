@@ -344,9 +344,9 @@ struct PlaneOps {
 
     // Node n of this level, plane j, from its nch children (rows ch0 ..
     // ch0 + nch - 1 of the level below).  sh: warp-private scratch of nch floats.
-    // gr: the children's g rows, child i's plane j' at gr + (i * R + j') * HD
-    // (the store, or a shared copy); bC: the level's plane offsets.
-    static __device__ void parent(const float *gr, const float *__restrict__ bC, int64_t ch0, int nch,
+    // gr / br: the children's g rows and plane offsets, child i's plane j' at
+    // gr + (i * R + j') * HD and br[i * R + j'] (the store, or a shared copy).
+    static __device__ void parent(const float *gr, const float *br, int nch,
                                   const float (&r)[VEC], int j, float scale, float *__restrict__ gP,
                                   float *__restrict__ bP, float *__restrict__ mP, int64_t n, float *sh, int lane) {
         // child estimates at r_j: max over the child's planes j'
@@ -370,7 +370,7 @@ struct PlaneOps {
             reduce_scatter<32>(v, lane);
             const int t = lane / R, jp = lane % R;
             float val = -INFINITY;
-            if (c0 + t < nch) val = bC[(ch0 + c0 + t) * R + jp] + scale * v[0];
+            if (c0 + t < nch) val = br[(c0 + t) * R + jp] + scale * v[0];
 #pragma unroll
             for (int off = 1; off < R; off <<= 1) val = fmaxf(val, __shfl_xor_sync(FULL, val, off));
             if (jp == 0 && c0 + t < nch) sh[c0 + t] = val;
@@ -417,7 +417,7 @@ template <typename KT, int HD, int R>
 __host__ __device__ __forceinline__ int64_t append_stage_bytes(int c, int D) {
     if (R == 1) return 0;
     const int64_t leaf_bytes = (int64_t)c * HD * (int64_t)sizeof(KT);
-    const int64_t child_bytes = D > 1 ? (int64_t)c * R * HD * 4 : 0;
+    const int64_t child_bytes = D > 1 ? (int64_t)c * R * (HD + 1) * 4 : 0;  // g rows, then plane offsets
     int64_t need = 0;
     if (leaf_bytes <= APPEND_STAGE) need = leaf_bytes;
     if (child_bytes <= APPEND_STAGE && child_bytes > need) need = child_bytes;
@@ -499,13 +499,16 @@ __global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict_
         const int nch = (int)min((int64_t)t.c, (int64_t)t.n_level[level - 2] - ch0);
         const int64_t capP = t.node_cap[level - 1], capC = t.node_cap[level - 2];
         const float *gr = t.g[level - 2] + ((int64_t)kh * capC + ch0) * R * HD;
-        const int64_t bytes = (int64_t)nch * R * HD * 4;
-        if (bytes <= stage_cap) {
+        const float *br = t.b[level - 2] + ((int64_t)kh * capC + ch0) * R;
+        const int64_t bytes = (int64_t)nch * R * HD * 4, bbytes = (int64_t)nch * R * 4;
+        if (bytes + bbytes <= stage_cap && bbytes % 16 == 0) {
             stage_copy(stg, gr, bytes);
+            stage_copy(stg + bytes, br, bbytes);
             __syncthreads();
             gr = reinterpret_cast<const float *>(stg);
+            br = reinterpret_cast<const float *>(stg + bytes);
         }
-        PlaneOps<KT, HD, R>::parent(gr, t.b[level - 2] + (int64_t)kh * capC * R, ch0, nch, r, j, t.scale,
+        PlaneOps<KT, HD, R>::parent(gr, br, nch, r, j, t.scale,
                                     t.g[level - 1] + (int64_t)kh * capP * R * HD, t.b[level - 1] + (int64_t)kh * capP * R,
                                     t.m[level - 1] + (int64_t)kh * capP * R, n, sh, lane);
         __syncthreads();
