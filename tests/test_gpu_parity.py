@@ -168,6 +168,39 @@ def test_edge_shapes(N, c, D, R, h_kv, h_q, d, dtype):
     assert cache.status() == 0
 
 
+@pytest.mark.parametrize("n_leaves", [400, 2048])
+def test_tied_nodes_keep_lowest_ids(n_leaves):
+    """Every leaf chunk holds the same keys, so every node has the same
+    estimate for every query (exact ties).  The cut must keep the lowest ids:
+    ceil(p * n) of them.  400 leaves: a team level small enough for each CTA
+    to cut alone (the candidates ranked by id); 2048 leaves: the team's
+    histogram with a boundary bucket too crowded to rank (taken in id
+    order)."""
+    c, D, R, h_kv, h_q, d = 4, 1, 16, 1, 4, 128
+    N = n_leaves * c
+    g = torch.Generator().manual_seed(n_leaves)
+    chunk = torch.randn(h_kv, c, d, generator=g)
+    K = chunk.repeat(1, n_leaves, 1).to(torch.bfloat16)
+    V = torch.randn(h_kv, N, d, generator=g).to(torch.bfloat16)
+    ref = torch.randn(h_kv, R, d, generator=g).to(torch.bfloat16).float()
+    cache = zha.ZhaCache(h_kv, h_q, d, R, c, D, zha.ZHA_BF16, N)
+    dK, dV, dref = K.cuda(), V.cuda(), ref.cuda()
+    cache.build(dK, dV, N, dref)
+    trees = oracle_trees(K, ref, N, c, D)
+    p = 0.3003  # p * n is not an integer: the boundary sits inside a node, away from rounding
+    want = int(np.ceil(p * n_leaves))
+    q = torch.randn(h_q, d, generator=g)
+    res = cache.decode(q.cuda(), p, trace_cap=n_leaves)
+    torch.cuda.synchronize()
+    assert cache.status() == 0
+    n_leaf = res["n_leaf"].cpu()
+    idx = res["leaf_idx"].cpu()
+    for h in range(h_q):
+        assert int(n_leaf[h]) == want, (h, int(n_leaf[h]), want)
+        assert torch.equal(idx[h, :want], torch.arange(want, dtype=torch.int32)), h
+    check_decode(res, trees, K, V, ref, q.double().numpy(), p, N, c, D, h_q // h_kv, "bf16")
+
+
 def test_append_matches_rebuild_bitexact():
     """Appending tokens one by one stores exactly the summaries of a fresh
     build over the longer cache (same device functions, same order)."""
