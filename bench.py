@@ -417,23 +417,29 @@ def run_zha(args, rank, world, local):
     dense = {"us_per_token": dense_us, "hbm_gbs": dense_bytes / (dense_us * 1e-6) / 1e9,
              "frac": dense_bytes / (dense_us * 1e-6) / 1e9 / peak, "bytes": dense_bytes, "n_tokens": n_dense}
 
-    # e2e: host buffers through the API, copies inside the timed region
+    # e2e: host buffers through the API, copies inside the timed region.  A
+    # step's inputs (q, then the token's k and v) sit packed in one pinned
+    # host row, so they cross in a single copy, as a serving loop would send
+    # them; the device views of that row are the API's inputs.
     cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
-    hq = qs.cpu().pin_memory()
-    hk = inp.K_app.cpu().pin_memory()
-    hv = inp.V_app.cpu().pin_memory()
+    qc, kc, vc = qs.cpu(), inp.K_app.cpu(), inp.V_app.cpu()
+    qb = w.h_q * w.d * 4
+    kb = w.h_kv * w.d * kc.element_size()
+    rows = [torch.cat([qc[i % w.steps].contiguous().view(torch.uint8).flatten(),
+                       kc[i].contiguous().view(torch.uint8).flatten(),
+                       vc[i].contiguous().view(torch.uint8).flatten()]) for i in range(W + K)]
+    hin = torch.stack(rows).pin_memory()
     hout = torch.empty(w.h_q, w.d, dtype=torch.float32).pin_memory()
-    dq = torch.empty(w.h_q, w.d, dtype=torch.float32, device=dev)
-    dk = torch.empty(w.h_kv, w.d, dtype=inp.K.dtype, device=dev)
-    dv = torch.empty_like(dk)
+    din = torch.empty(qb + 2 * kb, dtype=torch.uint8, device=dev)
+    dq = din[:qb].view(torch.float32).view(w.h_q, w.d)
+    dk = din[qb:qb + kb].view(inp.K.dtype).view(w.h_kv, w.d)
+    dv = din[qb + kb:].view(inp.K.dtype).view(w.h_kv, w.d)
     t_e2e = []
     for i in range(W + K):
         flush.zero_()
         torch.cuda._sleep(HOLD_CYCLES)
         ea.record(stream)
-        dq.copy_(hq[i % w.steps], non_blocking=True)
-        dk.copy_(hk[i], non_blocking=True)
-        dv.copy_(hv[i], non_blocking=True)
+        din.copy_(hin[i], non_blocking=True)
         cache.append(dk, dv)
         decode(dq)
         hout.copy_(out, non_blocking=True)
