@@ -19,9 +19,10 @@
 // depend on the order of addition), M_h the maximum over the frontier, and
 // the target is ceil(p * Z_h) of the total Z_h.  Every decision is
 // deterministic:
-//   one CTA, at most RANK_MAX slots: each slot is ranked exactly against all
-//   others by (estimate descending, node id ascending) and kept while the
-//   mass before it is below the target;
+//   one CTA, at most SOLO_MAX slots: each head's slots are ordered by
+//   (estimate descending, node id ascending) -- ranked slot against slot up
+//   to RANK_MAX slots, sorted above -- and kept while the mass before each is
+//   below the target;
 //   otherwise, round 0 histograms mass and count over buckets of width 1/32
 //   of a log-mass unit below M_h; the bucket where the cumulative mass first
 //   reaches the target holds the cut: every node of a lower bucket is kept,
@@ -49,8 +50,8 @@ namespace zha {
 
 constexpr int LOC_CAP = 2048;          // local slots held in shared memory
 constexpr int PWIN = LOC_CAP / 2 + 2;  // parents of LOC_CAP consecutive slots (c >= 2)
-constexpr int SOLO_MAX = GT;           // one-CTA levels up to this many slots
-constexpr int RANK_MAX = 32;           // ... ranked slot against slot up to this many; the histogram cut above
+constexpr int SOLO_MAX = GT;           // one-CTA levels up to this many slots (sorted by one warp per head)
+constexpr int RANK_MAX = 32;           // ... ranked slot against slot up to this many (shorter code)
 constexpr int RC_MAX = 512;            // team levels up to this many slots: cut by each CTA on its own
 
 enum CutMode : int { CUT_OPEN = 0, CUT_RANK = 1, CUT_ORDER = 2, CUT_ALL = 3, CUT_NONE = 4 };
@@ -513,7 +514,13 @@ __device__ __forceinline__ unsigned long long target_of(unsigned long long Z, fl
     return tg ? tg : 1ull;
 }
 
-// Exact cut of a one-CTA level with n <= SOLO_MAX slots: thread i ranks slot
+// Set head bit `bit` of keep[i] (byte array, any alignment) atomically.
+__device__ __forceinline__ void keep_or(uint8_t *keep, int64_t i, uint32_t bit) {
+    const uintptr_t at = reinterpret_cast<uintptr_t>(keep + i);
+    atomicOr(reinterpret_cast<uint32_t *>(at & ~(uintptr_t)3), bit << (8 * (at & 3)));
+}
+
+// Exact cut of a one-CTA level with n <= RANK_MAX slots: thread i ranks slot
 // i against every other slot of each head by (estimate descending, node id
 // ascending) -- the order of the masses, which are monotone in the estimate --
 // and sums the masses before it.  w: shared [SOLO_MAX][G] masses.
@@ -550,6 +557,100 @@ __device__ __noinline__ void solo_cut(const Level &L, HeadCut *cut, unsigned lon
             if (pre < cut[h].target) kb |= 1u << h;
         }
         L.keep[tid] = (uint8_t)kb;
+    }
+    gsync();
+}
+
+// Exact cut of a one-CTA level with RANK_MAX < n <= SOLO_MAX slots.  Warp h sorts head
+// h's slots by (estimate descending, slot ascending) -- the order of the
+// masses, which are monotone in the estimate; slots follow node ids -- with a
+// bitonic network over the warp (SOLO_MAX / 32 keys per lane: the float's
+// order-preserving bits above the complemented slot), then sums the masses in
+// that order and keeps each slot while the mass before it is below the
+// target.  Slots a head does not score (-inf) sort last and are not kept.
+template <int G>
+__device__ __noinline__ void sort_cut(const Level &L, const HeadCut *cut, float p) {
+    constexpr int E = SOLO_MAX / 32;  // keys per lane; key i = lane * E + k
+    static_assert(SOLO_MAX % 32 == 0 && (E & (E - 1)) == 0 && G <= GT / 32, "sort shape");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = (int)L.n;
+#pragma unroll 1
+    for (int i = threadIdx.x; i < n; i += GT) L.keep[i] = 0;
+    gsync();
+    if (warp < G) {
+        const int h = warp;
+        unsigned long long key[E];
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            const int i = lane * E + k;
+            const float e = i < n ? L.sc[i * G + h] : -INFINITY;
+            const uint32_t u = __float_as_uint(e);
+            const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+            key[k] = e == -INFINITY ? 0ull : ((unsigned long long)ord << 32) | (0xFFFFFFFFu - (uint32_t)i);
+        }
+        // bitonic network, descending overall, over the first nsort keys (a
+        // power of two >= n; the rest are 0 and already last); rolled loops
+        // keep the code short, the per-lane keys stay in registers
+        int nsort = 2;
+        while (nsort < n) nsort <<= 1;
+#pragma unroll 1
+        for (int size = 2; size <= nsort; size <<= 1) {
+#pragma unroll 1
+            for (int j = size >> 1; j >= E; j >>= 1) {
+#pragma unroll
+                for (int k = 0; k < E; ++k) {
+                    const int i = lane * E + k;
+                    const unsigned long long o = __shfl_xor_sync(FULL, key[k], j / E);
+                    const bool take_max = ((i & j) == 0) == ((i & size) == 0);
+                    key[k] = take_max ? (key[k] > o ? key[k] : o) : (key[k] < o ? key[k] : o);
+                }
+            }
+            // in-lane stages j = E/2 .. 1 (those below size)
+#pragma unroll
+            for (int j = E >> 1; j > 0; j >>= 1) {
+                if (j < size) {
+#pragma unroll
+                    for (int k = 0; k < E; ++k) {
+                        if (k & j) continue;
+                        const int i = lane * E + k;
+                        const unsigned long long a = key[k], b = key[k | j];
+                        const bool desc = (i & size) == 0;
+                        const unsigned long long hi = a > b ? a : b, lo = a > b ? b : a;
+                        key[k] = desc ? hi : lo;
+                        key[k | j] = desc ? lo : hi;
+                    }
+                }
+            }
+        }
+        // masses in sorted order, then the exclusive prefix over the warp
+        const float M = cut[h].M;
+        unsigned long long w[E], mine = 0ull;
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            w[k] = 0ull;
+            if (key[k]) {
+                const int i = (int)(0xFFFFFFFFu - (uint32_t)key[k]);
+                w[k] = mass_fx(expf(L.sc[i * G + h] - M));
+            }
+            mine += w[k];
+        }
+        unsigned long long incl = mine;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned long long y = __shfl_up_sync(FULL, incl, off);
+            if (lane >= off) incl += y;
+        }
+        const unsigned long long Z = __shfl_sync(FULL, incl, 31);
+        const unsigned long long target = target_of(Z, p);
+        unsigned long long run = incl - mine;
+#pragma unroll
+        for (int k = 0; k < E; ++k) {
+            if (key[k]) {
+                const int i = (int)(0xFFFFFFFFu - (uint32_t)key[k]);
+                if (run < target) keep_or(L.keep, i, 1u << h);
+                run += w[k];
+            }
+        }
     }
     gsync();
 }
@@ -658,11 +759,6 @@ __device__ __noinline__ void find_cut(HeadCut *cut, int r, const uint32_t *cnt, 
     gsync();
 }
 
-// Set head bit `bit` of keep[i] (byte array, any alignment) atomically.
-__device__ __forceinline__ void keep_or(uint8_t *keep, int64_t i, uint32_t bit) {
-    const uintptr_t at = reinterpret_cast<uintptr_t>(keep + i);
-    atomicOr(reinterpret_cast<uint32_t *>(at & ~(uintptr_t)3), bit << (8 * (at & 3)));
-}
 
 // Classify every local slot for every head: kept above the path, dropped
 // below it, boundary candidate on it.  Writes keep[], appends candidates
@@ -1234,6 +1330,8 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
         gsync();
     } else if (solo && L.n <= RANK_MAX) {
         solo_cut<G>(L, cut, reinterpret_cast<unsigned long long *>(smem + SM::off_hm), a.p);
+    } else if (solo && L.n <= SOLO_MAX) {
+        sort_cut<G>(L, cut, a.p);
     } else if (rc) {
         // every score of the team into shared memory (written before barrier A)
         float *alls = reinterpret_cast<float *>(smem + SM::off_sc);
