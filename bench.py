@@ -130,7 +130,11 @@ class Clocks:
 
     def __init__(self, local):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{local}.csv")
+        # raw samples: ZHA_CLOCKS_DIR when set (to keep them), else a temp dir
+        import tempfile
+
+        out_dir = os.environ.get("ZHA_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"zha_clocks_rank{local}.csv")
         vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
         self.index = vis[local].strip() if local < len(vis) else str(local)
 
