@@ -160,6 +160,9 @@ int zha_append(zha_ctx *ctx, const void *d_k, const void *d_v, void *stream);
  * over every token of the kept leaf chunks plus token 0, in fp32.
  * A list longer than its capacity is cut to the capacity and the device
  * status becomes ZHA_ERR_CAPACITY.
+ * Launch: one cooperative kernel, a programmatic dependent of the kernel
+ * before it on `stream` (its launch overlaps that kernel's tail); it reads no
+ * input before that kernel has completed, so stream order is kept.
  */
 int zha_decode(zha_ctx *ctx, const float *d_q, float p, float *d_out, int32_t *d_leaf_idx,
                int32_t leaf_cap, int32_t *d_n_leaf, int64_t *d_nodes_visited,
@@ -212,7 +215,8 @@ int zha_device_status(zha_ctx *ctx, int32_t *out_status, void *stream);
  * Profiling hook: zha_decode runs as one kernel; when a buffer is set, the
  * kernel writes the GPU global timer (nanoseconds) at its phase boundaries:
  *   d_ns  caller-owned device buffer of D + 3 int64 (8-byte aligned), kept
- *         alive while set; NULL clears.  d_ns[0] = start, d_ns[i] for
+ *         alive while set; NULL clears.  d_ns[0] = start (after the wait
+ *         for the kernel before it on the stream), d_ns[i] for
  *         i = 1 .. D-1 = end of routing level D - i + 1 as seen by the first
  *         CTA of KV head 0, d_ns[D] = end of the routing (every level, every
  *         KV head), d_ns[D + 1] = end of that CTA's share of the attention
