@@ -793,7 +793,7 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
 // merges its part online (running max, rescaled sum and columns), eight
 // partials' loads in flight; meanwhile warps 0..G-1 compute the sink scores.
 // Then threads q < NQ add the parts in order and the sink.  `sm` holds
-// 4 * GT + G floats.
+// 6 * GT + G floats (part columns, maxima, sums, sink scores).
 template <typename KT, int HD, int G>
 __device__ __noinline__ void combine_kvh(const Decode &a, const StageMap &map, int kh, int b0, int b1, bool gather,
                                          float *sm) {

@@ -32,7 +32,10 @@
 //   still larger than CAND_MAX holds estimates within 2^-25 of each other and
 //   is taken in node-id order.
 // Team barriers separate: the maxima (A), each histogram round (B), the
-// boundary lists (C) and the written segments (D).
+// boundary lists (C) and the written segments (D).  A team level of at most
+// RC_MAX slots skips B and C: after A every CTA copies all of the team's
+// scores and runs the histogram cut on them alone (same integer sums, same
+// decisions), keeping its own slots.
 //
 // Code size matters here as much as arithmetic: every function runs once per
 // level on little data, so cold instruction fetch dominates unless the code is
