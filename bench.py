@@ -51,6 +51,7 @@ METRIC = "µs per decoded token per layer and HBM GB/s (ZHA vs dense) at 256K–
 UNIT = "us/token"
 DEFAULT_WORKLOAD = "wide_256k"
 FLUSH_BYTES = 256 << 20
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (the measured copy peak is the roofline's denominator)
 # a bounded GPU-side delay queued before each timed step, so the host has
 # enqueued the whole step before the GPU reaches its first event
 HOLD_CYCLES = 400_000
@@ -399,6 +400,7 @@ def run_zha(args, rank, world, local):
     achieved = sum(dec_b) / (sum(t_dec) * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": "k_decode", "launches_per_step": 1,
                 "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                 "peak_kind": f"{peak_kind} copy bandwidth (burst)", "traffic": measured_traffic(w.name),
                 "algorithmic_bytes_per_launch": statistics.mean(dec_b), "us_per_launch": 1e3 * statistics.mean(t_dec)}
 
