@@ -154,6 +154,8 @@ def _small_cache(N, c, D, R, h_kv, h_q, d, dtype, seed, cap=None):
     (17, 4, 2, 16, 2, 8, 128, zha.ZHA_BF16),     # c^D + 1: a second top node
     (1000, 2, 9, 1, 1, 4, 128, zha.ZHA_BF16),    # deep binary tree
     (5000, 256, 1, 16, 1, 4, 128, zha.ZHA_BF16),  # wide leaves, ragged tail
+    (3000, 4, 3, 16, 4, 4, 64, zha.ZHA_F32),     # one query head per KV head: sorted, redundant and team cuts
+    (2000, 4, 3, 16, 2, 8, 64, zha.ZHA_BF16),    # d = 64 with groups of 4
 ])
 def test_edge_shapes(N, c, D, R, h_kv, h_q, d, dtype):
     cache, (K, V, ref), _ = _small_cache(N, c, D, R, h_kv, h_q, d, dtype, seed=N + c)
