@@ -30,8 +30,8 @@
  *     m_j = logsumexp_i(r_j.k_i/sqrt(d)) and its gradient g_j (the
  *     softmax-weighted mean key); the chunk's estimated log mass for a query
  *     q is the max over the tangent planes m_j + (q - r_j).g_j/sqrt(d)
- *     ([ZH-CN2]: "tangent planes ... take the max over several estimate
- *     planes").
+ *     ([ZH-CN2]: each reference query gives one linear estimate of the
+ *     chunk's log mass, and the chunk's estimate is the largest of them).
  *   - Parent summary: m_j = logsumexp over children of the child's estimate
  *     at q = r_j; g_j = children's g_j weighted by softmax of those
  *     estimates ([ZH-CN1]: summaries grouped and compressed recursively).
@@ -40,7 +40,7 @@
  *   - Top-p: softmax over the current frontier, order by probability
  *     descending with ties to the lower node id, keep the shortest prefix
  *     whose cumulative probability reaches p; p >= 1 keeps every node
- *     ([ZH-CN2]: "smallest node set whose cumulative mass reaches p";
+ *     ([ZH-CN2]: the kept set is the fewest nodes whose mass adds up to p;
  *     [ZH-JA]: top-p, not a fixed top-k).
  *   - Attention: exact softmax attention over the raw keys of the kept leaf
  *     chunks plus token 0, the attention sink ([ZH-RU]: attention uses the

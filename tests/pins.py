@@ -350,7 +350,112 @@ def pin_golden_geometry(lib):
         assert abs(m[2, 0] - logsumexp(s[2 * span:])) <= 1e-10 * max(1.0, abs(m[2, 0]))
 
 
+def pin_node_summary_subtree(lib):
+    """orc_node_summary, which recomputes one node from its own subtree's raw
+    keys, equals the log-sum-exp and softmax-weighted mean key of r_j.k/sqrt(d)
+    over exactly that subtree (ragged tails included), its plane offset is the
+    tangent plane's value at q = 0, and it equals the row the whole-tree build
+    stores for the same node."""
+    for case_i, (N, c, D, R, d) in enumerate(_tree_cases()):
+        rng = _rng(1400 + case_i)
+        K = rng.standard_normal((N, d)).astype(np.float32)
+        ref = rng.standard_normal((R, d))
+        K64 = K.astype(np.float64)
+        tree = oracle.build(K, N, ref, c, D, lib=lib)
+        for level in range(1, D + 1):
+            n_l = -(-N // c ** level)
+            tm, tg, tb = tree.level(level)
+            assert tm.shape[0] == n_l
+            for n in range(n_l):
+                m, g, b = oracle.node_summary(K, N, ref, c, level, n, lib=lib)
+                t0, t1 = _subtree(N, c, level, n)
+                for j in range(R):
+                    s = K64[t0:t1] @ ref[j] / math.sqrt(d)
+                    m_ref = logsumexp(s)
+                    g_ref = softmax(s) @ K64[t0:t1]
+                    # tangent plane of lse(q.k/sqrt(d)) at r_j, evaluated at q = 0
+                    b_ref = m_ref - ref[j] @ g_ref / math.sqrt(d)
+                    assert abs(m[j] - m_ref) <= 1e-10 * max(1.0, abs(m_ref)), (case_i, level, n, j)
+                    assert np.max(np.abs(g[j] - g_ref)) <= 1e-10 * max(1.0, np.max(np.abs(g_ref))), (level, n, j)
+                    assert abs(b[j] - b_ref) <= 1e-10 * max(1.0, abs(m_ref), abs(b_ref)), (level, n, j)
+                assert np.max(np.abs(m - tm[n])) <= 1e-12 * max(1.0, np.max(np.abs(m)))
+                assert np.max(np.abs(g - tg[n])) <= 1e-12 * max(1.0, np.max(np.abs(g)))
+
+
+def pin_estimate_many_rows(lib):
+    """The batch estimate of listed node ids of one level (rows offset by the
+    level's first row) is, at q = r_j, the exact log mass of each listed
+    node's subtree, and below it for any other q."""
+    for case_i, (N, c, D, R, d) in enumerate(_tree_cases()):
+        rng = _rng(1500 + case_i)
+        K = rng.standard_normal((N, d)).astype(np.float32)
+        ref = rng.standard_normal((R, d))
+        K64 = K.astype(np.float64)
+        tree = oracle.build(K, N, ref, c, D, lib=lib)
+        for level in range(1, D + 1):
+            n_l = -(-N // c ** level)
+            ids = rng.permutation(n_l)[: max(1, (2 * n_l) // 3)]
+            exact_at = {}
+            for j in range(R):
+                est = oracle.estimate_many(tree.m, tree.g, int(tree.level_off[level - 1]), ids, ref, ref[j],
+                                           lib=lib)
+                for i, n in enumerate(ids):
+                    t0, t1 = _subtree(N, c, level, int(n))
+                    m_ref = logsumexp(K64[t0:t1] @ ref[j] / math.sqrt(d))
+                    assert abs(est[i] - m_ref) <= 1e-10 * max(1.0, abs(m_ref)), (case_i, level, int(n), j)
+            q = rng.standard_normal(d) * 1.5
+            est = oracle.estimate_many(tree.m, tree.g, int(tree.level_off[level - 1]), ids, ref, q, lib=lib)
+            for i, n in enumerate(ids):
+                t0, t1 = _subtree(N, c, level, int(n))
+                assert est[i] <= logsumexp(K64[t0:t1] @ q / math.sqrt(d)) + 1e-9, (case_i, level, int(n))
+
+
+def pin_heads_drivers(lib):
+    """The multi-head drivers (several KV heads in one strided store, G query
+    heads per KV head) give, per KV head, the subtree closed form of every
+    node of that head's own keys, and per query head, exactly the single-head
+    decode with that head's own keys, values and reference queries; at p = 1
+    every query head's output is dense softmax attention over its KV head."""
+    rng = _rng(1600)
+    H_kv, G, cap, N, c, D, R, d = 2, 2, 160, 151, 3, 3, 2, 8
+    H_q = H_kv * G
+    K = np.zeros((H_kv, cap, d), dtype=np.float32)
+    V = np.zeros((H_kv, cap, d), dtype=np.float32)
+    K[:, :N] = rng.standard_normal((H_kv, N, d))
+    V[:, :N] = rng.standard_normal((H_kv, N, d))
+    K[:, N:] = 7.0  # rows past N must never be read
+    V[:, N:] = -7.0
+    ref = rng.standard_normal((H_kv, R, d))
+    ht = oracle.build_heads(K, N, ref, c, D, capacity=cap, lib=lib)
+    for kh in range(H_kv):
+        K64 = K[kh, :N].astype(np.float64)
+        tree = ht.head(kh)
+        single = oracle.build(K[kh], N, ref[kh], c, D, capacity=cap, lib=lib)
+        for level in range(1, D + 1):
+            m, g, b = tree.level(level)
+            sm, sg, sb = single.level(level)
+            assert np.array_equal(m, sm) and np.array_equal(g, sg) and np.array_equal(b, sb), (kh, level)
+            for n in range(m.shape[0]):
+                t0, t1 = _subtree(N, c, level, n)
+                for j in range(R):
+                    s = K64[t0:t1] @ ref[kh, j] / math.sqrt(d)
+                    assert abs(m[n, j] - logsumexp(s)) <= 1e-10 * max(1.0, abs(m[n, j])), (kh, level, n, j)
+                    b_ref = logsumexp(s) - ref[kh, j] @ (softmax(s) @ K64[t0:t1]) / math.sqrt(d)
+                    assert abs(b[n, j] - b_ref) <= 1e-10 * max(1.0, abs(b_ref), abs(m[n, j])), (kh, level, n, j)
+    for p in (0.5, 0.8, 1.0):
+        Q = rng.standard_normal((H_q, d)) * 2.0
+        out, leaves, vis = oracle.decode_heads(K, V, ht, ref, Q, p, lib=lib)
+        for h in range(H_q):
+            kh = h // G
+            o1, l1, v1 = oracle.decode_one(K[kh], V[kh], ht.head(kh), ref[kh], Q[h], p, lib=lib)
+            assert np.array_equal(out[h], o1) and list(leaves[h]) == list(l1) and int(vis[h]) == v1, (p, h)
+            if p >= 1.0:
+                w = softmax(K[kh, :N].astype(np.float64) @ Q[h] / math.sqrt(d))
+                assert np.max(np.abs(out[h] - w @ V[kh, :N].astype(np.float64))) <= 1e-12, h
+
+
 ALL_PINS = [pin_closed_form_subtree, pin_lower_bound_and_tangent, pin_single_plane_affine,
             pin_exact_leaves_token_topp, pin_dense_at_p1, pin_flat_chunk_topp, pin_routing_invariants,
             pin_ties_lower_id, pin_topp_brute_force, pin_attention_and_sink, pin_bf16_widening,
-            pin_append_equivalence, pin_golden_geometry]
+            pin_append_equivalence, pin_golden_geometry, pin_node_summary_subtree, pin_estimate_many_rows,
+            pin_heads_drivers]

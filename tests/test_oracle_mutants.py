@@ -42,6 +42,17 @@ MUTANTS = {
     "sink_dropped": ("if (nleaf == 0 || leaves[0] != 0)\n        tok[T++] = 0;", "if (0)\n        tok[T++] = 0;"),
     "attention_without_scale": ("s[t] = scale * acc;", "s[t] = acc;"),
     "append_skips_ancestors": ("        n /= c;\n    }\n}", "        n /= c;\n        break;\n    }\n}"),
+    "node_summary_tail_clip": ("    if (c1 > nbelow)\n        c1 = nbelow;\n    const int nch",
+                               "    if (c1 > nbelow)\n        c1 = nbelow - 1;\n    const int nch"),
+    "node_summary_leaf_clip": ("            t1 = N;\n        orc_leaf_summary(K, dtype, t0, t1, d, ref, R, m, g, b);",
+                               "            t1 = N - 1;\n        orc_leaf_summary(K, dtype, t0, t1, d, ref, R, m, g, b);"),
+    "node_summary_child_offset": ("orc_node_summary(K, dtype, N, d, ref, R, c, level - 1, c0 + ch,",
+                                  "orc_node_summary(K, dtype, N, d, ref, R, c, level - 1, ch,"),
+    "estimate_many_row_offset": ("const int64_t row = level_row0 + ids[i];", "const int64_t row = ids[i];"),
+    "decode_heads_ref_stride": ("level_off, R, c, D, ref + (size_t)kh * R * d,", "level_off, R, c, D, ref,"),
+    "decode_heads_value_stride": ("const char *Vh = (const char *)V + (size_t)kh * kv_stride * d * esize;",
+                                  "const char *Vh = (const char *)V + (size_t)kh * d * esize;"),
+    "build_heads_offset_stride": ("b + kh * m_stride, level_off);", "b, level_off);"),
 }
 
 
