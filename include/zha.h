@@ -196,8 +196,13 @@ int zha_dense_decode(zha_ctx *ctx, const float *d_q, float *d_out, void *stream)
  * 256), plus h_kv * 4 bytes of tickets, exceed ZHA_STATIC_SCRATCH_BYTES
  * (for d = 128 on 148 SMs: h_q <= 107).
  * The first call on each device looks up the scratch's device address
- * (cudaGetSymbolAddress, with that device current), so make it before any
- * stream capture begins.  Every call clears the tickets on `stream` first.
+ * (cudaGetSymbolAddress, with that device current).  Under CUDA's default
+ * lazy module loading, that first call (or any earlier use of this library's
+ * kernels on the device) also loads the library's device module, which
+ * reserves the fixed scratch and the kernel code in device memory.  So make
+ * the first call during engine set-up (warm-up), before serving starts and
+ * before any stream capture begins; later calls allocate nothing.  Every
+ * call clears the tickets on `stream` first.
  * One call at a time per device: calls in flight together, on any streams or
  * host threads, share the scratch and corrupt each other's outputs.
  */
@@ -224,6 +229,19 @@ int zha_device_status(zha_ctx *ctx, int32_t *out_status, void *stream);
  * No effect on results.
  */
 int zha_set_phase_timer(zha_ctx *ctx, int64_t *d_ns);
+
+/*
+ * Testing hook: the clock-cycle budget of each wait of zha_decode on other
+ * CTAs (its team and grid barriers; default 2e9 cycles, about one second).
+ * When a wait runs out, that CTA records ZHA_ERR_TIMEOUT in the device status
+ * word and raises an abort flag, every CTA of the decode leaves at its next
+ * wait without attending, and the call's outputs are invalid;
+ * zha_device_status then reports ZHA_ERR_TIMEOUT and clears the decode
+ * scratch, so the next decode starts clean.  0 makes every wait that is not
+ * already satisfied give up at once.  Waits for the decode's own bulk copies
+ * keep the default budget.  Returns ZHA_ERR_BAD_ARG for a negative budget.
+ */
+int zha_set_wait_budget(zha_ctx *ctx, int64_t cycles);
 
 /* Tokens currently in the cache (host-side count; 0 before zha_build). */
 int64_t zha_n_tokens(const zha_ctx *ctx);

@@ -78,6 +78,8 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.orc_estimate_many.restype = None
     lib.orc_node_summary.argtypes = [_P, _I32, _I64, _I32, _P, _I32, _I32, _I32, _I64, _P, _P, _P]
     lib.orc_node_summary.restype = None
+    lib.orc_set_threads.argtypes = [_I32]
+    lib.orc_set_threads.restype = None
     return lib
 
 
@@ -129,6 +131,11 @@ def f64(x) -> np.ndarray:
 
         x = x.detach().cpu().to(torch.float64).numpy()
     return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def set_threads(n: int, lib=None) -> None:
+    """Threads of the OpenMP drivers (build_heads, decode_heads)."""
+    (lib or load()).orc_set_threads(int(n))
 
 
 def level_nodes(n_tokens: int, c: int, level: int, lib=None) -> int:

@@ -54,6 +54,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_F32 0
 #define ORC_BF16 1
@@ -547,4 +550,15 @@ void orc_node_summary(const void *K, int dtype, int64_t N, int d, const double *
     free(cm);
     free(cg);
     free(cb);
+}
+
+/* Threads the multi-head drivers use (OpenMP builds); no arithmetic. */
+void orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
 }

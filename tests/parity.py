@@ -9,11 +9,16 @@ the scale of m).
 Routing parity (replay): the GPU writes its kept node ids per level and query
 head (the trace).  For each head the oracle walks the GPU's own path: at each
 level it scores the GPU's frontier in fp64, takes its own top-p cut, and
-checks that every node on which the two kept sets differ is ambiguous -- its
-oracle probability within 1e-5 of the probability at the cut, or the oracle's
-cumulative mass just before or after it within 1e-5 of p.  The next frontier
-is the children of the GPU's kept nodes, so one borderline node does not
-derail the levels below.  Ambiguous nodes are counted and reported.
+checks that every node on which the two kept sets differ is ambiguous: its
+oracle probability within a relative 1e-5 of the probability at the cut
+(|P_i - P_cut| <= 1e-5 max(P_i, P_cut); the band scales with the
+probabilities, so it does not swallow a whole level of tiny ones), or the
+oracle's cumulative mass just before or after it within 1e-5 of p.  The next
+frontier is the children of the GPU's kept nodes, so one borderline node does
+not derail the levels below.  Ambiguous nodes are counted, bounded (at most
+AMB_FRAC of the kept nodes compared, so none on the small cases) and
+appended, one JSON line per check, to the parity log (ZHA_PARITY_LOG, by
+default gpurun_out/parity_counts.jsonl at the repository root).
 
 Output parity: the oracle's exact attention over the GPU's own token set
 (kept leaves plus the sink) matches the GPU output within the dtype's
@@ -22,12 +27,18 @@ oracle's own, so this is also parity with the oracle's full decode.
 """
 from __future__ import annotations
 
+import json
+import os
+import time
+
 import numpy as np
 import torch
 
 import oracle
 
-AMBIG = 1e-5
+AMBIG_REL = 1e-5        # relative band on the probability at the cut
+AMBIG_CUM = 1e-5        # band on the cumulative mass around p
+AMB_FRAC = 1e-4         # most ambiguous nodes allowed per kept node compared
 OUT_TOL = {"f32": 1e-5, "bf16": 2e-3}
 BUILD_RTOL = 1e-5
 
@@ -42,29 +53,46 @@ def oracle_trees(K_cpu, ref_cpu, n_tokens: int, c: int, D: int, capacity: int | 
             for kh in range(K_cpu.shape[0])]
 
 
-def check_build(cache, trees, rtol: float = BUILD_RTOL, levels=None, sample=None, seed=0):
+def touched_nodes(t0: int, t1: int, c: int, D: int) -> dict:
+    """Node ids of every level whose subtree holds a token of [t0, t1)."""
+    return {lv: np.arange(t0 // c ** lv, (t1 - 1) // c ** lv + 1) for lv in range(1, D + 1)}
+
+
+def check_build(cache, trees, rtol: float = BUILD_RTOL, levels=None, sample=None, seed=0, ids=None,
+                heads=None):
     """Compare the GPU summary store with the oracle trees; returns the worst
-    relative errors (m, g, b).  `sample` limits the checked nodes per level."""
+    relative errors (m, g, b).  `sample` limits the checked nodes per level
+    (the last, possibly partial, node is always among them); `ids` (level ->
+    node ids) checks exactly those nodes instead; `heads` lists the KV heads
+    that `trees` holds, in order (default: all)."""
     cfg = cache.cfg
     worst = [0.0, 0.0, 0.0]
     rng = np.random.default_rng(seed)
-    for level in (levels or range(1, cfg.D + 1)):
+    heads = list(range(cfg.h_kv)) if heads is None else list(heads)
+    for level in (levels or (sorted(ids) if ids is not None else range(1, cfg.D + 1))):
         g, b, m = cache.summaries(level)
         n = m.shape[1]
-        ids = np.arange(n) if sample is None or n <= sample else np.sort(rng.choice(n, sample, replace=False))
-        idt = torch.as_tensor(ids, device=g.device)
-        g = g[:, idt].double().cpu().numpy()
-        b = b[:, idt].double().cpu().numpy()
-        m = m[:, idt].double().cpu().numpy()
-        for kh, tree in enumerate(trees):
+        if ids is not None:
+            sel = np.asarray(ids[level], dtype=np.int64)
+        elif sample is None or n <= sample:
+            sel = np.arange(n)
+        else:
+            sel = np.union1d(rng.choice(n, sample, replace=False), [n - 1])
+        ids_l = sel
+        idt = torch.as_tensor(ids_l, device=g.device)
+        for i, tree in enumerate(trees):
+            kh = heads[i]
+            gi = g[kh].index_select(0, idt).double().cpu().numpy()
+            bi = b[kh].index_select(0, idt).double().cpu().numpy()
+            mi = m[kh].index_select(0, idt).double().cpu().numpy()
             mo, go, bo = tree.level(level)
             assert mo.shape[0] == n, (level, mo.shape, n)
-            mo, go, bo = mo[ids], go[ids], bo[ids]
-            em = np.abs(m[kh] - mo) / np.maximum(1.0, np.abs(mo))
+            mo, go, bo = mo[ids_l], go[ids_l], bo[ids_l]
+            em = np.abs(mi - mo) / np.maximum(1.0, np.abs(mo))
             # b = m - r.g/sqrt(d) cancels: its fp32 error scales with |m| and |r.g|/sqrt(d)
-            eb = np.abs(b[kh] - bo) / np.maximum(1.0, np.maximum(np.abs(mo), np.abs(mo - bo)))
+            eb = np.abs(bi - bo) / np.maximum(1.0, np.maximum(np.abs(mo), np.abs(mo - bo)))
             scale_g = np.maximum(1.0, np.abs(go).max(axis=-1, keepdims=True))
-            eg = np.abs(g[kh] - go) / scale_g
+            eg = np.abs(gi - go) / scale_g
             worst = [max(worst[0], float(em.max())), max(worst[1], float(eg.max())), max(worst[2], float(eb.max()))]
             assert em.max() <= rtol, ("m", level, kh, float(em.max()))
             assert eg.max() <= rtol, ("g", level, kh, float(eg.max()))
@@ -72,9 +100,31 @@ def check_build(cache, trees, rtol: float = BUILD_RTOL, levels=None, sample=None
     return worst
 
 
-def replay_head(tree, ref_kh, q_h, p: float, trace_ids, trace_cnt, h: int, n_tokens: int, c: int, D: int):
+def parity_log_path() -> str:
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    return os.environ.get("ZHA_PARITY_LOG") or os.path.join(root, "gpurun_out", "parity_counts.jsonl")
+
+
+def record(case: str, **fields) -> None:
+    """Append one JSON line about a parity check to the parity log."""
+    path = parity_log_path()
+    try:
+        os.makedirs(os.path.dirname(path), exist_ok=True)
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": case, "time": time.time(), **fields}) + "\n")
+    except OSError:
+        pass
+
+
+def amb_bound(kept: int) -> int:
+    """Ambiguous nodes allowed when `kept` kept nodes were compared."""
+    return int(AMB_FRAC * kept)
+
+
+def replay_head(tree, ref_kh, q_h, p: float, trace_ids, trace_cnt, h: int, n_tokens: int, c: int, D: int,
+                stats=None):
     """Replay one query head's routing.  Returns (ambiguous count, visited,
-    GPU leaves)."""
+    GPU leaves); `stats` (a dict) accumulates the kept nodes compared."""
     amb = 0
     visited = 0
     front = np.arange(level_count(n_tokens, c, D), dtype=np.int64)
@@ -95,9 +145,12 @@ def replay_head(tree, ref_kh, q_h, p: float, trace_ids, trace_cnt, h: int, n_tok
             pos = {int(n): i for i, n in enumerate(front)}
             for n in diff:
                 i = pos[n]
-                near = (abs(prob[i] - p_cut) <= AMBIG or abs(cb[i] - p) <= AMBIG or abs(cb[i] + prob[i] - p) <= AMBIG)
+                near = (abs(prob[i] - p_cut) <= AMBIG_REL * max(prob[i], p_cut) or abs(cb[i] - p) <= AMBIG_CUM
+                        or abs(cb[i] + prob[i] - p) <= AMBIG_CUM)
                 assert near, ("routing differs on a non-ambiguous node", level, n, prob[i], p_cut, cb[i], p)
             amb += len(diff)
+        if stats is not None:
+            stats["kept"] = stats.get("kept", 0) + len(ok_set)
         visited += len(front)
         if level == 1:
             gpu_leaves = gk
@@ -109,8 +162,10 @@ def replay_head(tree, ref_kh, q_h, p: float, trace_ids, trace_cnt, h: int, n_tok
 
 
 def check_decode(res, trees, K_cpu, V_cpu, ref_cpu, q_cpu, p: float, n_tokens: int, c: int, D: int, G: int,
-                 kv_dtype: str, heads=None):
-    """Full protocol for one decode call; returns the ambiguous-node count."""
+                 kv_dtype: str, heads=None, case: str | None = None):
+    """Full protocol for one decode call; returns the ambiguous-node count,
+    after checking it against amb_bound and, when `case` names the check,
+    recording it in the parity log."""
     tid = res["trace_ids"].cpu().numpy()
     tcnt = res["trace_counts"].cpu().numpy()
     out = res["out"].double().cpu().numpy()
@@ -119,9 +174,12 @@ def check_decode(res, trees, K_cpu, V_cpu, ref_cpu, q_cpu, p: float, n_tokens: i
     visited = res["visited"].cpu().numpy()
     h_q = out.shape[0]
     amb_total = 0
-    for h in (heads if heads is not None else range(h_q)):
+    stats = {}
+    worst = 0.0
+    checked = list(heads if heads is not None else range(h_q))
+    for h in checked:
         kh = h // G
-        amb, vis, leaves = replay_head(trees[kh], ref_cpu[kh], q_cpu[h], p, tid, tcnt, h, n_tokens, c, D)
+        amb, vis, leaves = replay_head(trees[kh], ref_cpu[kh], q_cpu[h], p, tid, tcnt, h, n_tokens, c, D, stats)
         amb_total += amb
         assert int(visited[h]) == vis, ("nodes visited", h, int(visited[h]), vis)
         assert int(n_leaf[h]) == len(leaves), ("leaf count", h)
@@ -129,5 +187,11 @@ def check_decode(res, trees, K_cpu, V_cpu, ref_cpu, q_cpu, p: float, n_tokens: i
         toks = oracle.token_set(leaves, n_tokens, c)
         ref_out = oracle.attend(K_cpu[kh], V_cpu[kh], toks, q_cpu[h])
         err = float(np.max(np.abs(out[h] - ref_out)))
+        worst = max(worst, err)
         assert err <= OUT_TOL[kv_dtype], ("output", h, err)
+    kept = stats.get("kept", 0)
+    if case is not None:
+        record(case, heads=len(checked), kept_compared=kept, ambiguous=amb_total, bound=amb_bound(kept),
+               max_abs_err=worst, n_tokens=int(n_tokens))
+    assert amb_total <= amb_bound(kept), ("ambiguous nodes over the bound", amb_total, kept)
     return amb_total

@@ -1,11 +1,19 @@
 """CUDA path vs the fp64 oracle at the full sizes of the benchmark workloads,
 in the launch configuration the benchmark times (needs a B200).
 
-Build parity is checked on sampled nodes of every level.  Decode parity
-replays the GPU's routing trace of one decode step per workload against the
-oracle (every query head for the 256K and 1M workloads; the four query heads
-of KV head 0 for the 10M one, whose oracle estimates are computed node by node
-from the raw keys instead of a stored tree) and checks the outputs.
+Each workload runs its own schedule:
+  * wide_256k, light_1m: decodes only; the first and the last query of the
+    workload are replayed for every query head;
+  * deep_256k: 128 steps of (two appends, one decode); four steps are
+    replayed, and after the 256 appends every node they touched is checked;
+  * extreme_10m: 64 decodes, then 1,024 appends, then one more decode; the
+    first and last of the 64 and the decode after the appends are replayed
+    for all 16 query heads, and every node the appends touched is checked.
+The oracle side runs one KV head at a time (its tree, keys and values), so
+the 10M case needs about 10 GB of host memory at once.  Build parity is
+checked on sampled nodes of every level (always including the last, partial
+node) plus the appended nodes.  Each replay appends its ambiguous-node count
+to the parity log (see parity.py).
 """
 import numpy as np
 import pytest
@@ -13,27 +21,13 @@ import torch
 
 import oracle
 import workloads
-from parity import check_build, check_decode
+from parity import check_build, check_decode, touched_nodes
 
 import tree_indexed_sparse_b200 as zha
 
 pytestmark = pytest.mark.gpu
 
 W = workloads.WORKLOADS
-
-
-class LazyTree:
-    """Oracle estimates of any node, from its subtree's raw keys."""
-
-    def __init__(self, K, n_tokens, c, D):
-        self.K, self.n_tokens, self.c, self.D = K, n_tokens, c, D
-
-    def estimates(self, l, ids, ref, q):
-        out = np.empty(len(ids))
-        for i, n in enumerate(ids):
-            m, g, _ = oracle.node_summary(self.K, self.n_tokens, ref, self.c, l, int(n))
-            out[i] = oracle.estimate(m, g, ref, q)
-        return out
 
 
 def _gpu_cache(w, inp):
@@ -43,49 +37,112 @@ def _gpu_cache(w, inp):
     return cache
 
 
-@pytest.mark.parametrize("name", ["wide_256k", "deep_256k", "light_1m"])
+def _decode(cache, q, p, trace_cap):
+    """One traced decode; host copies of its outputs."""
+    res = cache.decode(q, p, trace_cap=trace_cap)
+    torch.cuda.synchronize()
+    assert cache.status() == zha.ZHA_OK
+    return {k: v.cpu() for k, v in res.items()}
+
+
+def _heads(kh, G):
+    return range(kh * G, (kh + 1) * G)
+
+
+@pytest.mark.parametrize("name", ["wide_256k", "light_1m"])
 def test_fullsize_parity(name):
     w = W[name]
     inp = workloads.generate(w, "cuda")
     cache = _gpu_cache(w, inp)
+    trace_cap = oracle.level_nodes(w.capacity, w.c, 1)
+    steps = [0, w.steps - 1]
+    res = {s: _decode(cache, inp.Q[s], w.p, trace_cap) for s in steps}
     K_cpu, V_cpu, ref_cpu = inp.K.cpu(), inp.V.cpu(), inp.ref.cpu()
-    trees = [oracle.build(K_cpu[kh], w.n_tokens, ref_cpu[kh], w.c, w.D) for kh in range(w.h_kv)]
+    ht = oracle.build_heads(K_cpu, w.n_tokens, ref_cpu, w.c, w.D)
+    trees = [ht.head(kh) for kh in range(w.h_kv)]
     worst = check_build(cache, trees, sample=64)
     print(f"{name}: build worst relative error m={worst[0]:.2e} g={worst[1]:.2e} b={worst[2]:.2e}")
-    trace_cap = oracle.level_nodes(w.n_tokens, w.c, 1)
-    res = cache.decode(inp.Q[0], w.p, trace_cap=trace_cap)
-    torch.cuda.synchronize()
-    assert cache.status() == zha.ZHA_OK
-    amb = check_decode(res, trees, K_cpu, V_cpu, ref_cpu, inp.Q[0].cpu(), w.p, w.n_tokens, w.c, w.D, w.group,
-                       w.kv_dtype)
-    print(f"{name}: one decode step, {w.h_q} heads, ambiguous nodes {amb}")
+    for s in steps:
+        amb = check_decode(res[s], trees, K_cpu, V_cpu, ref_cpu, inp.Q[s].cpu(), w.p, w.n_tokens, w.c, w.D,
+                           w.group, w.kv_dtype, case=f"{name} step {s}")
+        print(f"{name}: step {s}, {w.h_q} heads, ambiguous nodes {amb}")
 
 
-def test_fullsize_parity_10m():
-    w = W["extreme_10m"]
+def test_fullsize_deep_schedule():
+    """deep_256k with its own schedule: two appends before every decode."""
+    w = W["deep_256k"]
+    assert w.appends_per_step == 2
     inp = workloads.generate(w, "cuda")
     cache = _gpu_cache(w, inp)
-    K0 = inp.K[0].cpu()
-    V0 = inp.V[0].cpu()
-    ref0 = inp.ref[0].cpu()
-    # build parity: a few nodes of every level of KV head 0, from the raw keys
-    rng = np.random.default_rng(0)
-    for level in range(1, w.D + 1):
-        g, b, m = cache.summaries(level)
-        n = m.shape[1]
-        for node in sorted(set(rng.integers(0, n, 3).tolist()) | {n - 1}):
-            mo, go, bo = oracle.node_summary(K0, w.n_tokens, ref0, w.c, level, node)
-            mg = m[0, node].double().cpu().numpy()
-            gg = g[0, node].double().cpu().numpy()
-            assert np.max(np.abs(mg - mo) / np.maximum(1.0, np.abs(mo))) <= 1e-5, ("m", level, node)
-            assert np.max(np.abs(gg - go) / np.maximum(1.0, np.abs(go).max())) <= 1e-5, ("g", level, node)
-    trace_cap = oracle.level_nodes(w.n_tokens, w.c, 1)
-    res = cache.decode(inp.Q[0], w.p, trace_cap=trace_cap)
+    trace_cap = oracle.level_nodes(w.capacity, w.c, 1)
+    checked = [0, 1, w.steps // 2, w.steps - 1]
+    res = {}
+    app = 0
+    for s in range(w.steps):
+        for _ in range(w.appends_per_step):
+            cache.append(inp.K_app[app], inp.V_app[app])
+            app += 1
+        if s in checked:
+            res[s] = _decode(cache, inp.Q[s], w.p, trace_cap)
+        else:
+            cache.decode(inp.Q[s], w.p)
     torch.cuda.synchronize()
     assert cache.status() == zha.ZHA_OK
-    tree0 = LazyTree(K0, w.n_tokens, w.c, w.D)
-    K_cpu = [K0]
-    V_cpu = [V0]
-    amb = check_decode(res, [tree0], K_cpu, V_cpu, [ref0], inp.Q[0].cpu(), w.p, w.n_tokens, w.c, w.D, w.group,
-                       w.kv_dtype, heads=range(w.group))
-    print(f"extreme_10m: one decode step, KV head 0 ({w.group} heads), ambiguous nodes {amb}")
+    assert cache.n_tokens == w.n_tokens + w.total_appends
+    # the appended rows are in the device cache now; the oracle replays the
+    # schedule on its own tree, one KV head at a time
+    G = w.group
+    for kh in range(w.h_kv):
+        K_h, V_h, ref_h = inp.K[kh].cpu(), inp.V[kh].cpu(), inp.ref[kh].cpu()
+        tree = oracle.build(K_h, w.n_tokens, ref_h, w.c, w.D, capacity=w.capacity)
+        n = w.n_tokens
+        for s in range(w.steps):
+            for _ in range(w.appends_per_step):
+                oracle.append_update(tree, K_h, ref_h)
+                n += 1
+            if s in checked:
+                amb = check_decode(res[s], {kh: tree}, {kh: K_h}, {kh: V_h}, {kh: ref_h}, inp.Q[s].cpu(), w.p, n,
+                                   w.c, w.D, G, w.kv_dtype, heads=_heads(kh, G),
+                                   case=f"deep_256k step {s} kv head {kh}")
+                print(f"deep_256k: step {s} (after {n - w.n_tokens} appends), KV head {kh}, ambiguous {amb}")
+        check_build(cache, [tree], heads=[kh], ids=touched_nodes(w.n_tokens, n, w.c, w.D))
+        check_build(cache, [tree], heads=[kh], sample=64, seed=kh)
+
+
+def test_fullsize_extreme_10m():
+    """extreme_10m with its own schedule: 64 decodes, then 1,024 appends."""
+    w = W["extreme_10m"]
+    assert w.appends_after == 1024 and w.appends_per_step == 0
+    inp = workloads.generate(w, "cuda")
+    cache = _gpu_cache(w, inp)
+    trace_cap = oracle.level_nodes(w.capacity, w.c, 1)
+    checked = [0, w.steps - 1]
+    res = {}
+    for s in range(w.steps):
+        if s in checked:
+            res[s] = _decode(cache, inp.Q[s], w.p, trace_cap)
+        else:
+            cache.decode(inp.Q[s], w.p)
+    for i in range(w.appends_after):
+        cache.append(inp.K_app[i], inp.V_app[i])
+    res["after"] = _decode(cache, inp.Q[0], w.p, trace_cap)
+    n_end = w.n_tokens + w.appends_after
+    assert cache.n_tokens == n_end
+    G = w.group
+    for kh in range(w.h_kv):
+        K_h, V_h, ref_h = inp.K[kh].cpu(), inp.V[kh].cpu(), inp.ref[kh].cpu()
+        tree = oracle.build(K_h, w.n_tokens, ref_h, w.c, w.D, capacity=w.capacity)
+        one = ({kh: tree}, {kh: K_h}, {kh: V_h}, {kh: ref_h})
+        for s in checked:
+            amb = check_decode(res[s], *one, inp.Q[s].cpu(), w.p, w.n_tokens, w.c, w.D, G, w.kv_dtype,
+                               heads=_heads(kh, G), case=f"extreme_10m step {s} kv head {kh}")
+            print(f"extreme_10m: step {s}, KV head {kh}, ambiguous nodes {amb}")
+        for _ in range(w.appends_after):
+            oracle.append_update(tree, K_h, ref_h)
+        assert tree.n_tokens == n_end
+        check_build(cache, [tree], heads=[kh], ids=touched_nodes(w.n_tokens, n_end, w.c, w.D))
+        check_build(cache, [tree], heads=[kh], sample=256, seed=kh)
+        amb = check_decode(res["after"], *one, inp.Q[0].cpu(), w.p, n_end, w.c, w.D, G, w.kv_dtype,
+                           heads=_heads(kh, G), case=f"extreme_10m after appends kv head {kh}")
+        print(f"extreme_10m: after {w.appends_after} appends, KV head {kh}, ambiguous nodes {amb}")
+        del tree, K_h, V_h

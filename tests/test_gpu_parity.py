@@ -1,8 +1,8 @@
 """CUDA path vs the fp64 oracle, through the C ABI (needs a B200).
 
-Cases are the five workloads' structures at sizes the oracle finishes in
-seconds (several top nodes, ragged tails); the full-size workloads are in
-test_gpu_fullsize.py.
+Cases are the tiny fp32 workload at its own size (all 64 queries) and the
+other workloads' structures at sizes the oracle finishes in seconds (several
+top nodes, ragged tails); the full-size workloads are in test_gpu_fullsize.py.
 """
 import numpy as np
 import pytest
@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 W = workloads.WORKLOADS
 CASES = {
-    "tiny_f32": W["tiny_f32_16k"].scaled(16384, steps=16),
+    "tiny_f32": W["tiny_f32_16k"],  # the tiny workload itself: 16,384 tokens, all 64 queries
     "wide": W["wide_256k"].scaled(16384 + 100, steps=3),
     "deep": W["deep_256k"].scaled(16384 + 37, steps=3),
     "light": W["light_1m"].scaled(300000 + 5, steps=3),
@@ -85,7 +85,7 @@ def test_decode_parity(name):
         torch.cuda.synchronize()
         assert c.cache.status() == 0
         amb += check_decode(res, c.trees, c.K, c.V, c.inp.ref, q.double().numpy(), w.p, c.n, w.c, w.D, w.group,
-                            w.kv_dtype)
+                            w.kv_dtype, case=f"{name} step {s}")
     print(f"{name}: {w.steps} steps, ambiguous nodes {amb}")
 
 
@@ -253,3 +253,63 @@ def test_errors_and_capacity():
     assert cache.status() == zha.ZHA_ERR_CAPACITY
     assert torch.all(res["n_leaf"] == 16)
     assert cache.status() == 0
+
+
+def test_barrier_timeout_reports_status_and_next_decode_is_clean():
+    """A team or grid barrier wait that runs out of its clock budget ends the
+    decode with ZHA_ERR_TIMEOUT in the device status word (the kernel
+    returns; nothing traps), and the next decode at the normal budget is
+    valid.  A budget of 0 cycles makes every wait that is not satisfied at
+    its first poll give up."""
+    c = get_case("light")
+    w = c.w
+    q = c.inp.Q[0].cuda()
+    cap = oracle.level_nodes(c.w.capacity, c.w.c, 1)
+    zha.zha_set_wait_budget(c.cache.ctx, 0)
+    seen = []
+    try:
+        for _ in range(3):
+            c.cache.decode(q, w.p, trace_cap=cap)
+            torch.cuda.synchronize()
+            st = c.cache.status()
+            seen.append(st)
+            assert st in (zha.ZHA_OK, zha.ZHA_ERR_TIMEOUT), st
+            if st == zha.ZHA_ERR_TIMEOUT:
+                break
+    finally:
+        zha.zha_set_wait_budget(c.cache.ctx, 2_000_000_000)
+    assert zha.ZHA_ERR_TIMEOUT in seen, seen
+    res = c.cache.decode(q, w.p, trace_cap=cap)
+    torch.cuda.synchronize()
+    assert c.cache.status() == zha.ZHA_OK
+    check_decode(res, c.trees, c.K, c.V, c.inp.ref, c.inp.Q[0].double().numpy(), w.p, c.n, w.c, w.D, w.group,
+                 w.kv_dtype, case="light after a timed-out decode")
+    with pytest.raises(zha.ZhaError) as e:
+        zha.zha_set_wait_budget(c.cache.ctx, -1)
+    assert e.value.code == zha.ZHA_ERR_BAD_ARG
+
+
+def test_injected_host_faults(monkeypatch):
+    """ZHA_FAULT makes the host side report a failure without touching the
+    GPU: cuda_launch fails zha_build before its launch, capacity fails
+    zha_append; with the variable unset both work again."""
+    N, c, D, R, h_kv, h_q, d = 200, 4, 2, 16, 1, 4, 64
+    cache, (K, V, ref), (dK, dV, dref) = _small_cache(N, c, D, R, h_kv, h_q, d, zha.ZHA_F32, 9, cap=N + 1)
+    monkeypatch.setenv("ZHA_FAULT", "cuda_launch")
+    with pytest.raises(zha.ZhaError) as e:
+        cache.build(dK, dV, N, dref)
+    assert e.value.code == zha.ZHA_ERR_CUDA
+    monkeypatch.setenv("ZHA_FAULT", "capacity")
+    k = torch.zeros(h_kv, d, device="cuda")
+    with pytest.raises(zha.ZhaError) as e:
+        cache.append(k, k)
+    assert e.value.code == zha.ZHA_ERR_CAPACITY
+    monkeypatch.delenv("ZHA_FAULT")
+    cache.build(dK, dV, N, dref)
+    cache.append(k, k)
+    torch.cuda.synchronize()
+    assert cache.n_tokens == N + 1 and cache.status() == zha.ZHA_OK
+    K[:, N] = 0.0
+    V[:, N] = 0.0
+    trees = oracle_trees(K, ref, N + 1, c, D)
+    check_build(cache, trees)

@@ -27,8 +27,8 @@ ZHA_BF16 = 1
 
 # every symbol include/zha.h declares
 EXPORTS = ["zha_workspace_bytes", "zha_create", "zha_destroy", "zha_build", "zha_append", "zha_decode",
-           "zha_dense_decode", "zha_dense_decode_static", "zha_device_status", "zha_set_phase_timer", "zha_n_tokens",
-           "zha_summary_layout", "zha_strerror"]
+           "zha_dense_decode", "zha_dense_decode_static", "zha_device_status", "zha_set_phase_timer",
+           "zha_set_wait_budget", "zha_n_tokens", "zha_summary_layout", "zha_strerror"]
 
 
 class ZhaError(RuntimeError):
@@ -46,7 +46,7 @@ class zha_config(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m tree_indexed_sparse_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python tree_indexed_sparse_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     CFG = ctypes.POINTER(zha_config)
@@ -70,6 +70,8 @@ def _load() -> ctypes.CDLL:
     lib.zha_device_status.restype = ctypes.c_int
     lib.zha_set_phase_timer.argtypes = [P, P]
     lib.zha_set_phase_timer.restype = ctypes.c_int
+    lib.zha_set_wait_budget.argtypes = [P, I64]
+    lib.zha_set_wait_budget.restype = ctypes.c_int
     lib.zha_n_tokens.argtypes = [P]
     lib.zha_n_tokens.restype = I64
     lib.zha_summary_layout.argtypes = [P, I32, ctypes.POINTER(I64), ctypes.POINTER(I64),
@@ -153,6 +155,11 @@ def zha_set_phase_timer(ctx, d_ns) -> None:
     """d_ns: device int64 tensor of D + 3 entries for the decode phase stamps
     (global timer, ns), or None to clear.  Keep it alive while set."""
     _check(lib.zha_set_phase_timer(ctx, _vp(d_ns)), "zha_set_phase_timer")
+
+
+def zha_set_wait_budget(ctx, cycles: int) -> None:
+    """Testing hook: clock cycles each inter-CTA wait of zha_decode may take."""
+    _check(lib.zha_set_wait_budget(ctx, int(cycles)), "zha_set_wait_budget")
 
 
 def zha_n_tokens(ctx) -> int:

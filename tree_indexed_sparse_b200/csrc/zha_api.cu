@@ -11,6 +11,7 @@
 
 #include "../../include/zha.h"
 #include "zha_internal.cuh"
+#include "zha_tma.cuh"
 
 using namespace zha;
 
@@ -24,6 +25,7 @@ struct zha_ctx {
     unsigned char *scratch_begin;
     int64_t scratch_bytes;
     int64_t *phase_ns;        // caller's device buffer for phase stamps, or null
+    long long wait_budget;    // clock cycles one inter-CTA barrier wait of the decode may take
     int decode_cta;
     int n_sm;
     int attn_cta;
@@ -136,6 +138,7 @@ Decode make_decode(zha_ctx *ctx) {
     Decode dc = ctx->scratch;
     dc.t = ctx->t;
     dc.phase_ns = ctx->phase_ns;
+    dc.wait_budget = ctx->wait_budget;
     return dc;
 }
 
@@ -164,6 +167,7 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
     if (!ctx) return ZHA_ERR_BAD_ARG;
     std::memset(ctx, 0, sizeof *ctx);
     ctx->cfg = *cfg;
+    ctx->wait_budget = WAIT_BUDGET_CYCLES;
     unsigned char *ws = static_cast<unsigned char *>(d_workspace);
     ctx->ws = ws;
     ctx->ws_bytes = ws_bytes;
@@ -335,6 +339,12 @@ int zha_set_phase_timer(zha_ctx *ctx, int64_t *d_ns) {
     if (!ctx) return ZHA_ERR_BAD_ARG;
     if (d_ns && (reinterpret_cast<uintptr_t>(d_ns) & 7u)) return ZHA_ERR_BAD_ARG;
     ctx->phase_ns = d_ns;
+    return ZHA_OK;
+}
+
+int zha_set_wait_budget(zha_ctx *ctx, int64_t cycles) {
+    if (!ctx || cycles < 0) return ZHA_ERR_BAD_ARG;
+    ctx->wait_budget = cycles > 0 ? (long long)cycles : 0;
     return ZHA_OK;
 }
 

@@ -44,12 +44,9 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_dense(const __grid_constant__ 
 template <typename KT, int HD, int G>
 static cudaError_t dense_impl(const Decode &dc, int n_cta, cudaStream_t s) {
     const size_t smem = ASmem<KT, HD, G>::bytes;
-    static size_t attr = 0;
-    if (smem > attr) {
-        cudaError_t err = cudaFuncSetAttribute(k_dense<KT, HD, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        attr = smem;
-    }
+    static PerDeviceMax<> attr;
+    const cudaError_t err = allow_smem(k_dense<KT, HD, G>, smem, attr);
+    if (err != cudaSuccess) return err;
     k_dense<KT, HD, G><<<n_cta, A_THREADS, smem, s>>>(dc);
     return cudaGetLastError();
 }

@@ -522,24 +522,17 @@ static cudaError_t build_impl(const Tree &t, cudaStream_t s, int n_sm) {
     const int warps = BUILD_THREADS / 32;
     const int tt = leaf_tile_tokens(t.c, R);
     size_t smem = (size_t)warps * (tt * R + (tt / t.c + 1) * R) * sizeof(float);
-    cudaError_t err;
-    static size_t leaf_attr = 0, parent_attr = 0;
-    if (smem > leaf_attr) {
-        err = cudaFuncSetAttribute(k_build_leaves<KT, HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        leaf_attr = smem;
-    }
+    static PerDeviceMax<> leaf_attr, parent_attr;
+    cudaError_t err = allow_smem(k_build_leaves<KT, HD, R>, smem, leaf_attr);
+    if (err != cudaSuccess) return err;
     const int64_t tiles = ((t.n_tokens + tt - 1) / tt) * t.h_kv;
     int grid = (int)std::min<int64_t>((tiles + warps - 1) / warps, (int64_t)n_sm * 8);
     k_build_leaves<KT, HD, R><<<grid, BUILD_THREADS, smem, s>>>(t);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     size_t psmem = (size_t)warps * (t.c * R + R) * sizeof(float);
-    if (psmem > parent_attr) {
-        err = cudaFuncSetAttribute(k_build_parents<HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem);
-        if (err != cudaSuccess) return err;
-        parent_attr = psmem;
-    }
+    err = allow_smem(k_build_parents<HD, R>, psmem, parent_attr);
+    if (err != cudaSuccess) return err;
     for (int level = 2; level <= t.D; ++level) {
         const int64_t work = (int64_t)t.n_level[level - 1] * t.h_kv;
         int pgrid = (int)std::min<int64_t>((work + warps - 1) / warps, (int64_t)n_sm * 8);
@@ -555,12 +548,9 @@ static cudaError_t append_impl(const Tree &t, const void *k, const void *v, cuda
     // per plane warp: one score per token of a leaf, or one estimate per child
     size_t smem = (size_t)R * (t.c > 32 ? t.c : 32) * sizeof(float);
     smem += (size_t)append_stage_bytes<KT, HD, R>(t.c, t.D);  // the shared copy of the rows every plane reads
-    static size_t attr = 0;
-    if (smem > attr) {
-        cudaError_t err = cudaFuncSetAttribute(k_append<KT, HD, R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        attr = smem;
-    }
+    static PerDeviceMax<> attr;
+    const cudaError_t err = allow_smem(k_append<KT, HD, R>, smem, attr);
+    if (err != cudaSuccess) return err;
     k_append<KT, HD, R><<<t.h_kv, 32 * R, smem, s>>>(t, reinterpret_cast<const KT *>(k), reinterpret_cast<const KT *>(v));
     return cudaGetLastError();
 }

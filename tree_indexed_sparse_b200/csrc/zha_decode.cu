@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__
     const int kh = router ? b / nbk : 0, tr = router ? b % nbk : 0;
     bool ok = true;
     if (router && warp < ACW) {
-        TeamSync ts{words + kh, abortw, a.status, &s_flag, nbk, 0u};
+        TeamSync ts{words + kh, abortw, a.status, &s_flag, nbk, 0u, a.wait_budget};
         ok = route_kvh<HD, R, G>(a, kh, tr, nbk, smem, ts);
     }
     __shared__ int s_ok;
@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__
     if (!ok && threadIdx.x == 0) s_ok = 0;
     __syncthreads();
     unsigned gepoch = 0;
-    if (s_ok && grid_barrier(words + h_kv, nb, gepoch, abortw, a.status, &s_flag)) {
+    if (s_ok && grid_barrier(words + h_kv, nb, gepoch, abortw, a.status, &s_flag, a.wait_budget)) {
         stamp(a, a.t.D);
         stage_map_init<false, StageCfg<KT, HD>::TT>(a, map);
         if (router && warp < ACW) write_lists<G>(a, kh, tr);
@@ -238,13 +238,9 @@ static size_t decode_smem() {
 template <typename KT, int HD, int R, int G>
 static cudaError_t decode_impl(const Decode &dc, int n_cta, cudaStream_t s) {
     const size_t smem = decode_smem<KT, HD, R, G>();
-    static size_t attr = 0;
-    if (smem > attr) {
-        cudaError_t err =
-            cudaFuncSetAttribute(k_decode<KT, HD, R, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        attr = smem;
-    }
+    static PerDeviceMax<> attr;
+    const cudaError_t err = allow_smem(k_decode<KT, HD, R, G>, smem, attr);
+    if (err != cudaSuccess) return err;
     // cooperative (the CTAs meet at barriers), and a programmatic dependent
     // of the previous kernel so that its launch overlaps that kernel's tail
     cudaLaunchConfig_t cfg = {};
@@ -265,13 +261,8 @@ static cudaError_t decode_impl(const Decode &dc, int n_cta, cudaStream_t s) {
 template <typename KT, int HD, int R, int G>
 static int decode_occupancy() {
     const size_t smem = decode_smem<KT, HD, R, G>();
-    static size_t attr = 0;
-    if (smem > attr) {
-        if (cudaFuncSetAttribute(k_decode<KT, HD, R, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-            cudaSuccess)
-            return 0;
-        attr = smem;
-    }
+    static PerDeviceMax<> attr;
+    if (allow_smem(k_decode<KT, HD, R, G>, smem, attr) != cudaSuccess) return 0;
     int blocks = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k_decode<KT, HD, R, G>, A_THREADS, smem) != cudaSuccess)
         return 0;

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "zha_attr.h"
+
 namespace zha {
 
 constexpr int MAXD = 16;          // deepest tree supported
@@ -65,6 +67,7 @@ struct Decode {
     int part_cap;
     unsigned *sync;               // barrier words, see zha_sync.cuh
     int64_t *phase_ns;            // nullable: globaltimer stamps per decode phase
+    long long wait_budget;        // clock cycles one inter-CTA barrier wait may take
     int32_t *status;
     float *out;
     int32_t *leaf_idx;
@@ -83,6 +86,19 @@ constexpr int32_t ZHA_TIMEOUT_CODE = -5;
 // status word helpers (first error wins)
 __device__ __forceinline__ void set_status(int32_t *status, int32_t code) {
     atomicCAS(status, 0, code);
+}
+
+// Let kernel `fn` use `bytes` of dynamic shared memory on the current device.
+// The attribute is per device: `rec` (one static record per kernel) makes
+// the call once per device and size.
+template <typename Fn>
+cudaError_t allow_smem(Fn *fn, size_t bytes, PerDeviceMax<> &rec) {
+    int dev = 0;
+    const cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    return static_cast<cudaError_t>(rec.raise(dev, (long long)bytes, [&](long long b) {
+        return static_cast<int>(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)b));
+    }));
 }
 
 // host-side launchers; each returns a cudaError_t (0 on success)

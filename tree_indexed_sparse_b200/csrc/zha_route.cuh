@@ -130,12 +130,13 @@ struct TeamSync {
     int *flag;
     int T;
     unsigned epoch;
+    long long budget;  // clock cycles one barrier wait may take
     __device__ __forceinline__ bool sync() {
         if (T == 1) {
             gsync();
             return true;
         }
-        return team_barrier(ctr, T, epoch, abortw, status, flag);
+        return team_barrier(ctr, T, epoch, abortw, status, flag, budget);
     }
 };
 

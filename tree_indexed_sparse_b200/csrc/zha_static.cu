@@ -9,6 +9,12 @@
 // one, so the library supplies the scratch itself, from static storage that
 // exists as soon as the module is loaded.
 //
+// Set-up: the first call on a device looks up the scratch's address there,
+// and, under CUDA's default lazy module loading, loading the module for that
+// device is what reserves the scratch (and the kernel code).  Callers make
+// that first call while setting up, before they serve and before any stream
+// capture; from then on a call allocates nothing.
+//
 // Limits: one call at a time per device.  Every call uses the same scratch, so
 // two calls in flight together (other streams, other host threads) race on it
 // and corrupt each other's outputs.  Configurations whose partials do not fit
@@ -19,6 +25,7 @@
 
 #include "../../include/zha.h"
 #include "zha_internal.cuh"
+#include "zha_tma.cuh"
 
 using namespace zha;
 
@@ -109,6 +116,7 @@ int zha_dense_decode_static(const zha_config *cfg, const void *d_K, const void *
     dc.part_cap = n_cta;
     dc.ticket = reinterpret_cast<uint32_t *>(ds.ptr + part_bytes);
     dc.status = d_status;
+    dc.wait_budget = WAIT_BUDGET_CYCLES;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the merge tickets must start at zero (a call that gave up on a wait can
     // leave them raised); the partials are written before they are read

@@ -5,7 +5,8 @@
 // its own epoch x the number of participants.  One L2 round trip per arrival,
 // no reset between barriers.  The counters are cleared by the last CTA to
 // leave the kernel (exit counter), so each launch starts from zero.  Every
-// wait is bounded by a clock budget; on expiry the CTA records
+// wait is bounded by a clock budget (Decode::wait_budget, about one second
+// unless a test lowers it); on expiry the CTA records
 // ZHA_TIMEOUT_CODE, raises the abort word and returns false, and every other
 // waiter returns false as soon as it sees the abort word.
 //
@@ -35,7 +36,9 @@ __device__ __forceinline__ void red_release_add_u32(unsigned *p, unsigned v) {
 }
 
 // Thread-level arrive-and-wait on a counter; false on abort or timeout.
-__device__ __noinline__ bool counter_arrive_wait(unsigned *ctr, unsigned target, unsigned *abortw, int32_t *status) {
+// `budget`: clock cycles the wait may take (Decode::wait_budget).
+__device__ __noinline__ bool counter_arrive_wait(unsigned *ctr, unsigned target, unsigned *abortw, int32_t *status,
+                                                 long long budget) {
     red_release_add_u32(ctr, 1u);
     const long long t0 = clock64();
     for (;;) {
@@ -47,7 +50,7 @@ __device__ __noinline__ bool counter_arrive_wait(unsigned *ctr, unsigned target,
             return true;
         }
         if (ab) return false;
-        if (clock64() - t0 > WAIT_BUDGET_CYCLES) {
+        if (clock64() - t0 > budget) {
             set_status(status, ZHA_TIMEOUT_CODE);
             atomicExch(abortw, 1u);
             return false;
@@ -59,11 +62,11 @@ __device__ __noinline__ bool counter_arrive_wait(unsigned *ctr, unsigned target,
 // routing threads (named barrier 1) of each CTA.  `epoch` counts the
 // barriers this CTA has passed on this counter.
 __device__ __forceinline__ bool team_barrier(unsigned *ctr, int members, unsigned &epoch, unsigned *abortw,
-                                             int32_t *status, int *s_flag) {
+                                             int32_t *status, int *s_flag, long long budget) {
     gsync();
     if (threadIdx.x == 0) {
         epoch += 1u;
-        *s_flag = counter_arrive_wait(ctr, epoch * (unsigned)members, abortw, status) ? 1 : 0;
+        *s_flag = counter_arrive_wait(ctr, epoch * (unsigned)members, abortw, status, budget) ? 1 : 0;
     }
     gsync();
     return *s_flag != 0;
@@ -71,11 +74,11 @@ __device__ __forceinline__ bool team_barrier(unsigned *ctr, int members, unsigne
 
 // The same for all threads of the CTA (__syncthreads).
 __device__ __forceinline__ bool grid_barrier(unsigned *ctr, int members, unsigned &epoch, unsigned *abortw,
-                                             int32_t *status, int *s_flag) {
+                                             int32_t *status, int *s_flag, long long budget) {
     __syncthreads();
     if (threadIdx.x == 0) {
         epoch += 1u;
-        *s_flag = counter_arrive_wait(ctr, epoch * (unsigned)members, abortw, status) ? 1 : 0;
+        *s_flag = counter_arrive_wait(ctr, epoch * (unsigned)members, abortw, status, budget) ? 1 : 0;
     }
     __syncthreads();
     return *s_flag != 0;
