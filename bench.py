@@ -335,7 +335,7 @@ def run_zha(args, rank, world, local):
         if i >= W:
             leaves_per_head.append(n_leaf.float().mean().item())
             vis_per_head.append(visited.float().mean().item())
-    per_step = per_step_all[W:]
+    timed_b = per_step_all[W:]
     ref_out = out.clone()
     assert cache.status() == 0, "device status not OK after the traced pass"
     if os.environ.get("ZHA_STEP_BYTES"):
@@ -425,9 +425,9 @@ def run_zha(args, rank, world, local):
         t_lvl.append([(ns[j + 1] - ns[j]) * 1e-3 for j in range(w.D)])
     torch.cuda.synchronize()
 
-    route_b = [s[0] for s in per_step]
-    attn_b = [s[1] for s in per_step]
-    app_b = [s[2] for s in per_step]
+    route_b = [s[0] for s in timed_b]
+    attn_b = [s[1] for s in timed_b]
+    app_b = [s[2] for s in timed_b]
     step_b = [r + a + p for r, a, p in zip(route_b, attn_b, app_b)]
     peak, peak_kind = peaks()
     gbs = sum(step_b) / (sum(t_step) * 1e-3) / 1e9
@@ -541,8 +541,8 @@ def run_zha(args, rank, world, local):
         "routing": {"kept_leaves_per_head": statistics.mean(leaves_per_head),
                     "nodes_visited_per_head": statistics.mean(vis_per_head),
                     "keys_touched_frac": statistics.mean(leaves_per_head) * w.c / w.n_tokens,
-                    "union_slots_per_step": statistics.mean(s[3] for s in per_step),
-                    "union_slots_per_level": {f"level_{lv}": statistics.mean(s[5][lv] for s in per_step)
+                    "union_slots_per_step": statistics.mean(s[3] for s in timed_b),
+                    "union_slots_per_level": {f"level_{lv}": statistics.mean(s[5][lv] for s in timed_b)
                                               for lv in range(w.D, 0, -1)},
                     "timed_pass_reproduces_traced": bool(same)},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
