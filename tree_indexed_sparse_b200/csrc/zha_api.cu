@@ -63,7 +63,7 @@ struct Layout {
     int64_t node_cap[MAXD], slot_cap[MAXD];
     int64_t g_off[MAXD], b_off[MAXD], m_off[MAXD];
     int64_t kid_off[MAXD], kmask_off[MAXD];
-    int64_t seg_off, hseg_off, lvl_off, cur_off, scores_off, snode_off, skeep_off, tmax_off, tcnt_off, tsum_off;
+    int64_t seg_off, hseg_off, lvl_off, rdsc_off, scores_off, snode_off, skeep_off, tmax_off, tcnt_off, tsum_off;
     int64_t hcnt_off, hmass_off, cw_off, cs_off, ccnt_off, ticket_off, part_off, sync_off, status_off;
     int64_t scratch_off, total;
     int64_t score_cap;
@@ -105,7 +105,7 @@ void make_layout(const zha_config *cfg, Layout *L) {
     take(L->seg_off, (int64_t)MAXD * H * SEG_CAP * 4);
     take(L->hseg_off, (int64_t)MAXD * H * SEG_CAP * G * 4);
     take(L->lvl_off, (int64_t)MAXD * H * 2 * 4);
-    take(L->cur_off, H * 4);
+    take(L->rdsc_off, H * 2 * LOC_CAP * G * 4);
     take(L->scores_off, H * sc * G * 4);
     take(L->snode_off, H * sc * 4);
     take(L->skeep_off, H * sc + 4);
@@ -199,7 +199,7 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
     d.seg = reinterpret_cast<uint32_t *>(ws + L.seg_off);
     d.hseg = reinterpret_cast<uint32_t *>(ws + L.hseg_off);
     d.lvl = reinterpret_cast<int32_t *>(ws + L.lvl_off);
-    d.cur = reinterpret_cast<int32_t *>(ws + L.cur_off);
+    d.rd_scores = reinterpret_cast<float *>(ws + L.rdsc_off);
     d.scores = reinterpret_cast<float *>(ws + L.scores_off);
     d.slot_node = reinterpret_cast<int32_t *>(ws + L.snode_off);
     d.slot_keep = reinterpret_cast<uint8_t *>(ws + L.skeep_off);

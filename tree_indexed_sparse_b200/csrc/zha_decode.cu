@@ -7,11 +7,11 @@
 // expand only their children, repeat down to the raw entries; "Zyphra
 // 分层注意力（ZHA）…", section "机制拆解：树形索引如何高效筛选长上下文"):
 //   the grid's CTAs are split into h_kv teams of nbk = gridDim / h_kv CTAs,
-//   one per KV head, which route independently, level D .. 1:
-//     a frontier whose summaries fit SMALL_BYTES is scored and cut by the
-//     team's first CTA alone, with no inter-CTA barrier, and so are the small
-//     levels that follow it; the rest of the team waits at one team barrier;
-//     a larger frontier is split over the whole team (zha_route.cuh).
+//   one per KV head, which route independently, level D .. 1: a small
+//   frontier is scored and cut by every CTA of the team on its own (no
+//   inter-CTA wait), a mid-size one is scored in slices and cut by every CTA
+//   after one team barrier, and a large one is scored and cut in slices
+//   against the team's histograms (zha_route.cuh, LevelMode).
 //   a grid barrier ends the routing; every CTA then writes the leaf lists and
 //   traces of its own segments while the attention over the kept leaves plus
 //   the sink token runs split over every CTA (zha_attend.cuh); the last CTA
@@ -24,8 +24,6 @@
 #include "zha_sync.cuh"
 
 namespace zha {
-
-constexpr int64_t SMALL_BYTES = 256 * 1024;
 
 __device__ __forceinline__ void stamp(const Decode &a, int i) {
     if (a.phase_ns && blockIdx.x == 0 && threadIdx.x == 0) {
@@ -94,68 +92,65 @@ __device__ __noinline__ void write_lists(const Decode &a, int kh, int tr) {
     }
 }
 
-// All routing levels of KV head kh as rank tr of a team of T CTAs.  Warps 0-7.
+// All routing levels of KV head kh as rank tr of a team of T CTAs, level D
+// down to 1, each in the way level_mode picks from its frontier size.  The
+// parents of a level are either the kept list every CTA holds in shared
+// memory (after an LV_ALL or LV_SPLIT level) or the segments of an LV_TEAM
+// level in global memory; a level routed by every CTA after an LV_TEAM level
+// first copies those segments in.  Warps 0-7.
 template <int HD, int R, int G>
 __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, unsigned char *smem, TeamSync &ts) {
     using SM = RouteSmem<G>;
     uint32_t *pref = reinterpret_cast<uint32_t *>(smem + SM::off_pref);
     uint32_t *scratch = reinterpret_cast<uint32_t *>(smem + SM::off_misc) + 8;
+    int32_t *pid = reinterpret_cast<int32_t *>(smem + SM::off_pid);
+    uint8_t *pmk = smem + SM::off_pmk;
     const int D = a.t.D;
-    const int64_t node_bytes = (int64_t)R * (HD + 1) * 4;
     int64_t vis[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) vis[h] = 0;
-    int l = D;
-    int Tp = 1;       // team size and frontier size of level l + 1
+    int Tp = 1;            // team size and frontier size of level l + 1 (its segments)
     int64_t Sp = 0;
     int64_t S = a.t.n_level[D - 1];
-    auto small = [&](int64_t s) { return T == 1 || (s <= SOLO_MAX && s * node_bytes <= SMALL_BYTES); };
+    bool par_local = true;  // level l's parents are the kept list in pid / pmk
+    int buf = 0;           // team score buffer of the next LV_SPLIT level
     stages_init<G>(smem);
 #pragma unroll 1
-    while (l >= 1) {
-        if (small(S)) {
-            if (tr == 0) {
-                TeamSync solo = ts;
-                solo.T = 1;
-#pragma unroll 1
-                for (;;) {
-                    uint32_t F[G];
-                    int Tout;
-                    route_level<HD, R, G>(a, l, kh, 1, 0, S, Tp, Sp, smem, solo, F, Tout);
-#pragma unroll
-                    for (int h = 0; h < G; ++h) vis[h] += F[h];
-                    if (l > 1) stamp(a, D - l + 1);
-                    Tp = 1;
-                    Sp = S;
-                    --l;
-                    if (l < 1) break;
-                    S = load_segments(a, l + 1, kh, 1, pref, scratch) * a.t.c;
-                    if (!small(S)) break;
-                }
-                if (threadIdx.x == 0) a.cur[kh] = l;
+    for (int l = D; l >= 1; --l) {
+        const int mode = level_mode<HD, R>(S, T);
+        uint32_t F[G];
+        int64_t Snext = 0;
+        if (mode != LV_TEAM) {
+            if (!par_local) {
+                // the whole kept list of level l + 1 from its segments
+                Level P;
+                P.l = l;
+                P.kh = kh;
+                P.Tp = Tp;
+                P.Sp = Sp;
+                int64_t k0 = 0;
+                load_parents(a, P, 0, S, pref, pid, pmk, k0);
+                gsync();
+                par_local = true;
             }
-            if (T > 1) {
-                if (!ts.sync()) return false;
-                l = __ldcg(a.cur + kh);
-                if (l >= 1) {
-                    const int32_t *lv = lvl_ptr(a, l + 1, kh);
-                    Tp = __ldcg(lv);
-                    Sp = __ldcg(lv + 1);
-                    S = load_segments(a, l + 1, kh, Tp, pref, scratch) * a.t.c;
-                }
-            }
+            int64_t nk = 0;
+            if (!route_level_rd<HD, R, G>(a, l, kh, T, tr, S, mode, buf, smem, ts, F, nk)) return false;
+            if (mode == LV_SPLIT) buf ^= 1;
+            Tp = 1;
+            Sp = S;
+            Snext = nk * a.t.c;
         } else {
-            uint32_t F[G];
             int Tout;
-            if (!route_level<HD, R, G>(a, l, kh, T, tr, S, Tp, Sp, smem, ts, F, Tout)) return false;
-#pragma unroll
-            for (int h = 0; h < G; ++h) vis[h] += F[h];
-            if (l > 1) stamp(a, D - l + 1);
+            if (!route_level<HD, R, G>(a, l, kh, T, tr, S, Tp, Sp, par_local, smem, ts, F, Tout)) return false;
+            par_local = false;
             Tp = Tout;
             Sp = S;
-            --l;
-            if (l >= 1) S = load_segments(a, l + 1, kh, Tp, pref, scratch) * a.t.c;
+            if (l > 1) Snext = load_segments(a, l, kh, Tp, pref, scratch) * a.t.c;
         }
+#pragma unroll
+        for (int h = 0; h < G; ++h) vis[h] += F[h];
+        if (l > 1) stamp(a, D - l + 1);
+        S = Snext;
     }
     stages_inval<G>(smem);
     if (tr == 0 && threadIdx.x < G && a.visited) {

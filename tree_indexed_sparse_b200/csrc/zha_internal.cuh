@@ -14,6 +14,7 @@ constexpr int NB = 1024;          // top-p buckets per round
 constexpr int CAND_MAX = 1024;    // boundary candidates ranked exactly per head
 constexpr int SEG_CAP = 256;      // most CTAs in one KV head's team (grid <= 256 CTAs)
 constexpr int HIST_ROUNDS = 3;    // bucket widths 1/32, 1/32768, 1/2^25 of a log-mass unit
+constexpr int LOC_CAP = 2048;     // frontier slots one CTA holds in shared memory
 
 // Summary store of every level (pointers for KV head 0; head stride is
 // node_cap[l] rows).  g: [node][R][d], b and m: [node][R].
@@ -49,8 +50,8 @@ struct Decode {
     uint32_t *seg;                // [MAXD][h_kv][SEG_CAP] kept nodes per team rank
     uint32_t *hseg;               // [MAXD][h_kv][SEG_CAP][G] kept nodes per team rank and head
     int32_t *lvl;                 // [MAXD][h_kv][2] team size and frontier size of level l
-    int32_t *cur;                 // [h_kv] next level after a one-CTA run
     float *scores;                // [h_kv][score_cap][G] scores when a rank's slots overflow shared memory
+    float *rd_scores;             // [h_kv][2][LOC_CAP][G] slices of LV_SPLIT levels (two buffers in turn)
     int32_t *slot_node;           // [h_kv][score_cap] node of each slot (same case)
     uint8_t *slot_keep;           // [h_kv][score_cap] kept heads of each slot (same case)
     int64_t score_cap;

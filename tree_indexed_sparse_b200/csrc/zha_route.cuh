@@ -11,9 +11,19 @@
 //
 // The frontier of KV head kh is the union over its G query heads: the
 // children of every node any head kept one level up, each with the bitmask of
-// the heads that kept its parent.  It is split into T contiguous slot ranges,
-// one per CTA of the team (T = 1 for a frontier small enough for one SM).
-// Each CTA streams its nodes' summary rows once (bulk copies into per-warp
+// the heads that kept its parent.  A team of T CTAs routes it, in one of
+// three ways (LevelMode), chosen by the frontier size alone:
+//   LV_ALL (small frontiers): every CTA scores every slot itself and cuts
+//   the whole frontier, so every CTA knows the kept list without waiting for
+//   another (the summaries come from L2 after the first CTA's read);
+//   LV_SPLIT (up to RDS_MAX slots): each CTA scores a contiguous slice of
+//   the slots into a team buffer, one team barrier, then every CTA copies all
+//   the scores in and cuts the whole frontier itself;
+//   LV_TEAM (larger): each CTA scores and cuts its own slice against the
+//   team's histograms (below) and writes its kept nodes as a segment.
+// Every CTA of a team computes the same integers in the same order, so the
+// cuts of the first two ways agree on every CTA.
+// Scoring streams each node's summary rows once (bulk copies into per-warp
 // shared-memory stages) and scores each node for all G heads.  Masses are
 // w = exp(est - M_h) in 2^-40 fixed point (integer sums are exact and do not
 // depend on the order of addition), M_h the maximum over the frontier, and
@@ -31,11 +41,8 @@
 //   nodes of the final bucket are ranked exactly as above; a final bucket
 //   still larger than CAND_MAX holds estimates within 2^-25 of each other and
 //   is taken in node-id order.
-// Team barriers separate: the maxima (A), each histogram round (B), the
-// boundary lists (C) and the written segments (D).  A team level of at most
-// RC_MAX slots skips B and C: after A every CTA copies all of the team's
-// scores and runs the histogram cut on them alone (same integer sums, same
-// decisions), keeping its own slots.
+// On an LV_TEAM level, team barriers separate: the maxima (A), each
+// histogram round (B), the boundary lists (C) and the written segments (D).
 //
 // Code size matters here as much as arithmetic: every function runs once per
 // level on little data, so cold instruction fetch dominates unless the code is
@@ -51,11 +58,22 @@
 
 namespace zha {
 
-constexpr int LOC_CAP = 2048;          // local slots held in shared memory
-constexpr int PWIN = LOC_CAP / 2 + 2;  // parents of LOC_CAP consecutive slots (c >= 2)
-constexpr int SOLO_MAX = GT;           // one-CTA levels up to this many slots (sorted by one warp per head)
+constexpr int PAR_CAP = LOC_CAP;        // parents held in shared memory: a whole kept list, or the
+                                        // window of LOC_CAP consecutive slots (c >= 2)
+constexpr int SOLO_MAX = GT;           // one-CTA cuts up to this many slots are sorted (one warp per head)
 constexpr int RANK_MAX = 32;           // ... ranked slot against slot up to this many (shorter code)
-constexpr int RC_MAX = 512;            // team levels up to this many slots: cut by each CTA on its own
+constexpr int RDA_SLOTS = SOLO_MAX;     // every CTA scores every slot itself up to this many slots
+constexpr int64_t RDA_BYTES = 160 * 1024;  // ... and this many summary bytes
+constexpr int RDS_MAX = 1000;           // scored in slices and cut by every CTA up to this many slots (a
+                                        // larger frontier is cut faster in slices against team histograms)
+
+// How a level is routed (the same choice on every CTA of the team):
+//   LV_ALL   every CTA scores and cuts the whole frontier (no inter-CTA wait);
+//   LV_SPLIT each CTA scores a slice, one team barrier, every CTA cuts the
+//            whole frontier from all the scores;
+//   LV_TEAM  each CTA scores and cuts a slice against the team's histograms
+//            (barriers A-D), and writes its slice's kept nodes as a segment.
+enum LevelMode : int { LV_ALL = 0, LV_SPLIT = 1, LV_TEAM = 2 };
 
 enum CutMode : int { CUT_OPEN = 0, CUT_RANK = 1, CUT_ORDER = 2, CUT_ALL = 3, CUT_NONE = 4 };
 
@@ -78,10 +96,10 @@ constexpr int SW_N = (GT / 32) * SW_STAGES;  // stages of the CTA
 // with the histogram and boundary lists, which are used only after scoring.
 template <int G>
 struct RouteSmem {
-    // [LOC_CAP][G] f32 local scores; on a redundantly cut team level
-    // (at most RC_MAX slots) every score of the level, [S][G]
+    // [LOC_CAP][G] f32 scores: this CTA's slots of a team level, or every
+    // slot of a level cut by every CTA (at most RDS_MAX slots)
     static constexpr size_t off_sc = 0;
-    static_assert(RC_MAX <= LOC_CAP, "a redundantly cut level fits the local score array");
+    static_assert(RDS_MAX <= LOC_CAP, "a level cut by every CTA fits the local score array");
     static constexpr size_t off_node = off_sc + (size_t)LOC_CAP * G * 4;  // [LOC_CAP] i32
     static constexpr size_t off_keep = off_node + (size_t)LOC_CAP * 4;    // [LOC_CAP] u8
     static constexpr size_t off_u = off_keep + LOC_CAP;                   // union: chunks | cut scratch
@@ -94,9 +112,9 @@ struct RouteSmem {
     static constexpr size_t u_end = off_own + (size_t)G * CAND_MAX * 4 > off_u + (size_t)SW_N * SW_BYTES
                                         ? off_own + (size_t)G * CAND_MAX * 4
                                         : off_u + (size_t)SW_N * SW_BYTES;
-    static constexpr size_t off_pid = u_end;                              // [PWIN] i32
-    static constexpr size_t off_pmk = off_pid + (size_t)PWIN * 4;         // [PWIN] u8
-    static constexpr size_t off_pref = (off_pmk + PWIN + 15) / 16 * 16;   // [SEG_CAP + 1] u32
+    static constexpr size_t off_pid = u_end;                              // [PAR_CAP] i32 parents
+    static constexpr size_t off_pmk = off_pid + (size_t)PAR_CAP * 4;      // [PAR_CAP] u8 their head masks
+    static constexpr size_t off_pref = (off_pmk + PAR_CAP + 15) / 16 * 16;  // [SEG_CAP + 1] u32
     static constexpr size_t off_cut = (off_pref + (SEG_CAP + 1) * 4 + 15) / 16 * 16;  // [G] HeadCut
     static constexpr size_t off_wm = (off_cut + G * sizeof(HeadCut) + 15) / 16 * 16;  // [8][G] f32 warp maxima
     static constexpr size_t off_wc = off_wm + 8 * G * 4;                  // [8][G] u32 warp counts
@@ -1085,134 +1103,14 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
     return true;
 }
 
-// Classification of a redundantly cut level (every score in shared memory,
-// LA: all S slots): every slot is visited for the boundary lists and for the
-// boundary mass before this CTA's range (CUT_ORDER heads, into obefore[h]);
-// keep bits and own[] entries are written for this CTA's slots [s0, s0 + n)
-// only (keep: L's local array).
-template <int G>
-__device__ __noinline__ void classify_rc(const Level &LA, int64_t s0, int64_t n, uint8_t *keep, const HeadCut *cut,
-                                         unsigned long long *lw, uint32_t *ls, uint32_t *lcnt, uint32_t *own,
-                                         uint32_t *own_cnt, unsigned long long *obefore) {
-    const int lane = threadIdx.x & 31;
-    const int64_t iters = (LA.n + GT - 1) / GT;
-#pragma unroll 1
-    for (int64_t it = 0; it < iters; ++it) {
-        const int64_t s = it * GT + threadIdx.x;
-        const bool mine = s >= s0 && s < s0 + n;
-        uint32_t kbits = 0u;
-        float ev[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) ev[h] = s < LA.n ? LA.sc[s * G + h] : -INFINITY;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const HeadCut &H = cut[h];
-            const float e = ev[h];
-            bool cand = false;
-            unsigned long long w = 0ull;
-            if (e != -INFINITY) {
-                if (H.mode == CUT_ALL) {
-                    kbits |= 1u << h;
-                } else if (H.mode == CUT_RANK || H.mode == CUT_ORDER) {
-                    const int pc = path_cmp(H, e, H.rounds);
-                    if (pc < 0) kbits |= 1u << h;
-                    else if (pc == 0) {
-                        w = mass_fx(expf(e - H.M));
-                        if (H.mode == CUT_RANK) cand = true;
-                        else if (s < s0) atomicAdd(&obefore[h], w);
-                    }
-                }
-            }
-            const unsigned bal = __ballot_sync(FULL, cand);
-            if (bal) {
-                const unsigned bown = __ballot_sync(FULL, cand && mine);
-                const int leader = __ffs(bal) - 1;
-                uint32_t base = 0, obase = 0;
-                if (lane == leader) {
-                    base = atomicAdd(&lcnt[h], (uint32_t)__popc(bal));
-                    if (bown) obase = atomicAdd(own_cnt, (uint32_t)__popc(bown));
-                }
-                base = __shfl_sync(FULL, base, leader);
-                obase = __shfl_sync(FULL, obase, leader);
-                if (cand) {
-                    const uint32_t at = base + __popc(bal & ((1u << lane) - 1u));
-                    if (at < (uint32_t)CAND_MAX) {
-                        lw[h * CAND_MAX + at] = w;
-                        ls[h * CAND_MAX + at] = (uint32_t)s;
-                    }
-                    if (mine) {
-                        const uint32_t o = obase + __popc(bown & ((1u << lane) - 1u));
-                        if (o < (uint32_t)(G * CAND_MAX)) own[o] = ((uint32_t)(s - s0) << 3) | (uint32_t)h;
-                    }
-                }
-            }
-        }
-        if (mine) keep[s - s0] = (uint8_t)kbits;
-    }
-    gsync();
-}
-
-// The cut of a small team level (S <= RC_MAX; every score fits the local
-// score array): after the maxima barrier each CTA copies the team's
-// scores in and cuts the whole frontier by itself (the same integer
-// histograms as the team's, hence the same decisions), then keeps its own
-// slots.  No histogram atomics and no barriers B and C.  L.sc points at this
-// CTA's first slot inside the shared copy.
-template <int G>
-__device__ __noinline__ void rc_cut(const Decode &a, const Level &L, unsigned char *smem) {
-    using SM = RouteSmem<G>;
-    HeadCut *cut = reinterpret_cast<HeadCut *>(smem + SM::off_cut);
-    unsigned long long *red = reinterpret_cast<unsigned long long *>(smem + SM::off_red);
-    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + SM::off_misc);
-    uint32_t *hc = reinterpret_cast<uint32_t *>(smem + SM::off_hc);
-    unsigned long long *hm = reinterpret_cast<unsigned long long *>(smem + SM::off_hm);
-    unsigned long long *cw = reinterpret_cast<unsigned long long *>(smem + SM::off_cw);
-    uint32_t *cs = reinterpret_cast<uint32_t *>(smem + SM::off_cs);
-    uint32_t *own = reinterpret_cast<uint32_t *>(smem + SM::off_own);
-    const int tid = threadIdx.x;
-    Level LA = L;
-    LA.s0 = 0;
-    LA.n = L.S;
-    LA.T = 1;
-    LA.tr = 0;
-    LA.sc = reinterpret_cast<float *>(smem + SM::off_sc);
-#pragma unroll 1
-    for (int r = 0; r < HIST_ROUNDS; ++r) {
-        bool open = false;
-#pragma unroll 1
-        for (int h = 0; h < G; ++h) open |= cut[h].mode == CUT_OPEN;
-        if (!open) break;
-        local_hist<G>(LA, cut, r, hc, hm);
-        find_cut<G>(cut, r, hc, nullptr, hm, a.p, red);
-    }
-    unsigned long long *obefore = red + 64;
-    if (tid < 8) misc[tid] = 0u;  // [0]: own count, [4 + h]: list counters
-    if (tid < G) obefore[tid] = 0ull;
-    gsync();
-    classify_rc<G>(LA, L.s0, L.n, L.keep, cut, cw, cs, misc + 4, own, misc, obefore);
-    bool any_order = false, any_rank = false;
-#pragma unroll 1
-    for (int h = 0; h < G; ++h) {
-        any_order |= cut[h].mode == CUT_ORDER;
-        any_rank |= cut[h].mode == CUT_RANK;
-    }
-    const uint32_t n_own = min(misc[0], (uint32_t)(G * CAND_MAX));
-    if (any_rank && n_own > 0) rank_own<G>(L, cut, cw, cs, own, n_own);
-    if (any_order) {
-        unsigned long long *base = red + 72;
-        if (tid < G) base[tid] = cut[tid].C + obefore[tid];
-        gsync();
-        order_own<G>(L, cut, base, red);
-    }
-}
-
 // Score and cut level l of KV head kh as rank tr of a team of T CTAs (T = 1:
 // this CTA alone).  `S` is the frontier size, `pref`/Tp/Sp the parent level's
 // segments (loaded by the caller).  F[h] receives the frontier counts.
 // Returns false when a team barrier gave up.
 template <int HD, int R, int G>
 __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, int tr, int64_t S, int Tp, int64_t Sp,
-                                         unsigned char *smem, TeamSync &ts, uint32_t (&F)[G], int &Tout) {
+                                         bool par_local, unsigned char *smem, TeamSync &ts, uint32_t (&F)[G],
+                                         int &Tout) {
     using SM = RouteSmem<G>;
     HeadCut *cut = reinterpret_cast<HeadCut *>(smem + SM::off_cut);
     uint32_t *pref = reinterpret_cast<uint32_t *>(smem + SM::off_pref);
@@ -1232,16 +1130,13 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
     L.Sp = Sp;
     Tout = T;
     const bool team = T > 1;
-    // a team level whose scores all fit shared memory is cut by every CTA
-    // on its own copy of them (rc_cut); the scores go out through global
-    const bool rc = team && S <= RC_MAX;
     if (L.n > LOC_CAP) {
         const int64_t base = (int64_t)kh * a.score_cap + L.s0;
         L.sc = a.scores + base * G;
         L.node = a.slot_node + base;
         L.keep = a.slot_keep + base;
     } else {
-        L.sc = rc ? a.scores + ((int64_t)kh * a.score_cap + L.s0) * G : reinterpret_cast<float *>(smem + SM::off_sc);
+        L.sc = reinterpret_cast<float *>(smem + SM::off_sc);
         L.node = reinterpret_cast<int32_t *>(smem + SM::off_node);
         L.keep = smem + SM::off_keep;
     }
@@ -1255,8 +1150,8 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
 #pragma unroll 1
     for (int64_t c0 = L.s0; c0 < L.s0 + L.n; c0 += LOC_CAP) {
         const int64_t c1 = min(L.s0 + L.n, c0 + LOC_CAP);
-        int64_t k0 = 0;
-        if (!L.top) load_parents(a, L, c0, c1, pref, pid, pmk, k0);
+        int64_t k0 = 0;  // parents already local: the whole kept list from rank 0
+        if (!L.top && !par_local) load_parents(a, L, c0, c1, pref, pid, pmk, k0);
         gsync();
         score_chunks<HD, R, G>(a, L, c0, c1, k0, pid, pmk, smem, wm, wc);
         gsync();
@@ -1336,22 +1231,6 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
         solo_cut<G>(L, cut, reinterpret_cast<unsigned long long *>(smem + SM::off_hm), a.p);
     } else if (solo && L.n <= SOLO_MAX) {
         sort_cut<G>(L, cut, a.p);
-    } else if (rc) {
-        // every score of the team into shared memory (written before barrier A)
-        float *alls = reinterpret_cast<float *>(smem + SM::off_sc);
-        const float *src = a.scores + (int64_t)kh * a.score_cap * G;
-        if constexpr (G == 4) {
-            const float4 *s4 = reinterpret_cast<const float4 *>(src);
-            float4 *d4 = reinterpret_cast<float4 *>(alls);
-#pragma unroll 8
-            for (int64_t i = tid; i < S; i += GT) d4[i] = __ldcg(s4 + i);
-        } else {
-#pragma unroll 8
-            for (int64_t i = tid; i < S * G; i += GT) alls[i] = __ldcg(src + i);
-        }
-        gsync();
-        L.sc = alls + L.s0 * G;
-        rc_cut<G>(a, L, smem);
     } else {
         if (!hist_cut<G>(a, L, smem, ts)) return false;
     }
@@ -1363,6 +1242,234 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
     } else {
         gsync();
     }
+    return true;
+}
+
+// ---- levels cut by every CTA over the whole frontier ------------------------------
+
+// The way level l is routed by a team of T CTAs, from its frontier size S
+// (the same on every CTA).
+template <int HD, int R>
+__device__ __forceinline__ int level_mode(int64_t S, int T) {
+    constexpr int64_t node_bytes = (int64_t)R * (HD + 1) * 4;
+    if (S <= LOC_CAP && (T == 1 || (S <= RDA_SLOTS && S * node_bytes <= RDA_BYTES))) return LV_ALL;
+    if (S <= RDS_MAX) return LV_SPLIT;
+    return LV_TEAM;
+}
+
+// Node of frontier slot s of level l whose parents are the kept list in
+// pid (none at the top level): child s % c of parent s / c; -1 past the
+// level's last node.
+__device__ __forceinline__ int32_t slot_node(const Decode &a, int l, bool top, const int32_t *pid, int64_t s) {
+    const int c = a.t.c, clog = a.t.c_log2;
+    int64_t nd = s;
+    if (!top) {
+        const int64_t k = clog >= 0 ? (s >> clog) : s / c;
+        nd = (int64_t)pid[k] * c + (s - k * c);
+    }
+    return nd < a.t.n_level[l - 1] ? (int32_t)nd : -1;
+}
+
+// Score and cut level l of KV head kh (frontier of S <= LOC_CAP slots) so
+// that every CTA of the team ends with the same kept list, ascending, in
+// pid / pmk (*nk entries) -- the parents of the next level -- without
+// waiting for another CTA to write it.  On entry pid / pmk hold the kept
+// list of level l + 1 (unused at the top level).
+//   LV_ALL: this CTA scores every slot.
+//   LV_SPLIT: this CTA scores its slice [S r / T, S (r + 1) / T) into the
+//   team's score buffer `buf` (global); after one team barrier it copies
+//   every slot's scores in.  Consecutive LV_SPLIT levels use the two
+//   buffers in turn: a CTA writes a buffer again only after the barrier of
+//   the LV_SPLIT level in between, which every CTA reaches after reading it.
+// Then every CTA cuts the whole frontier alone (one-CTA rank, sort or
+// histogram path; the same integers on every CTA) and compacts the kept
+// slots.  Rank 0 also writes the kept list as the level's single segment
+// (team size 1), which the leaf lists, the trace and the attention read
+// after the grid barrier.  F[h]: frontier counts.  false: the barrier gave
+// up.
+template <int HD, int R, int G>
+__device__ __noinline__ bool route_level_rd(const Decode &a, int l, int kh, int T, int tr, int64_t S, int mode,
+                                            int buf, unsigned char *smem, TeamSync &ts, uint32_t (&F)[G],
+                                            int64_t &nk) {
+    using SM = RouteSmem<G>;
+    HeadCut *cut = reinterpret_cast<HeadCut *>(smem + SM::off_cut);
+    float *wm = reinterpret_cast<float *>(smem + SM::off_wm);
+    uint32_t *wc = reinterpret_cast<uint32_t *>(smem + SM::off_wc);
+    int32_t *pid = reinterpret_cast<int32_t *>(smem + SM::off_pid);
+    uint8_t *pmk = smem + SM::off_pmk;
+    float *sc = reinterpret_cast<float *>(smem + SM::off_sc);
+    int32_t *node = reinterpret_cast<int32_t *>(smem + SM::off_node);
+    uint8_t *keep = smem + SM::off_keep;
+    uint32_t *red32 = reinterpret_cast<uint32_t *>(smem + SM::off_red);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool top = (l == a.t.D);
+    float *gsc = a.rd_scores + (int64_t)(kh * 2 + buf) * LOC_CAP * G;
+    Level L;
+    L.l = l;
+    L.kh = kh;
+    L.T = 1;
+    L.tr = 0;
+    L.top = top;
+    L.S = S;
+    L.Tp = 1;
+    L.Sp = 0;
+    L.keep = keep;
+    if (mode == LV_ALL) {
+        L.s0 = 0;
+        L.n = S;
+        L.sc = sc;
+        L.node = node;
+    } else {
+        L.s0 = seg_start(S, T, tr);
+        L.n = seg_start(S, T, tr + 1) - L.s0;
+        L.sc = gsc + L.s0 * G;   // indexed by slot - s0
+        L.node = node + L.s0;
+    }
+    // ---- score (the parents' kept list is the whole window: k0 = 0)
+    if (tid < 8 * G) {
+        wm[tid] = -INFINITY;
+        wc[tid] = 0u;
+    }
+    gsync();
+    if (L.n > 0) score_chunks<HD, R, G>(a, L, L.s0, L.s0 + L.n, 0, pid, pmk, smem, wm, wc);
+    if (mode == LV_SPLIT) {
+        if (!ts.sync()) return false;
+        // every slot's scores (written before the barrier) and node
+        if constexpr (G == 4) {
+            const float4 *s4 = reinterpret_cast<const float4 *>(gsc);
+            float4 *d4 = reinterpret_cast<float4 *>(sc);
+#pragma unroll 8
+            for (int64_t i = tid; i < S; i += GT) d4[i] = __ldcg(s4 + i);
+        } else {
+#pragma unroll 8
+            for (int64_t i = tid; i < S * G; i += GT) sc[i] = __ldcg(gsc + i);
+        }
+#pragma unroll 4
+        for (int64_t i = tid; i < S; i += GT) node[i] = slot_node(a, l, top, pid, i);
+        gsync();
+    }
+    // ---- maxima and frontier counts of every head over the whole frontier
+    {
+        // GT is a multiple of G: every entry this thread visits is head tid % G
+        float m = -INFINITY;
+        uint32_t cnt = 0u;
+#pragma unroll 4
+        for (int64_t i = tid; i < S * G; i += GT) {
+            const float e = sc[i];
+            m = fmaxf(m, e);
+            cnt += e != -INFINITY;
+        }
+#pragma unroll
+        for (int off = G; off < 32; off <<= 1) {
+            m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+            cnt += __shfl_xor_sync(FULL, cnt, off);
+        }
+        if (lane < G) {
+            wm[warp * G + lane] = m;
+            wc[warp * G + lane] = cnt;
+        }
+        gsync();
+        if (tid < G) {
+            float mm = -INFINITY;
+            uint32_t cc = 0u;
+#pragma unroll 1
+            for (int w = 0; w < GT / 32; ++w) {
+                mm = fmaxf(mm, wm[w * G + tid]);
+                cc += wc[w * G + tid];
+            }
+            HeadCut &H = cut[tid];
+            H.M = mm;
+            H.F = cc;
+            H.rounds = 0;
+            H.nfin = 0u;
+            H.mode = cc == 0u ? CUT_NONE : (!(a.p < 1.f) ? CUT_ALL : CUT_OPEN);
+        }
+        gsync();
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) F[h] = cut[h].F;
+    // ---- the cut of the whole frontier, by this CTA alone
+    Level LA = L;
+    LA.s0 = 0;
+    LA.n = S;
+    LA.sc = sc;
+    LA.node = node;
+    if (!(a.p < 1.f)) {
+#pragma unroll 1
+        for (int64_t i = tid; i < S; i += GT) {
+            uint32_t kb = 0u;
+#pragma unroll
+            for (int h = 0; h < G; ++h) kb |= (sc[i * G + h] != -INFINITY ? 1u : 0u) << h;
+            keep[i] = (uint8_t)kb;
+        }
+        gsync();
+    } else if (S <= RANK_MAX) {
+        solo_cut<G>(LA, cut, reinterpret_cast<unsigned long long *>(smem + SM::off_hm), a.p);
+    } else if (S <= SOLO_MAX) {
+        sort_cut<G>(LA, cut, a.p);
+    } else {
+        TeamSync solo = ts;
+        solo.T = 1;
+        hist_cut<G>(a, LA, smem, solo);  // no inter-CTA barrier with a team of one
+        gsync();
+    }
+    // ---- compaction: the kept list, ascending, into pid / pmk (the node ids
+    // of every slot are in node[], so the old list is no longer needed)
+    const int64_t per = (S + GT - 1) / GT;
+    const int64_t i0 = min(S, per * tid), i1 = min(S, i0 + per);
+    uint32_t mine = 0u;
+    uint32_t hc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) hc[h] = 0u;
+#pragma unroll 4
+    for (int64_t i = i0; i < i1; ++i) {
+        const uint32_t k = keep[i];
+        mine += k != 0u;
+#pragma unroll
+        for (int h = 0; h < G; ++h) hc[h] += (k >> h) & 1u;
+    }
+    uint32_t tot;
+    uint32_t at = g_scan_u32(mine, red32, &tot) - mine;
+#pragma unroll 4
+    for (int64_t i = i0; i < i1; ++i) {
+        const uint32_t k = keep[i];
+        if (k) {
+            pid[at] = node[i];
+            pmk[at] = (uint8_t)k;
+            ++at;
+        }
+    }
+    uint32_t *hs = red32 + 16;
+    if (tid < G) hs[tid] = 0u;
+    gsync();
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        uint32_t x = hc[h];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+        if (lane == 0 && x) atomicAdd(&hs[h], x);
+    }
+    gsync();
+    nk = tot;
+    if (tr == 0) {
+        // the level's single segment: team size 1, all tot kept nodes
+        const int64_t dst = (int64_t)kh * a.slot_cap[l - 1];
+        int32_t *ids = a.kept_ids[l - 1] + dst;
+        uint8_t *msk = a.kept_mask[l - 1] + dst;
+#pragma unroll 4
+        for (uint32_t i = tid; i < tot; i += GT) {
+            ids[i] = pid[i];
+            msk[i] = pmk[i];
+        }
+        if (tid == 0) {
+            seg_ptr(a, l, kh)[0] = tot;
+            int32_t *lv = lvl_ptr(a, l, kh);
+            lv[0] = 1;
+            lv[1] = (int32_t)S;
+        }
+        if (tid < G) hseg_ptr(a, l, kh)[tid] = hs[tid];
+    }
+    gsync();
     return true;
 }
 
