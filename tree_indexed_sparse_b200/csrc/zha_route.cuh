@@ -519,6 +519,48 @@ __device__ __forceinline__ int round_bucket(const HeadCut &H, float e, int r) {
     return f < (float)(NB - 1) ? (int)f : NB - 1;
 }
 
+// A head's cut state in registers: the passes over every slot (histogram,
+// classification) read these fields for every score, and shared-memory
+// loads of them would sit on each score's dependency chain.
+struct PathReg {
+    float M;
+    int p0, p1, p2, rounds, mode;
+    PathReg() = default;
+    __device__ __forceinline__ explicit PathReg(const HeadCut &H)
+        : M(H.M), p0(H.path[0]), p1(H.path[1]), p2(H.path[2]), rounds(H.rounds), mode(H.mode) {}
+    // round_bucket of score e in round r (the same arithmetic)
+    __device__ __forceinline__ int bucket(float e, int r) const {
+        const float x = M - e;
+        float f;
+        if (r == 0) {
+            f = x * 32.f;
+        } else if (r == 1) {
+            f = x * 32768.f - 1024.f * (float)p0;
+        } else {
+            f = x * 33554432.f - 1024.f * (1024.f * (float)p0 + (float)p1);
+        }
+        if (!(f >= 0.f)) return 0;
+        return f < (float)(NB - 1) ? (int)f : NB - 1;
+    }
+    // path_cmp over the first n rounds (n <= HIST_ROUNDS)
+    __device__ __forceinline__ int cmp(float e, int n) const {
+        static_assert(HIST_ROUNDS == 3, "three rounds");
+        if (n > 0) {
+            const int b = bucket(e, 0);
+            if (b != p0) return b < p0 ? -1 : 1;
+        }
+        if (n > 1) {
+            const int b = bucket(e, 1);
+            if (b != p1) return b < p1 ? -1 : 1;
+        }
+        if (n > 2) {
+            const int b = bucket(e, 2);
+            if (b != p2) return b < p2 ? -1 : 1;
+        }
+        return 0;
+    }
+};
+
 // -1: above the fixed path (kept), 1: below (dropped), 0: on it.
 __device__ __forceinline__ int path_cmp(const HeadCut &H, float e, int rounds) {
 #pragma unroll 1
@@ -681,16 +723,18 @@ __device__ __noinline__ void sort_cut(const Level &L, const HeadCut *cut, float 
 // head, into hc/hm (shared; cleared here).
 template <int G>
 __device__ __noinline__ void local_hist(const Level &L, const HeadCut *cut, int r, uint32_t *hc,
-                                        unsigned long long *hm) {
+                                        unsigned long long *hm, bool clear = true) {
+    if (clear) {
 #pragma unroll 1
-    for (int i = threadIdx.x; i < G * NB; i += GT) {
-        hc[i] = 0u;
-        hm[i] = 0ull;
+        for (int i = threadIdx.x; i < G * NB; i += GT) {
+            hc[i] = 0u;
+            hm[i] = 0ull;
+        }
+        gsync();
     }
-    gsync();
     // GT is a multiple of G: every entry this thread visits belongs to head tid % G
     const int h = (int)(threadIdx.x % G);
-    const HeadCut &H = cut[h];
+    const PathReg H(cut[h]);
     if (H.mode == CUT_OPEN && H.rounds == r) {
         const int64_t total = L.n * G;
 #pragma unroll 1
@@ -700,8 +744,8 @@ __device__ __noinline__ void local_hist(const Level &L, const HeadCut *cut, int 
             for (int u = 0; u < 4; ++u) e[u] = i0 + u * GT < total ? L.sc[i0 + u * GT] : -INFINITY;
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                if (e[u] == -INFINITY || path_cmp(H, e[u], r) != 0) continue;
-                const int b = round_bucket(H, e[u], r);
+                if (e[u] == -INFINITY || H.cmp(e[u], r) != 0) continue;
+                const int b = H.bucket(e[u], r);
                 atomicAdd(&hc[h * NB + b], 1u);
                 atomicAdd(&hm[h * NB + b], mass_fx(expf(e[u] - H.M)));
             }
@@ -788,9 +832,14 @@ __device__ __noinline__ void find_cut(HeadCut *cut, int r, const uint32_t *cnt, 
 // and sums boundary masses (CUT_ORDER) into osum[h] (shared).
 template <int G>
 __device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsigned long long *lw, uint32_t *ls,
-                                      uint32_t *lcnt, uint32_t *own, uint32_t *own_cnt, unsigned long long *osum) {
+                                      uint32_t *lcnt, uint32_t *own, uint32_t *own_cnt, unsigned long long *osum,
+                                      int64_t ibase = 0) {
     const int lane = threadIdx.x & 31;
     const int64_t iters = (L.n + GT - 1) / GT;
+    // every head's cut state in registers (see PathReg)
+    PathReg Hr[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) Hr[h] = PathReg(cut[h]);
 #pragma unroll 1
     for (int64_t it = 0; it < iters; ++it) {
         const int64_t i = it * GT + threadIdx.x;
@@ -800,7 +849,7 @@ __device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsign
         for (int h = 0; h < G; ++h) ev[h] = i < L.n ? L.sc[i * G + h] : -INFINITY;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-            const HeadCut &H = cut[h];
+            const PathReg &H = Hr[h];
             const float e = ev[h];
             bool cand = false;
             unsigned long long w = 0ull;
@@ -808,7 +857,7 @@ __device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsign
                 if (H.mode == CUT_ALL) {
                     kbits |= 1u << h;
                 } else if (H.mode == CUT_RANK || H.mode == CUT_ORDER) {
-                    const int pc = path_cmp(H, e, H.rounds);
+                    const int pc = H.cmp(e, H.rounds);
                     if (pc < 0) kbits |= 1u << h;
                     else if (pc == 0) {
                         w = mass_fx(expf(e - H.M));
@@ -834,7 +883,8 @@ __device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsign
                         lw[h * CAND_MAX + at] = w;
                         ls[h * CAND_MAX + at] = (uint32_t)(L.s0 + i);
                     }
-                    if (obase + rank < (uint32_t)(G * CAND_MAX)) own[obase + rank] = ((uint32_t)i << 3) | (uint32_t)h;
+                    if (obase + rank < (uint32_t)(G * CAND_MAX))
+                        own[obase + rank] = ((uint32_t)(ibase + i) << 3) | (uint32_t)h;
                 }
             }
         }
@@ -963,6 +1013,138 @@ __device__ __noinline__ void write_segment(const Decode &a, const Level &L, uint
     if (threadIdx.x < G) hseg_ptr(a, L.l, L.kh)[(int64_t)L.tr * G + threadIdx.x] = hs[threadIdx.x];
 }
 
+// ---- levels whose slots spill to global memory --------------------------------
+
+// Copy local slots [c0, c0 + n) (n <= LOC_CAP) of a spilled level's scores
+// into the shared score array: every thread's loads are issued together, so
+// a chunk costs one round trip to L2 instead of one per few slots.
+template <int G>
+__device__ __forceinline__ void chunk_scores_in(const Level &L, int64_t c0, int64_t n, float *ssc) {
+    if constexpr (G == 4) {
+        const float4 *src = reinterpret_cast<const float4 *>(L.sc + c0 * G);
+        float4 *dst = reinterpret_cast<float4 *>(ssc);
+        constexpr int PER = LOC_CAP / GT;
+        float4 v[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int64_t i = threadIdx.x + (int64_t)k * GT;
+            if (i < n) v[k] = __ldcg(src + i);
+        }
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int64_t i = threadIdx.x + (int64_t)k * GT;
+            if (i < n) dst[i] = v[k];
+        }
+    } else {
+        constexpr int PER = LOC_CAP * G / GT;
+        float v[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int64_t i = threadIdx.x + (int64_t)k * GT;
+            if (i < n * G) v[k] = __ldcg(L.sc + c0 * G + i);
+        }
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int64_t i = threadIdx.x + (int64_t)k * GT;
+            if (i < n * G) ssc[i] = v[k];
+        }
+    }
+}
+
+// The local slots [c0, c0 + n) of a spilled level as a level of their own
+// whose scores are the shared copy `ssc` (keep bits stay in global memory).
+__device__ __forceinline__ Level chunk_level(const Level &L, int64_t c0, int64_t n, float *ssc) {
+    Level C = L;
+    C.s0 = L.s0 + c0;
+    C.n = n;
+    C.sc = ssc;
+    C.node = L.node + c0;
+    C.keep = L.keep + c0;
+    return C;
+}
+
+// write_segment for a spilled level: the keep bits and node ids come in by
+// chunks of LOC_CAP slots into the shared arrays, each chunk compacted in
+// slot order after the chunks before it.
+template <int G>
+__device__ __noinline__ void write_segment_spilled(const Decode &a, const Level &L, int32_t *snode, uint8_t *skeep,
+                                                   uint32_t *red32) {
+    const int64_t dst = (int64_t)L.kh * a.slot_cap[L.l - 1] + L.s0;
+    int32_t *ids = a.kept_ids[L.l - 1] + dst;
+    uint8_t *msk = a.kept_mask[L.l - 1] + dst;
+    uint32_t hc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) hc[h] = 0u;
+    uint32_t base = 0u;
+    constexpr int PER = LOC_CAP / GT;
+#pragma unroll 1
+    for (int64_t c0 = 0; c0 < L.n; c0 += LOC_CAP) {
+        const int64_t n = min((int64_t)LOC_CAP, L.n - c0);
+        {
+            uint32_t kv[PER];
+            int32_t nv[PER];
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                const int64_t i = threadIdx.x + (int64_t)k * GT;
+                kv[k] = i < n ? (uint32_t)__ldcg(L.keep + c0 + i) : 0u;
+                nv[k] = i < n ? __ldcg(L.node + c0 + i) : -1;
+            }
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                const int64_t i = threadIdx.x + (int64_t)k * GT;
+                if (i < n) {
+                    skeep[i] = (uint8_t)kv[k];
+                    snode[i] = nv[k];
+                }
+            }
+        }
+        gsync();
+        const int64_t per = (n + GT - 1) / GT;
+        const int64_t i0 = min(n, per * threadIdx.x), i1 = min(n, i0 + per);
+        uint32_t mine = 0u;
+#pragma unroll 4
+        for (int64_t i = i0; i < i1; ++i) {
+            const uint32_t k = skeep[i];
+            mine += k != 0u;
+#pragma unroll
+            for (int h = 0; h < G; ++h) hc[h] += (k >> h) & 1u;
+        }
+        uint32_t tot;
+        uint32_t at = base + g_scan_u32(mine, red32, &tot) - mine;
+#pragma unroll 4
+        for (int64_t i = i0; i < i1; ++i) {
+            const uint32_t k = skeep[i];
+            if (k) {
+                ids[at] = snode[i];
+                msk[at] = (uint8_t)k;
+                ++at;
+            }
+        }
+        base += tot;
+        gsync();
+    }
+    uint32_t *hs = red32 + 16;
+    if (threadIdx.x < G) hs[threadIdx.x] = 0u;
+    gsync();
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        uint32_t x = hc[h];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+        if ((threadIdx.x & 31) == 0 && x) atomicAdd(&hs[h], x);
+    }
+    gsync();
+    if (threadIdx.x == 0) {
+        seg_ptr(a, L.l, L.kh)[L.tr] = base;
+        if (L.tr == 0) {
+            int32_t *lv = lvl_ptr(a, L.l, L.kh);
+            lv[0] = L.T;
+            lv[1] = (int32_t)L.S;
+        }
+    }
+    if (threadIdx.x < G) hseg_ptr(a, L.l, L.kh)[(int64_t)L.tr * G + threadIdx.x] = hs[threadIdx.x];
+}
+
 // ---- one level ------------------------------------------------------------------
 
 // The histogram path of the cut (team, or one CTA with more than SOLO_MAX
@@ -988,7 +1170,19 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
 #pragma unroll 1
         for (int h = 0; h < G; ++h) open |= cut[h].mode == CUT_OPEN;
         if (!open) break;
-        local_hist<G>(L, cut, r, hc, hm);
+        if (L.n <= LOC_CAP) {
+            local_hist<G>(L, cut, r, hc, hm);
+        } else {
+            // spilled slots: by chunks through the shared score array
+            float *ssc = reinterpret_cast<float *>(smem + SM::off_sc);
+#pragma unroll 1
+            for (int64_t c0 = 0; c0 < L.n; c0 += LOC_CAP) {
+                const int64_t n = min((int64_t)LOC_CAP, L.n - c0);
+                chunk_scores_in<G>(L, c0, n, ssc);
+                gsync();
+                local_hist<G>(chunk_level(L, c0, n, ssc), cut, r, hc, hm, c0 == 0);
+            }
+        }
         rounds_used = r + 1;
         if (team) {
             uint32_t *gc = a.hist_cnt + hbase + (int64_t)r * G * NB;
@@ -1016,7 +1210,18 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
     gsync();
     // candidates go to shared lists first (shared counters); a team then
     // reserves room in its global lists with one atomic per head
-    classify<G>(L, cut, cw, cs, misc + 4, own, misc, osum);
+    if (L.n <= LOC_CAP) {
+        classify<G>(L, cut, cw, cs, misc + 4, own, misc, osum);
+    } else {
+        float *ssc = reinterpret_cast<float *>(smem + SM::off_sc);
+#pragma unroll 1
+        for (int64_t c0 = 0; c0 < L.n; c0 += LOC_CAP) {
+            const int64_t n = min((int64_t)LOC_CAP, L.n - c0);
+            chunk_scores_in<G>(L, c0, n, ssc);
+            gsync();
+            classify<G>(chunk_level(L, c0, n, ssc), cut, cw, cs, misc + 4, own, misc, osum, c0);
+        }
+    }
     unsigned long long *lw = team ? a.cand_w + (int64_t)kh * G * CAND_MAX : cw;
     uint32_t *ls = team ? a.cand_slot + (int64_t)kh * G * CAND_MAX : cs;
     if (team) {
@@ -1234,7 +1439,11 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
     } else {
         if (!hist_cut<G>(a, L, smem, ts)) return false;
     }
-    write_segment<G>(a, L, reinterpret_cast<uint32_t *>(smem + SM::off_red));
+    if (L.n <= LOC_CAP)
+        write_segment<G>(a, L, reinterpret_cast<uint32_t *>(smem + SM::off_red));
+    else
+        write_segment_spilled<G>(a, L, reinterpret_cast<int32_t *>(smem + SM::off_node), smem + SM::off_keep,
+                                 reinterpret_cast<uint32_t *>(smem + SM::off_red));
     if (team) {
         if (!ts.sync()) return false;  // D
         // the boundary lists are consumed: rank 0 clears the counters
