@@ -78,6 +78,10 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.orc_estimate_many.restype = None
     lib.orc_node_summary.argtypes = [_P, _I32, _I64, _I32, _P, _I32, _I32, _I32, _I64, _P, _P, _P]
     lib.orc_node_summary.restype = None
+    lib.orc_depth_for.argtypes = [_I64, _I32, _I32, _I32]
+    lib.orc_depth_for.restype = _I32
+    lib.orc_build_level.argtypes = [_P, _I32, _I64, _I32, _P, _I32, _I32, _I32, _P, _P, _P, _P]
+    lib.orc_build_level.restype = None
     lib.orc_set_threads.argtypes = [_I32]
     lib.orc_set_threads.restype = None
     return lib
@@ -210,10 +214,19 @@ def node_summary(K, n_tokens: int, ref, c: int, level: int, n: int, lib=None):
     return m, g, b
 
 
+def depth_for(n_tokens: int, c: int, D0: int, max_depth: int = 0, lib=None) -> int:
+    """Depth of a tree that grows with the context: the smallest depth in
+    [D0, max_depth] whose top level holds at most c nodes (max_depth <= D0:
+    the depth stays D0)."""
+    return int((lib or load()).orc_depth_for(int(n_tokens), int(c), int(D0), int(max_depth)))
+
+
 @dataclass
 class Tree:
     """Summary store of one head.  Node (level l, id n) is row
-    ``level_off[l-1] + n`` of m[rows, R], g[rows, R, d], b[rows, R]."""
+    ``level_off[l-1] + n`` of m[rows, R], g[rows, R, d], b[rows, R].  D is
+    the current depth; with max_depth > D0 the store has room for
+    max_depth levels and D grows as tokens are appended."""
 
     m: np.ndarray
     g: np.ndarray
@@ -222,6 +235,8 @@ class Tree:
     n_tokens: int
     c: int
     D: int
+    D0: int = 0
+    max_depth: int = 0
 
     def estimates(self, l: int, ids, ref, q, lib=None) -> np.ndarray:
         """Estimates for query q of the listed node ids of level l."""
@@ -242,15 +257,22 @@ def _alloc_tree(capacity: int, R: int, d: int, c: int, D: int) -> Tree:
     return Tree(np.zeros((rows, R)), np.zeros((rows, R, d)), np.zeros((rows, R)), off, 0, c, D)
 
 
-def build(K, n_tokens: int, ref, c: int, D: int, capacity: int | None = None, lib=None) -> Tree:
-    """Tree of one head over its first n_tokens keys K[>=n_tokens, d]."""
+def build(K, n_tokens: int, ref, c: int, D: int, capacity: int | None = None, max_depth: int = 0,
+          lib=None) -> Tree:
+    """Tree of one head over its first n_tokens keys K[>=n_tokens, d].  D is
+    the depth, or with max_depth > D the least depth: the tree then starts
+    at depth_for(n_tokens, c, D, max_depth) and has room to grow to
+    max_depth levels."""
     lib = lib or load()
     Ka, dt = kv_array(K)
     ref = f64(ref)
     R, d = ref.shape
-    t = _alloc_tree(max(capacity or n_tokens, n_tokens), R, d, c, D)
+    Dm = max(D, max_depth)
+    t = _alloc_tree(max(capacity or n_tokens, n_tokens), R, d, c, Dm)
+    t.D = depth_for(n_tokens, c, D, max_depth, lib=lib)
+    t.D0, t.max_depth = D, max_depth
     t.n_tokens = n_tokens
-    lib.orc_build(_ptr(Ka), dt, n_tokens, d, _ptr(ref), R, c, D, _ptr(t.m), _ptr(t.g), _ptr(t.b),
+    lib.orc_build(_ptr(Ka), dt, n_tokens, d, _ptr(ref), R, c, t.D, _ptr(t.m), _ptr(t.g), _ptr(t.b),
                   _ptr(t.level_off))
     return t
 
@@ -258,7 +280,9 @@ def build(K, n_tokens: int, ref, c: int, D: int, capacity: int | None = None, li
 def append_update(tree: Tree, K, ref, lib=None) -> None:
     """Tree maintenance after the caller stored one new key at row
     tree.n_tokens of K: the count grows by one and the new token's leaf and
-    all its ancestors are recomputed."""
+    all its ancestors are recomputed.  When the top level then holds more
+    than c nodes and the tree may still grow, a new top level is built over
+    it (every node of the new level, from its children)."""
     lib = lib or load()
     Ka, dt = kv_array(K)
     ref = f64(ref)
@@ -266,6 +290,11 @@ def append_update(tree: Tree, K, ref, lib=None) -> None:
     tree.n_tokens += 1
     lib.orc_append_update(_ptr(Ka), dt, tree.n_tokens, d, _ptr(ref), R, tree.c, tree.D,
                           _ptr(tree.m), _ptr(tree.g), _ptr(tree.b), _ptr(tree.level_off))
+    D_new = depth_for(tree.n_tokens, tree.c, tree.D0 or tree.D, tree.max_depth, lib=lib)
+    while tree.D < D_new:
+        tree.D += 1
+        lib.orc_build_level(_ptr(Ka), dt, tree.n_tokens, d, _ptr(ref), R, tree.c, tree.D, _ptr(tree.m),
+                            _ptr(tree.g), _ptr(tree.b), _ptr(tree.level_off))
 
 
 def topp(est, ids, p: float, lib=None):

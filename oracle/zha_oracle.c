@@ -241,6 +241,34 @@ void orc_build(const void *K, int dtype, int64_t N, int d, const double *ref, in
 }
 
 /*
+ * Depth of a tree whose depth grows with the context ([ZH-RU] section
+ * "Дерево сокращает сам поиск нужных ключей", last paragraph: levels are
+ * added as the context grows; the reading taken: a level is added on top
+ * whenever the top level would hold more than c nodes): the smallest depth
+ * D in [D0, Dmax] whose top level holds at most c nodes for N tokens, or
+ * Dmax when none does.  Dmax <= D0 keeps the depth fixed at D0.
+ */
+int orc_depth_for(int64_t N, int c, int D0, int Dmax)
+{
+    if (Dmax <= D0)
+        return D0;
+    for (int D = D0; D < Dmax; ++D)
+        if (orc_level_nodes(N, c, D) <= c)
+            return D;
+    return Dmax;
+}
+
+/* Every node of one level, from the raw keys (level 1) or from the level
+ * below (the parent summary of each node's children). */
+void orc_build_level(const void *K, int dtype, int64_t N, int d, const double *ref, int R, int c, int level,
+                     double *m, double *g, double *b, const int64_t *level_off)
+{
+    const int64_t nl = orc_level_nodes(N, c, level);
+    for (int64_t n = 0; n < nl; ++n)
+        node_recompute(K, dtype, N, d, ref, R, c, level, n, m, g, b, level_off);
+}
+
+/*
  * Tree maintenance for one appended token.  The caller has stored the new
  * key as row N-1 (N already counts it).  The leaf holding it is recomputed
  * from its tokens, then each ancestor from its children; a node that did not

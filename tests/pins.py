@@ -454,8 +454,48 @@ def pin_heads_drivers(lib):
                 assert np.max(np.abs(out[h] - w @ V[kh, :N].astype(np.float64))) <= 1e-12, h
 
 
+def pin_depth_growth(lib):
+    """A tree whose depth grows with the context: the depth is the least one
+    (from the given minimum) whose top level holds at most c nodes -- chunk
+    4 and 6 levels cover 4,096 tokens per top node, so 16,384 tokens fit
+    depth 6 and one more token needs depth 7 -- and appending tokens across
+    a growth step gives exactly the tree built over all of them, whose new
+    top level holds the log mass of its whole subtree (closed form)."""
+    assert oracle.depth_for(16384, 4, 6, 8, lib=lib) == 6
+    assert oracle.depth_for(16385, 4, 6, 8, lib=lib) == 7
+    assert oracle.depth_for(16385, 4, 6, 0, lib=lib) == 6      # no growth without room
+    assert oracle.depth_for(4 ** 9, 4, 6, 8, lib=lib) == 8      # capped at the maximum
+    rng = _rng(1700)
+    # the first case grows at its last append (nothing after it rebuilds the new level)
+    for (N, a, c, D0, Dm, R, d) in [(16, 1, 4, 1, 3, 2, 4), (16, 3, 4, 1, 3, 2, 4), (60, 8, 2, 2, 6, 1, 4),
+                                    (250, 10, 4, 2, 4, 3, 6)]:
+        K = rng.standard_normal((N + a, d)).astype(np.float32)
+        ref = rng.standard_normal((R, d))
+        t_inc = oracle.build(K, N, ref, c, D0, capacity=N + a, max_depth=Dm, lib=lib)
+        D_start = t_inc.D
+        for _ in range(a):
+            oracle.append_update(t_inc, K, ref, lib=lib)
+        t_full = oracle.build(K, N + a, ref, c, D0, max_depth=Dm, lib=lib)
+        assert t_inc.D == t_full.D > D_start, (N, a, D_start, t_inc.D, t_full.D)
+        K64 = K.astype(np.float64)
+        for level in range(1, t_full.D + 1):
+            mi, gi, bi = t_inc.level(level)
+            mf, gf, bf = t_full.level(level)
+            assert mi.shape == mf.shape
+            assert np.max(np.abs(mi - mf)) <= 1e-12 and np.max(np.abs(gi - gf)) <= 1e-12, (N, level)
+        mt, gt, bt = t_inc.level(t_inc.D)
+        for n in range(mt.shape[0]):
+            t0, t1 = _subtree(N + a, c, t_inc.D, n)
+            for j in range(R):
+                m_ref = logsumexp(K64[t0:t1] @ ref[j] / math.sqrt(d))
+                assert abs(mt[n, j] - m_ref) <= 1e-10 * max(1.0, abs(m_ref)), (N, n, j)
+        # routing over a grown tree starts at its new top level
+        kept, visited = oracle.route(t_inc, ref, rng.standard_normal(d), 1.0, lib=lib)
+        assert visited == sum(-(-(N + a) // c ** l) for l in range(1, t_inc.D + 1))
+
+
 ALL_PINS = [pin_closed_form_subtree, pin_lower_bound_and_tangent, pin_single_plane_affine,
             pin_exact_leaves_token_topp, pin_dense_at_p1, pin_flat_chunk_topp, pin_routing_invariants,
             pin_ties_lower_id, pin_topp_brute_force, pin_attention_and_sink, pin_bf16_widening,
             pin_append_equivalence, pin_golden_geometry, pin_node_summary_subtree, pin_estimate_many_rows,
-            pin_heads_drivers]
+            pin_heads_drivers, pin_depth_growth]

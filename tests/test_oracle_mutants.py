@@ -53,6 +53,9 @@ MUTANTS = {
     "decode_heads_value_stride": ("const char *Vh = (const char *)V + (size_t)kh * kv_stride * d * esize;",
                                   "const char *Vh = (const char *)V + (size_t)kh * d * esize;"),
     "build_heads_offset_stride": ("b + kh * m_stride, level_off);", "b, level_off);"),
+    "growth_when_top_level_is_full": ("if (orc_level_nodes(N, c, D) <= c)", "if (orc_level_nodes(N, c, D) < c)"),
+    "grown_level_skips_last_node": ("    for (int64_t n = 0; n < nl; ++n)\n        node_recompute(",
+                                    "    for (int64_t n = 0; n + 1 < nl; ++n)\n        node_recompute("),
 }
 
 
