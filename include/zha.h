@@ -69,14 +69,22 @@ extern "C" {
  *   R                reference queries per KV head (compiled: 1, 16)
  *   c                chunk size = children per node (>= 2)
  *   D                depth: routing levels; a top node covers c^D tokens
- *                    (1 <= D <= 16)
+ *                    (1 <= D <= 16); with max_depth > D, the least depth
  *   kv_dtype         ZHA_F32 or ZHA_BF16
+ *   max_depth        0: the depth stays D.  D < max_depth <= 16: the depth
+ *                    grows with the context (rit.work "ZHA tree indexer",
+ *                    section "Дерево сокращает сам поиск нужных ключей",
+ *                    last paragraph): it is always the least depth >= D
+ *                    whose top level holds at most c nodes (at most
+ *                    max_depth), so zha_build starts there and an append
+ *                    that leaves c + 1 top nodes adds a new top level over
+ *                    them; zha_depth gives the current depth
  *   capacity_tokens  rows per KV head in K and V (room for appends)
  */
 typedef struct {
     int32_t h_kv, h_q, d, R, c, D;
     int32_t kv_dtype;
-    int32_t reserved;
+    int32_t max_depth;
     int64_t capacity_tokens;
 } zha_config;
 
@@ -131,8 +139,10 @@ int zha_build(zha_ctx *ctx, void *d_K, void *d_V, int64_t n_tokens, const float 
  *   d_k, d_v   [h_kv][d] kv_dtype: the new row of each KV head
  * Writes row n_tokens of the built K and V, recomputes the leaf holding it and
  * every ancestor (creating a node, or a new top node, at a boundary), then
- * n_tokens += 1.  Returns ZHA_ERR_CAPACITY when the cache is full and
- * ZHA_ERR_NOT_BUILT before zha_build.
+ * n_tokens += 1.  With a growing depth (zha_config.max_depth), when the top
+ * level then holds c + 1 nodes a new top level is built over it (a second
+ * launch on `stream`) and the depth grows by one.  Returns ZHA_ERR_CAPACITY
+ * when the cache is full and ZHA_ERR_NOT_BUILT before zha_build.
  */
 int zha_append(zha_ctx *ctx, const void *d_k, const void *d_v, void *stream);
 
@@ -149,8 +159,9 @@ int zha_append(zha_ctx *ctx, const void *d_k, const void *d_v, void *stream);
  *                    attended but not listed)
  *   d_n_leaf         [h_q] int32: number of kept leaf chunks per head
  *   d_nodes_visited  [h_q] int64: nodes scored over all levels per head
- *   d_trace_ids      nullable; [D][h_q][trace_cap] int32: ascending kept
- *                    node ids of level l (1-based) at ((l-1)*h_q+i)*trace_cap
+ *   d_trace_ids      nullable; [D][h_q][trace_cap] int32, D the current
+ *                    depth (zha_depth): ascending kept node ids of level l
+ *                    (1-based) at ((l-1)*h_q+i)*trace_cap
  *   d_trace_counts   nullable together with d_trace_ids; [D][h_q] int32
  * Routing per query head, level D down to 1: the frontier is every top node,
  * then the children of the nodes kept one level up; estimates are
@@ -243,11 +254,15 @@ int zha_set_phase_timer(zha_ctx *ctx, int64_t *d_ns);
  */
 int zha_set_wait_budget(zha_ctx *ctx, int64_t cycles);
 
+/* Current depth of the tree (routing levels; 0 before zha_build).  Equals
+ * the configuration's D unless its max_depth lets the tree grow. */
+int32_t zha_depth(const zha_ctx *ctx);
+
 /* Tokens currently in the cache (host-side count; 0 before zha_build). */
 int64_t zha_n_tokens(const zha_ctx *ctx);
 
 /*
- * Where level `level` (1..D) of the summary store lives inside the workspace,
+ * Where level `level` (1..max(D, max_depth)) of the summary store lives inside the workspace,
  * for inspection: byte offsets of g [h_kv][node_cap][R][d] fp32, b
  * [h_kv][node_cap][R] fp32 and m [h_kv][node_cap][R] fp32, and node_cap (the
  * node rows per KV head).  Returns ZHA_ERR_BAD_ARG for an invalid level.

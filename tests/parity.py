@@ -69,7 +69,7 @@ def check_build(cache, trees, rtol: float = BUILD_RTOL, levels=None, sample=None
     worst = [0.0, 0.0, 0.0]
     rng = np.random.default_rng(seed)
     heads = list(range(cfg.h_kv)) if heads is None else list(heads)
-    for level in (levels or (sorted(ids) if ids is not None else range(1, cfg.D + 1))):
+    for level in (levels or (sorted(ids) if ids is not None else range(1, cache.depth + 1))):
         g, b, m = cache.summaries(level)
         n = m.shape[1]
         if ids is not None:

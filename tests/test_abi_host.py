@@ -48,7 +48,8 @@ def test_workspace_sizes(name):
     ("h_kv", 0, zha.ZHA_ERR_BAD_ARG), ("h_q", 6, zha.ZHA_ERR_BAD_ARG), ("c", 1, zha.ZHA_ERR_BAD_ARG),
     ("D", 0, zha.ZHA_ERR_BAD_ARG), ("D", 17, zha.ZHA_ERR_BAD_ARG), ("kv_dtype", 7, zha.ZHA_ERR_BAD_ARG),
     ("capacity_tokens", 0, zha.ZHA_ERR_BAD_ARG), ("d", 96, zha.ZHA_ERR_UNSUPPORTED),
-    ("R", 3, zha.ZHA_ERR_UNSUPPORTED),
+    ("R", 3, zha.ZHA_ERR_UNSUPPORTED), ("max_depth", 1, zha.ZHA_ERR_BAD_ARG),
+    ("max_depth", 17, zha.ZHA_ERR_BAD_ARG), ("max_depth", -1, zha.ZHA_ERR_BAD_ARG),
 ])
 def test_bad_config(field, value, code):
     cfg = _cfg(workloads.WORKLOADS["wide_256k"])

@@ -313,3 +313,79 @@ def test_injected_host_faults(monkeypatch):
     V[:, N] = 0.0
     trees = oracle_trees(K, ref, N + 1, c, D)
     check_build(cache, trees)
+
+
+@pytest.mark.parametrize("N,a,c,D,Dm,R,h_kv,h_q,d,dtype", [
+    (16384 - 2, 6, 4, 6, 8, 16, 1, 1, 64, zha.ZHA_F32),    # the tiny workload's tree grows from 6 to 7 levels
+    (510, 5, 8, 2, 4, 1, 2, 8, 128, zha.ZHA_BF16),         # chunk 8: grows from 2 to 3 levels
+])
+def test_depth_growth(N, a, c, D, Dm, R, h_kv, h_q, d, dtype):
+    """A tree whose depth grows with the context: the append that leaves c + 1
+    top nodes adds a new top level.  Before, across and after the step the
+    summaries and the routing match the oracle growing the same way, and the
+    grown tree is bit-identical to a fresh build over all the tokens."""
+    g = torch.Generator().manual_seed(N + c)
+    tdt = torch.float32 if dtype == zha.ZHA_F32 else torch.bfloat16
+    cap = N + a
+    K = torch.zeros(h_kv, cap, d, dtype=tdt)
+    V = torch.zeros(h_kv, cap, d, dtype=tdt)
+    K[:, :cap] = torch.randn(h_kv, cap, d, generator=g).to(tdt)
+    V[:, :cap] = torch.randn(h_kv, cap, d, generator=g).to(tdt)
+    ref = torch.randn(h_kv, R, d, generator=g)
+    if dtype == zha.ZHA_BF16:
+        ref = ref.to(torch.bfloat16).float()
+    kv = "f32" if dtype == zha.ZHA_F32 else "bf16"
+    cache = zha.ZhaCache(h_kv, h_q, d, R, c, D, dtype, cap, max_depth=Dm)
+    dK, dV, dref = K.cuda(), V.cuda(), ref.cuda()
+    dK[:, N:] = 0
+    dV[:, N:] = 0
+    cache.build(dK, dV, N, dref)
+    trees = [oracle.build(K[kh], N, ref[kh], c, D, capacity=cap, max_depth=Dm) for kh in range(h_kv)]
+    assert cache.depth == trees[0].D == oracle.depth_for(N, c, D, Dm)
+    D_start = cache.depth
+    qs = torch.randn(a + 1, h_q, d, generator=g) * 2
+    n = N
+    for i in range(a + 1):
+        if i > 0:
+            cache.append(K[:, n].cuda(), V[:, n].cuda())
+            for kh in range(h_kv):
+                oracle.append_update(trees[kh], K[kh], ref[kh])
+            n += 1
+        torch.cuda.synchronize()
+        assert cache.depth == trees[0].D, (n, cache.depth, trees[0].D)
+        check_build(cache, trees)
+        res = cache.decode(qs[i].cuda(), 0.9, trace_cap=oracle.level_nodes(cap, c, 1))
+        torch.cuda.synchronize()
+        assert cache.status() == zha.ZHA_OK
+        check_decode(res, trees, K, V, ref, qs[i].double().numpy(), 0.9, n, c, cache.depth, h_q // h_kv, kv,
+                     case=f"depth growth N={n} c={c} depth {cache.depth}")
+    assert cache.depth == D_start + 1
+    fresh = zha.ZhaCache(h_kv, h_q, d, R, c, D, dtype, cap, max_depth=Dm)
+    fK, fV = K.cuda(), V.cuda()
+    fresh.build(fK, fV, n, dref)
+    torch.cuda.synchronize()
+    assert fresh.depth == cache.depth
+    for level in range(1, cache.depth + 1):
+        for x, y in zip(cache.summaries(level), fresh.summaries(level)):
+            assert torch.equal(x, y), level
+
+
+def test_depth_growth_build_starts_deeper():
+    """With room to grow, a build starts at the least depth whose top level
+    holds at most c nodes (here 4 levels where 2 are the minimum)."""
+    N, c, D, Dm, R, h_kv, h_q, d = 5000, 8, 2, 4, 1, 2, 8, 128
+    cache, (K, V, ref), _ = _small_cache(N, c, D, R, h_kv, h_q, d, zha.ZHA_BF16, 21)
+    assert cache.depth == D  # a fixed-depth cache of the same data
+    grow = zha.ZhaCache(h_kv, h_q, d, R, c, D, zha.ZHA_BF16, N, max_depth=Dm)
+    dK, dV, dref = K.cuda(), V.cuda(), ref.cuda()
+    grow.build(dK, dV, N, dref)
+    torch.cuda.synchronize()
+    assert grow.depth == oracle.depth_for(N, c, D, Dm) == 4
+    trees = [oracle.build(K[kh], N, ref[kh], c, D, max_depth=Dm) for kh in range(h_kv)]
+    check_build(grow, trees)
+    q = torch.randn(h_q, d, generator=torch.Generator().manual_seed(3)) * 2
+    res = grow.decode(q.cuda(), 0.8, trace_cap=oracle.level_nodes(N, c, 1))
+    torch.cuda.synchronize()
+    assert grow.status() == zha.ZHA_OK
+    check_decode(res, trees, K, V, ref, q.double().numpy(), 0.8, N, c, grow.depth, h_q // h_kv, "bf16",
+                 case="depth growth build N=5000 c=8 depth 4")

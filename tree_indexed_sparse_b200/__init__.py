@@ -28,7 +28,7 @@ ZHA_BF16 = 1
 # every symbol include/zha.h declares
 EXPORTS = ["zha_workspace_bytes", "zha_create", "zha_destroy", "zha_build", "zha_append", "zha_decode",
            "zha_dense_decode", "zha_dense_decode_static", "zha_device_status", "zha_set_phase_timer",
-           "zha_set_wait_budget", "zha_n_tokens", "zha_summary_layout", "zha_strerror"]
+           "zha_set_wait_budget", "zha_depth", "zha_n_tokens", "zha_summary_layout", "zha_strerror"]
 
 
 class ZhaError(RuntimeError):
@@ -40,7 +40,7 @@ class ZhaError(RuntimeError):
 class zha_config(ctypes.Structure):
     _fields_ = [("h_kv", ctypes.c_int32), ("h_q", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("R", ctypes.c_int32), ("c", ctypes.c_int32), ("D", ctypes.c_int32),
-                ("kv_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("kv_dtype", ctypes.c_int32), ("max_depth", ctypes.c_int32),
                 ("capacity_tokens", ctypes.c_int64)]
 
 
@@ -72,6 +72,8 @@ def _load() -> ctypes.CDLL:
     lib.zha_set_phase_timer.restype = ctypes.c_int
     lib.zha_set_wait_budget.argtypes = [P, I64]
     lib.zha_set_wait_budget.restype = ctypes.c_int
+    lib.zha_depth.argtypes = [P]
+    lib.zha_depth.restype = I32
     lib.zha_n_tokens.argtypes = [P]
     lib.zha_n_tokens.restype = I64
     lib.zha_summary_layout.argtypes = [P, I32, ctypes.POINTER(I64), ctypes.POINTER(I64),
@@ -162,6 +164,10 @@ def zha_set_wait_budget(ctx, cycles: int) -> None:
     _check(lib.zha_set_wait_budget(ctx, int(cycles)), "zha_set_wait_budget")
 
 
+def zha_depth(ctx) -> int:
+    return int(lib.zha_depth(ctx))
+
+
 def zha_n_tokens(ctx) -> int:
     return int(lib.zha_n_tokens(ctx))
 
@@ -183,10 +189,10 @@ class ZhaCache:
     """
 
     def __init__(self, h_kv: int, h_q: int, d: int, R: int, c: int, D: int, kv_dtype: int,
-                 capacity_tokens: int, device="cuda"):
+                 capacity_tokens: int, device="cuda", max_depth: int = 0):
         import torch
 
-        self.cfg = zha_config(h_kv, h_q, d, R, c, D, kv_dtype, 0, capacity_tokens)
+        self.cfg = zha_config(h_kv, h_q, d, R, c, D, kv_dtype, max_depth, capacity_tokens)
         nbytes = zha_workspace_bytes(self.cfg)
         if nbytes < 0:
             raise ZhaError(nbytes, "zha_workspace_bytes")
@@ -222,12 +228,17 @@ class ZhaCache:
     def n_tokens(self) -> int:
         return zha_n_tokens(self.ctx)
 
+    @property
+    def depth(self) -> int:
+        """Current depth (routing levels) of the tree."""
+        return zha_depth(self.ctx)
+
     def decode(self, q, p: float, leaf_cap: int | None = None, trace_cap: int = 0, stream=None, out=None):
         """Returns a dict of device tensors: out, leaf_idx, n_leaf, visited
         (+ trace_ids, trace_counts when trace_cap > 0)."""
         import torch
 
-        h_q, D = self.cfg.h_q, self.cfg.D
+        h_q, D = self.cfg.h_q, self.depth
         dev = self.device
         if leaf_cap is None:
             leaf_cap = -(-self.n_tokens // self.cfg.c)

@@ -29,6 +29,7 @@ struct zha_ctx {
     int decode_cta;
     int n_sm;
     int attn_cta;
+    int D0, Dmax;             // least and greatest depth (equal unless the depth grows)
 };
 
 namespace {
@@ -53,6 +54,7 @@ int check_config(const zha_config *cfg) {
     if (cfg->d <= 0 || cfg->R <= 0 || cfg->c < 2 || cfg->D < 1 || cfg->D > MAXD) return ZHA_ERR_BAD_ARG;
     if (cfg->kv_dtype != ZHA_F32 && cfg->kv_dtype != ZHA_BF16) return ZHA_ERR_BAD_ARG;
     if (cfg->capacity_tokens < 1 || cfg->capacity_tokens > (int64_t)0x7fffffff) return ZHA_ERR_BAD_ARG;
+    if (cfg->max_depth != 0 && (cfg->max_depth <= cfg->D || cfg->max_depth > MAXD)) return ZHA_ERR_BAD_ARG;
     const int G = cfg->h_q / cfg->h_kv;
     if (!compiled_combo(cfg->kv_dtype, cfg->d, cfg->R, G)) return ZHA_ERR_UNSUPPORTED;
     return ZHA_OK;
@@ -69,11 +71,23 @@ struct Layout {
     int64_t score_cap;
 };
 
+// Levels the workspace holds: the greatest depth.
+int max_levels(const zha_config *cfg) { return cfg->max_depth > cfg->D ? cfg->max_depth : cfg->D; }
+
+// Depth over n tokens: the least depth in [D0, Dmax] whose top level holds
+// at most c nodes, or Dmax (D0 when the depth does not grow).
+int depth_for(int64_t n, int c, int D0, int Dmax) {
+    int D = D0;
+    while (D < Dmax && level_nodes(n, c, D) > c) ++D;
+    return D;
+}
+
 void make_layout(const zha_config *cfg, Layout *L) {
     const int G = cfg->h_q / cfg->h_kv;
     const int64_t H = cfg->h_kv;
+    const int DL = max_levels(cfg);
     int64_t off = 0;
-    for (int l = 1; l <= cfg->D; ++l) {
+    for (int l = 1; l <= DL; ++l) {
         const int64_t nc = level_nodes(cfg->capacity_tokens, cfg->c, l);
         L->node_cap[l - 1] = nc;
         L->g_off[l - 1] = off;
@@ -86,13 +100,13 @@ void make_layout(const zha_config *cfg, Layout *L) {
     // frontier slots of level l: every top node, or c children of each node
     // of level l + 1
     int64_t sc = 0;
-    for (int l = 1; l <= cfg->D; ++l) {
-        L->slot_cap[l - 1] = (l == cfg->D) ? L->node_cap[l - 1] : (int64_t)cfg->c * L->node_cap[l];
+    for (int l = 1; l <= DL; ++l) {
+        L->slot_cap[l - 1] = (l == DL) ? L->node_cap[l - 1] : (int64_t)cfg->c * L->node_cap[l];
         sc = std::max(sc, L->slot_cap[l - 1]);
     }
     L->score_cap = sc;
     L->scratch_off = off;
-    for (int l = 1; l <= cfg->D; ++l) {
+    for (int l = 1; l <= DL; ++l) {
         L->kid_off[l - 1] = off;
         off = align256(off + H * L->slot_cap[l - 1] * 4);
         L->kmask_off[l - 1] = off;
@@ -185,9 +199,11 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
         if ((1 << s) == cfg->c) t.c_log2 = s;
     t.kv_cap = cfg->capacity_tokens;
     t.scale = (float)(1.0 / std::sqrt((double)cfg->d));
+    ctx->D0 = cfg->D;
+    ctx->Dmax = max_levels(cfg);
     Decode &d = ctx->scratch;
     std::memset(&d, 0, sizeof d);
-    for (int l = 1; l <= cfg->D; ++l) {
+    for (int l = 1; l <= ctx->Dmax; ++l) {
         t.node_cap[l - 1] = L.node_cap[l - 1];
         t.g[l - 1] = reinterpret_cast<float *>(ws + L.g_off[l - 1]);
         t.b[l - 1] = reinterpret_cast<float *>(ws + L.b_off[l - 1]);
@@ -265,6 +281,7 @@ int zha_build(zha_ctx *ctx, void *d_K, void *d_V, int64_t n_tokens, const float 
     t.V = d_V;
     t.ref = d_ref_q;
     t.n_tokens = n_tokens;
+    t.D = depth_for(n_tokens, t.c, ctx->D0, ctx->Dmax);
     fill_tree_levels(ctx);
     if (fault_injected("cuda_launch")) return ZHA_ERR_CUDA;
     if (launch_build(t, static_cast<cudaStream_t>(stream), ctx->n_sm) != cudaSuccess) return ZHA_ERR_CUDA;
@@ -279,7 +296,16 @@ int zha_append(zha_ctx *ctx, const void *d_k, const void *d_v, void *stream) {
     Tree t = ctx->t;
     t.n_tokens += 1;
     for (int l = 1; l <= t.D; ++l) t.n_level[l - 1] = (int32_t)level_nodes(t.n_tokens, t.c, l);
-    if (launch_append(t, d_k, d_v, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZHA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (launch_append(t, d_k, d_v, s) != cudaSuccess) return ZHA_ERR_CUDA;
+    // a growing tree whose top level now holds c + 1 nodes: a new top level
+    const int D_new = depth_for(t.n_tokens, t.c, ctx->D0, ctx->Dmax);
+    if (D_new > t.D) {
+        const int D_old = t.D;
+        t.D = D_new;
+        for (int l = 1; l <= t.D; ++l) t.n_level[l - 1] = (int32_t)level_nodes(t.n_tokens, t.c, l);
+        if (launch_build_levels(t, D_old + 1, D_new, s, ctx->n_sm) != cudaSuccess) return ZHA_ERR_CUDA;
+    }
     ctx->t = t;
     return ZHA_OK;
 }
@@ -348,11 +374,13 @@ int zha_set_wait_budget(zha_ctx *ctx, int64_t cycles) {
     return ZHA_OK;
 }
 
+int32_t zha_depth(const zha_ctx *ctx) { return ctx && ctx->built ? ctx->t.D : 0; }
+
 int64_t zha_n_tokens(const zha_ctx *ctx) { return ctx && ctx->built ? ctx->t.n_tokens : 0; }
 
 int zha_summary_layout(const zha_ctx *ctx, int32_t level, int64_t *g_offset, int64_t *b_offset, int64_t *m_offset,
                        int64_t *node_cap) {
-    if (!ctx || level < 1 || level > ctx->cfg.D) return ZHA_ERR_BAD_ARG;
+    if (!ctx || level < 1 || level > ctx->Dmax) return ZHA_ERR_BAD_ARG;
     const unsigned char *ws = ctx->ws;
     if (g_offset) *g_offset = reinterpret_cast<const unsigned char *>(ctx->t.g[level - 1]) - ws;
     if (b_offset) *b_offset = reinterpret_cast<const unsigned char *>(ctx->t.b[level - 1]) - ws;

@@ -543,6 +543,25 @@ static cudaError_t build_impl(const Tree &t, cudaStream_t s, int n_sm) {
     return cudaSuccess;
 }
 
+// Parent levels [from, to] over the current tree (a tree growing a new top
+// level after an append).
+template <typename KT, int HD, int R>
+static cudaError_t build_levels_impl(const Tree &t, int from, int to, cudaStream_t s, int n_sm) {
+    const int warps = BUILD_THREADS / 32;
+    const size_t psmem = (size_t)warps * (t.c * R + R) * sizeof(float);
+    static PerDeviceMax<> parent_attr;
+    cudaError_t err = allow_smem(k_build_parents<HD, R>, psmem, parent_attr);
+    if (err != cudaSuccess) return err;
+    for (int level = from; level <= to; ++level) {
+        const int64_t work = (int64_t)t.n_level[level - 1] * t.h_kv;
+        const int pgrid = (int)std::min<int64_t>((work + warps - 1) / warps, (int64_t)n_sm * 8);
+        k_build_parents<HD, R><<<pgrid, BUILD_THREADS, psmem, s>>>(t, level);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
+    return cudaSuccess;
+}
+
 template <typename KT, int HD, int R>
 static cudaError_t append_impl(const Tree &t, const void *k, const void *v, cudaStream_t s) {
     // per plane warp: one score per token of a leaf, or one estimate per child
@@ -575,6 +594,11 @@ cudaError_t launch_build(const Tree &t, cudaStream_t s, int n_sm) { ZHA_BUILD_DI
 
 cudaError_t launch_append(const Tree &t, const void *k, const void *v, cudaStream_t s) {
     ZHA_BUILD_DISPATCH(append_impl, t, k, v, s);
+}
+
+cudaError_t launch_build_levels(const Tree &t, int from, int to, cudaStream_t s, int n_sm) {
+    if (from < 2 || to > t.D || from > to) return cudaErrorInvalidValue;
+    ZHA_BUILD_DISPATCH(build_levels_impl, t, from, to, s, n_sm);
 }
 
 }  // namespace zha

@@ -19,7 +19,7 @@ constexpr int LOC_CAP = 2048;     // frontier slots one CTA holds in shared memo
 // Summary store of every level (pointers for KV head 0; head stride is
 // node_cap[l] rows).  g: [node][R][d], b and m: [node][R].
 struct Tree {
-    int h_kv, h_q, G, d, R, c, D, kv_dtype;
+    int h_kv, h_q, G, d, R, c, D, kv_dtype;  // D: current depth
     int c_log2;                   // log2(c) when c is a power of two, else -1
     int64_t kv_cap;               // rows per KV head in K and V
     int64_t n_tokens;             // tokens present
@@ -105,6 +105,7 @@ cudaError_t allow_smem(Fn *fn, size_t bytes, PerDeviceMax<> &rec) {
 // host-side launchers; each returns a cudaError_t (0 on success)
 cudaError_t launch_build(const Tree &t, cudaStream_t s, int n_sm);
 cudaError_t launch_append(const Tree &t, const void *k, const void *v, cudaStream_t s);
+cudaError_t launch_build_levels(const Tree &t, int from, int to, cudaStream_t s, int n_sm);
 cudaError_t launch_decode(const Decode &dc, int n_cta, cudaStream_t s);
 int decode_blocks_per_sm(const Decode &dc);
 cudaError_t launch_dense(const Decode &dc, int n_cta, cudaStream_t s);
