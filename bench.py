@@ -201,16 +201,17 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def step_bytes(w, trace_ids, trace_cnt, n_tokens):
+def step_bytes(w, trace_ids, trace_cnt, n_tokens, router_bf16=False):
     """Algorithmic bytes of one decode from its per-level kept sets.
 
     Routing reads each node of the union frontier of a KV head once (g and b:
-    R*(d+1)*4 bytes), whatever the number of its query heads that need it;
+    R*(d+1)*4 bytes, or R*(2d+4) with the bf16 router copy), whatever the
+    number of its query heads that need it;
     attention reads the K and V rows of the union of the heads' token sets
     once; plus the queries and outputs."""
     c, D, d, R, G = w.c, w.D, w.d, w.R, w.group
     e = 4 if w.kv_dtype == "f32" else 2
-    node = R * (d + 1) * 4
+    node = R * (2 * d + 4) if router_bf16 else R * (d + 1) * 4
     route = 0
     attn = 0
     slots_total = 0
@@ -281,7 +282,9 @@ def run_zha(args, rank, world, local):
     torch.cuda.synchronize()
     gen_s = time.time() - t0
     dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
-    cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, device=dev)
+    router_bf16 = args.router == "bf16"
+    cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, device=dev,
+                         router_dtype=zha.ZHA_BF16 if router_bf16 else zha.ZHA_F32)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     n1cap = -(-w.capacity // w.c)
@@ -329,7 +332,7 @@ def run_zha(args, rank, world, local):
         ids = tr_ids.cpu().numpy()
         cnt = tr_cnt.cpu().numpy()
         n_now = w.n_tokens + (i + 1) * per_step
-        rb, ab, slots, slots_level = step_bytes(w, ids, cnt, n_now)
+        rb, ab, slots, slots_level = step_bytes(w, ids, cnt, n_now, router_bf16)
         app_b = sum(append_bytes(w, n_now - per_step + j + 1) for j in range(per_step))
         per_step_all.append((rb, ab, app_b, slots, n_now, slots_level))
         if i >= W:
@@ -526,6 +529,7 @@ def run_zha(args, rank, world, local):
                    "c": w.c, "D": w.D, "R": w.R, "p": w.p, "kv_dtype": w.kv_dtype, "keys": w.keys,
                    "step": step_desc,
                    "appends_after_steps": burst if base.appends_after else 0,
+                   "router": "bf16 copy of g (reduced-precision router)" if router_bf16 else "fp32",
                    "l2": "256 MiB written between steps, outside the per-step events",
                    "parallelism": f"replicas x{world}"},
         "hbm_gbs": gbs, "hbm_frac": gbs / peak,
@@ -643,6 +647,60 @@ def run_reference(args, rank, world):
             "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_growth(args, local):
+    """A tree whose depth grows with the context, measured where it grows:
+    the light workload's settings (chunk 8, depth 6, R = 1, p = 0.75,
+    mixture keys) at 2,097,152 - 4 tokens (8 top nodes of 262,144 tokens)
+    with room for a 7th level.  Device times (L2 flushed before each call):
+    decodes at depth 6, the appends up to and past 2,097,152 tokens (the
+    5th adds the new top level), decodes at depth 7."""
+    import tree_indexed_sparse_b200 as zha
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    base = workloads.WORKLOADS["light_1m"]
+    steps, n_app = 16, 8
+    N = base.c ** (base.D + 1) - 4
+    w = dataclasses.replace(base.scaled(N, steps=steps), appends_per_step=0, appends_after=n_app)
+    inp = workloads.generate(w, dev)
+    dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
+    cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, device=dev, max_depth=w.D + 1)
+    cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
+    out = torch.empty(w.h_q, w.d, dtype=torch.float32, device=dev)
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        flush.zero_()
+        torch.cuda._sleep(HOLD_CYCLES)
+        ea.record(stream)
+        fn()
+        eb.record(stream)
+        torch.cuda.synchronize()
+        return ea.elapsed_time(eb) * 1e3
+
+    depth0 = cache.depth
+    before = [timed(lambda: cache.decode(inp.Q[i % steps], w.p, out=out)) for i in range(3 + steps)][3:]
+    apps = []
+    for i in range(n_app):
+        d0 = cache.depth
+        us = timed(lambda: cache.append(inp.K_app[i], inp.V_app[i]))
+        apps.append({"n_tokens": cache.n_tokens, "depth": cache.depth, "adds_level": cache.depth > d0, "us": us})
+    after = [timed(lambda: cache.decode(inp.Q[i % steps], w.p, out=out)) for i in range(3 + steps)][3:]
+    assert cache.status() == 0
+    grow = [x["us"] for x in apps if x["adds_level"]]
+    plain = [x["us"] for x in apps if not x["adds_level"]]
+    return {"metric": "growing depth: decode before and after the tree adds a level, and the append that adds it",
+            "unit": "us", "n_gpus": 1, "steps": steps, "data": "synthetic",
+            "config": {"workload": f"light_1m settings at {N} tokens, depth {w.D} growing to {w.D + 1}",
+                       "l2": "256 MiB written before every call"},
+            "depth_before": depth0, "depth_after": cache.depth,
+            "decode_us_before": statistics.median(before), "decode_us_after": statistics.median(after),
+            "append_us_adding_level": grow[0] if grow else None,
+            "append_us_other": statistics.median(plain) if plain else None, "appends": apps}
+
+
 CROSSOVER_N = [16384, 32768, 49152, 65536, 98304, 131072, 196608, 262144, 524288, 1048576]
 
 
@@ -713,12 +771,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--crossover", action="store_true",
                     help="sweep the light workload's settings over context lengths, routed vs dense")
+    ap.add_argument("--router", choices=["f32", "bf16"], default="f32",
+                    help="summaries the routing reads: fp32 (default) or the bf16 router copy")
+    ap.add_argument("--growth", action="store_true",
+                    help="time the step where a tree with room to grow adds a level (light settings, 2M tokens)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_setup(args.gpus)
-    if args.crossover:
+    if args.crossover or args.growth:
         if rank == 0:
-            print(json.dumps(run_crossover(args, local)), flush=True)
+            print(json.dumps(run_crossover(args, local) if args.crossover else run_growth(args, local)), flush=True)
         if world > 1:
             torch.distributed.destroy_process_group()
         return

@@ -80,12 +80,24 @@ extern "C" {
  *                    that leaves c + 1 top nodes adds a new top level over
  *                    them; zha_depth gives the current depth
  *   capacity_tokens  rows per KV head in K and V (room for appends)
+ *   router_dtype     ZHA_F32: the routing reads the fp32 g rows.  ZHA_BF16:
+ *                    the build and every append also store a bf16 copy of
+ *                    each node's g rows (round to nearest even) with plane
+ *                    offsets recomputed from that copy, m_j - r_j.g~_j/sqrt(d)
+ *                    (so each rounded plane still passes through (r_j, m_j)),
+ *                    and the routing reads those: half the router's bytes
+ *                    ("ZHA 用树形稀疏注意力改造现有大模型", section
+ *                    "几百倍加速，离实际部署还有多远": a reduced-precision
+ *                    router).  Compiled for bf16 caches with d = 128.
+ *   reserved         0
  */
 typedef struct {
     int32_t h_kv, h_q, d, R, c, D;
     int32_t kv_dtype;
     int32_t max_depth;
     int64_t capacity_tokens;
+    int32_t router_dtype;
+    int32_t reserved;
 } zha_config;
 
 typedef struct zha_ctx zha_ctx; /* opaque host-side state: pointers and sizes only */
@@ -269,6 +281,14 @@ int64_t zha_n_tokens(const zha_ctx *ctx);
  */
 int zha_summary_layout(const zha_ctx *ctx, int32_t level, int64_t *g_offset, int64_t *b_offset,
                        int64_t *m_offset, int64_t *node_cap);
+
+/*
+ * Where the bf16 router copy of level `level` lives inside the workspace
+ * (router_dtype ZHA_BF16): byte offsets of g~ [h_kv][node_cap][R][d] bf16
+ * and of its plane offsets [h_kv][node_cap][R] fp32, and node_cap.
+ * ZHA_ERR_BAD_ARG for an invalid level or a context without the copy.
+ */
+int zha_router_layout(const zha_ctx *ctx, int32_t level, int64_t *g_offset, int64_t *b_offset, int64_t *node_cap);
 
 /* Static description of a status code. */
 const char *zha_strerror(int code);

@@ -100,6 +100,52 @@ def check_build(cache, trees, rtol: float = BUILD_RTOL, levels=None, sample=None
     return worst
 
 
+def router_trees(cache):
+    """Oracle trees over the GPU's bf16 router copy (router_dtype ZHA_BF16):
+    per KV head, every present level's m (the GPU's fp32 m) and g~ (the
+    bf16 copy, widened exactly) as an oracle summary store, so that the
+    oracle routes over the same quantised summaries as the GPU."""
+    cfg = cache.cfg
+    D = cache.depth
+    n = cache.n_tokens
+    counts = [level_count(n, cfg.c, lv) for lv in range(1, D + 1)]
+    off = np.zeros(D, dtype=np.int64)
+    off[1:] = np.cumsum(counts)[:-1]
+    trees = []
+    for kh in range(cfg.h_kv):
+        ms, gs, bs = [], [], []
+        for lv in range(1, D + 1):
+            g16, b16 = cache.router_summaries(lv)
+            _, _, m = cache.summaries(lv)
+            ms.append(m[kh].double().cpu().numpy())
+            gs.append(g16[kh].double().cpu().numpy())
+            bs.append(b16[kh].double().cpu().numpy())
+        trees.append(oracle.Tree(np.ascontiguousarray(np.concatenate(ms)), np.ascontiguousarray(np.concatenate(gs)),
+                                 np.ascontiguousarray(np.concatenate(bs)), off, n, cfg.c, D))
+    return trees
+
+
+def check_router_copy(cache, trees, ref_cpu, rtol: float = BUILD_RTOL):
+    """The bf16 router copy against the oracle's exact summaries: every g~
+    element is the exact g_j rounded to bf16 (within one bf16 step of it,
+    plus the fp32 tolerance), and every plane offset is m_j - r_j.g~_j/sqrt(d)
+    recomputed in fp64 from the GPU's own g~ and the oracle's m_j."""
+    cfg = cache.cfg
+    for lv in range(1, cache.depth + 1):
+        g16, b16 = cache.router_summaries(lv)
+        for kh, tree in enumerate(trees):
+            mo, go, _ = tree.level(lv)
+            gq = g16[kh].double().cpu().numpy()
+            bq = b16[kh].double().cpu().numpy()
+            scale_g = np.maximum(1.0, np.abs(go).max(axis=-1, keepdims=True))
+            err = np.abs(gq - go) - 2.0 ** -8 * np.abs(go)
+            assert np.max(err / scale_g) <= 2 * rtol, ("router g", lv, kh, float(np.max(err / scale_g)))
+            r = np.asarray(ref_cpu[kh], dtype=np.float64)
+            b_ref = mo - np.einsum("nrd,rd->nr", gq, r) / np.sqrt(cfg.d)
+            eb = np.abs(bq - b_ref) / np.maximum(1.0, np.maximum(np.abs(mo), np.abs(mo - b_ref)))
+            assert eb.max() <= rtol, ("router b", lv, kh, float(eb.max()))
+
+
 def parity_log_path() -> str:
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     return os.environ.get("ZHA_PARITY_LOG") or os.path.join(root, "gpurun_out", "parity_counts.jsonl")

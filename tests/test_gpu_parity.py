@@ -389,3 +389,47 @@ def test_depth_growth_build_starts_deeper():
     assert grow.status() == zha.ZHA_OK
     check_decode(res, trees, K, V, ref, q.double().numpy(), 0.8, N, c, grow.depth, h_q // h_kv, "bf16",
                  case="depth growth build N=5000 c=8 depth 4")
+
+
+ROUTER_CASES = {
+    "wide": W["wide_256k"].scaled(16384 + 100, steps=2),
+    "deep": W["deep_256k"].scaled(16384 + 37, steps=2),
+    "light": W["light_1m"].scaled(300000 + 5, steps=2),
+}
+
+
+@pytest.mark.parametrize("name", list(ROUTER_CASES))
+def test_bf16_router(name):
+    """router_dtype ZHA_BF16: the routing reads a bf16 copy of every g row.
+    The copy is the oracle's exact g rounded to bf16, its plane offsets are
+    recomputed from it, and the GPU's routing matches the oracle routing over
+    that same quantised store (the attention is exact as always); appends
+    keep the copy current."""
+    from parity import check_router_copy, router_trees
+    w = ROUTER_CASES[name]
+    inp = workloads.generate(w, "cpu")
+    K, V = inp.K.clone(), inp.V.clone()
+    cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, zha.ZHA_BF16, w.capacity, router_dtype=zha.ZHA_BF16)
+    dK, dV, dref = inp.K.cuda(), inp.V.cuda(), inp.ref.cuda()
+    cache.build(dK, dV, w.n_tokens, dref)
+    trees = oracle_trees(K, inp.ref, w.n_tokens, w.c, w.D, capacity=w.capacity)
+    n = w.n_tokens
+    app = 0
+    for s in range(w.steps):
+        for _ in range(w.appends_per_step):
+            cache.append(inp.K_app[app].cuda(), inp.V_app[app].cuda())
+            K[:, n] = inp.K_app[app]
+            V[:, n] = inp.V_app[app]
+            for kh in range(w.h_kv):
+                oracle.append_update(trees[kh], K[kh], inp.ref[kh])
+            n += 1
+            app += 1
+        torch.cuda.synchronize()
+        check_build(cache, trees)
+        check_router_copy(cache, trees, inp.ref)
+        q = inp.Q[s]
+        res = cache.decode(q.cuda(), w.p, trace_cap=oracle.level_nodes(w.capacity, w.c, 1))
+        torch.cuda.synchronize()
+        assert cache.status() == zha.ZHA_OK
+        check_decode(res, router_trees(cache), K, V, inp.ref, q.double().numpy(), w.p, n, w.c, w.D, w.group,
+                     w.kv_dtype, case=f"bf16 router {name} step {s}")

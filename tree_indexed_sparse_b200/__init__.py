@@ -28,7 +28,8 @@ ZHA_BF16 = 1
 # every symbol include/zha.h declares
 EXPORTS = ["zha_workspace_bytes", "zha_create", "zha_destroy", "zha_build", "zha_append", "zha_decode",
            "zha_dense_decode", "zha_dense_decode_static", "zha_device_status", "zha_set_phase_timer",
-           "zha_set_wait_budget", "zha_depth", "zha_n_tokens", "zha_summary_layout", "zha_strerror"]
+           "zha_set_wait_budget", "zha_depth", "zha_n_tokens", "zha_summary_layout", "zha_router_layout",
+           "zha_strerror"]
 
 
 class ZhaError(RuntimeError):
@@ -41,7 +42,8 @@ class zha_config(ctypes.Structure):
     _fields_ = [("h_kv", ctypes.c_int32), ("h_q", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("R", ctypes.c_int32), ("c", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("kv_dtype", ctypes.c_int32), ("max_depth", ctypes.c_int32),
-                ("capacity_tokens", ctypes.c_int64)]
+                ("capacity_tokens", ctypes.c_int64), ("router_dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -79,6 +81,8 @@ def _load() -> ctypes.CDLL:
     lib.zha_summary_layout.argtypes = [P, I32, ctypes.POINTER(I64), ctypes.POINTER(I64),
                                        ctypes.POINTER(I64), ctypes.POINTER(I64)]
     lib.zha_summary_layout.restype = ctypes.c_int
+    lib.zha_router_layout.argtypes = [P, I32, ctypes.POINTER(I64), ctypes.POINTER(I64), ctypes.POINTER(I64)]
+    lib.zha_router_layout.restype = ctypes.c_int
     lib.zha_strerror.argtypes = [ctypes.c_int]
     lib.zha_strerror.restype = ctypes.c_char_p
     return lib
@@ -179,6 +183,13 @@ def zha_summary_layout(ctx, level: int):
     return int(g.value), int(b.value), int(m.value), int(n.value)
 
 
+def zha_router_layout(ctx, level: int):
+    g, b, n = (ctypes.c_int64() for _ in range(3))
+    _check(lib.zha_router_layout(ctx, int(level), ctypes.byref(g), ctypes.byref(b), ctypes.byref(n)),
+           "zha_router_layout")
+    return int(g.value), int(b.value), int(n.value)
+
+
 # ---- convenience owner of one context's device buffers ----------------------
 
 class ZhaCache:
@@ -189,10 +200,10 @@ class ZhaCache:
     """
 
     def __init__(self, h_kv: int, h_q: int, d: int, R: int, c: int, D: int, kv_dtype: int,
-                 capacity_tokens: int, device="cuda", max_depth: int = 0):
+                 capacity_tokens: int, device="cuda", max_depth: int = 0, router_dtype: int = ZHA_F32):
         import torch
 
-        self.cfg = zha_config(h_kv, h_q, d, R, c, D, kv_dtype, max_depth, capacity_tokens)
+        self.cfg = zha_config(h_kv, h_q, d, R, c, D, kv_dtype, max_depth, capacity_tokens, router_dtype, 0)
         nbytes = zha_workspace_bytes(self.cfg)
         if nbytes < 0:
             raise ZhaError(nbytes, "zha_workspace_bytes")
@@ -287,3 +298,16 @@ class ZhaCache:
         b = view(bo, (c.h_kv, cap, c.R))[:, :n]
         m = view(mo, (c.h_kv, cap, c.R))[:, :n]
         return g, b, m
+
+    def router_summaries(self, level: int):
+        """(g~ [h_kv, nodes, R, d] bf16, b~ [h_kv, nodes, R] fp32): the bf16
+        router copy of level `level` (router_dtype ZHA_BF16)."""
+        import torch
+
+        go, bo, cap = zha_router_layout(self.ctx, level)
+        c = self.cfg
+        n = -(-self.n_tokens // c.c ** level) if self.n_tokens else 0
+        ws = self.workspace
+        g = ws[go:go + 2 * c.h_kv * cap * c.R * c.d].view(torch.bfloat16).view(c.h_kv, cap, c.R, c.d)[:, :n]
+        b = ws[bo:bo + 4 * c.h_kv * cap * c.R].view(torch.float32).view(c.h_kv, cap, c.R)[:, :n]
+        return g, b

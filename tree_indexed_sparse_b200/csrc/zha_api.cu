@@ -55,15 +55,16 @@ int check_config(const zha_config *cfg) {
     if (cfg->kv_dtype != ZHA_F32 && cfg->kv_dtype != ZHA_BF16) return ZHA_ERR_BAD_ARG;
     if (cfg->capacity_tokens < 1 || cfg->capacity_tokens > (int64_t)0x7fffffff) return ZHA_ERR_BAD_ARG;
     if (cfg->max_depth != 0 && (cfg->max_depth <= cfg->D || cfg->max_depth > MAXD)) return ZHA_ERR_BAD_ARG;
+    if ((cfg->router_dtype != ZHA_F32 && cfg->router_dtype != ZHA_BF16) || cfg->reserved != 0) return ZHA_ERR_BAD_ARG;
     const int G = cfg->h_q / cfg->h_kv;
-    if (!compiled_combo(cfg->kv_dtype, cfg->d, cfg->R, G)) return ZHA_ERR_UNSUPPORTED;
+    if (!compiled_combo(cfg->kv_dtype, cfg->d, cfg->R, G, cfg->router_dtype)) return ZHA_ERR_UNSUPPORTED;
     return ZHA_OK;
 }
 
 // Byte layout of the workspace.  Each region starts 256-byte aligned.
 struct Layout {
     int64_t node_cap[MAXD], slot_cap[MAXD];
-    int64_t g_off[MAXD], b_off[MAXD], m_off[MAXD];
+    int64_t g_off[MAXD], b_off[MAXD], m_off[MAXD], g16_off[MAXD], b16_off[MAXD];
     int64_t kid_off[MAXD], kmask_off[MAXD];
     int64_t seg_off, hseg_off, lvl_off, rdsc_off, scores_off, snode_off, skeep_off, tmax_off, tcnt_off, tsum_off;
     int64_t hcnt_off, hmass_off, cw_off, cs_off, ccnt_off, ticket_off, part_off, sync_off, status_off;
@@ -96,6 +97,13 @@ void make_layout(const zha_config *cfg, Layout *L) {
         off = align256(off + H * nc * cfg->R * 4);
         L->m_off[l - 1] = off;
         off = align256(off + H * nc * cfg->R * 4);
+        L->g16_off[l - 1] = L->b16_off[l - 1] = -1;
+        if (cfg->router_dtype == ZHA_BF16) {
+            L->g16_off[l - 1] = off;
+            off = align256(off + H * nc * cfg->R * cfg->d * 2);
+            L->b16_off[l - 1] = off;
+            off = align256(off + H * nc * cfg->R * 4);
+        }
     }
     // frontier slots of level l: every top node, or c children of each node
     // of level l + 1
@@ -208,6 +216,8 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
         t.g[l - 1] = reinterpret_cast<float *>(ws + L.g_off[l - 1]);
         t.b[l - 1] = reinterpret_cast<float *>(ws + L.b_off[l - 1]);
         t.m[l - 1] = reinterpret_cast<float *>(ws + L.m_off[l - 1]);
+        t.g16[l - 1] = L.g16_off[l - 1] >= 0 ? reinterpret_cast<uint16_t *>(ws + L.g16_off[l - 1]) : nullptr;
+        t.b16[l - 1] = L.b16_off[l - 1] >= 0 ? reinterpret_cast<float *>(ws + L.b16_off[l - 1]) : nullptr;
         d.kept_ids[l - 1] = reinterpret_cast<int32_t *>(ws + L.kid_off[l - 1]);
         d.kept_mask[l - 1] = reinterpret_cast<uint8_t *>(ws + L.kmask_off[l - 1]);
         d.slot_cap[l - 1] = L.slot_cap[l - 1];
@@ -385,6 +395,15 @@ int zha_summary_layout(const zha_ctx *ctx, int32_t level, int64_t *g_offset, int
     if (g_offset) *g_offset = reinterpret_cast<const unsigned char *>(ctx->t.g[level - 1]) - ws;
     if (b_offset) *b_offset = reinterpret_cast<const unsigned char *>(ctx->t.b[level - 1]) - ws;
     if (m_offset) *m_offset = reinterpret_cast<const unsigned char *>(ctx->t.m[level - 1]) - ws;
+    if (node_cap) *node_cap = ctx->t.node_cap[level - 1];
+    return ZHA_OK;
+}
+
+int zha_router_layout(const zha_ctx *ctx, int32_t level, int64_t *g_offset, int64_t *b_offset, int64_t *node_cap) {
+    if (!ctx || level < 1 || level > ctx->Dmax || !ctx->t.g16[level - 1]) return ZHA_ERR_BAD_ARG;
+    const unsigned char *ws = ctx->ws;
+    if (g_offset) *g_offset = reinterpret_cast<const unsigned char *>(ctx->t.g16[level - 1]) - ws;
+    if (b_offset) *b_offset = reinterpret_cast<const unsigned char *>(ctx->t.b16[level - 1]) - ws;
     if (node_cap) *node_cap = ctx->t.node_cap[level - 1];
     return ZHA_OK;
 }

@@ -67,8 +67,8 @@ cudaError_t launch_dense(const Decode &dc, int n_cta, cudaStream_t s) {
     return cudaErrorInvalidValue;
 }
 
-bool compiled_combo(int kv_dtype, int d, int R, int G) {
-    (void)kv_dtype;
+bool compiled_combo(int kv_dtype, int d, int R, int G, int router) {
+    if (router == 1 && (kv_dtype != 1 || d != 128)) return false;  // bf16 router: bf16 caches, d = 128
     return (d == 64 || d == 128) && (R == 1 || R == 16) && (G == 1 || G == 4);
 }
 

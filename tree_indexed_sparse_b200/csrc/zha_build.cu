@@ -20,6 +20,8 @@
 // d-slice [l*VEC, (l+1)*VEC) of every key, reference query and g row; dot
 // products are per-lane fmaf chains followed by a 32-lane reduce-scatter.
 // The kernels are bound by HBM for R = 1 and by fp32 FMA for R = 16.
+#include <cuda_bf16.h>
+
 #include <algorithm>
 
 #include "zha_device.cuh"
@@ -32,6 +34,24 @@ template <int HD, int R>
 __device__ __forceinline__ void load_ref(const float *ref_h, float (&rj)[R][HD / 32], int lane) {
 #pragma unroll
     for (int j = 0; j < R; ++j) Vec<float, HD / 32>::load(ref_h + j * HD + lane * (HD / 32), rj[j]);
+}
+
+// The router's bf16 copy of one plane (this lane's VEC elements of g_j) and
+// its plane offset recomputed from that copy, b~_j = m_j - r_j.g~_j/sqrt(d),
+// so that the rounded plane still passes through (r_j, m_j).  The dot
+// product takes the same order as b_j's.  `writer` stores the offset.
+template <int VEC>
+__device__ __forceinline__ void router_plane(const float (&g)[VEC], const float (&r)[VEC], float m, float scale,
+                                             uint16_t *g16dst, float *b16dst, int lane, int writer) {
+    float gq[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(g[e]);
+        g16dst[e] = __bfloat16_as_ushort(h);
+        gq[e] = __bfloat162float(h);
+    }
+    const float dot = warp_sum(lane_dot<VEC>(r, gq));
+    if (lane == writer) *b16dst = m - scale * dot;
 }
 
 // Tokens per leaf tile processed by one warp: a whole number of leaves and at
@@ -49,9 +69,11 @@ struct LeafOps {
     // Summaries of the leaves covering tokens [tok0, tok0 + ntok) of one head
     // (tok0 a multiple of c).  sh: warp-private shared scratch of
     // ntok*R + (ntok/c + 1)*R floats.
+    // g16L / b16L: the router's bf16 copy and its offsets (null: none).
     static __device__ void tile(const KT *__restrict__ Kh, int64_t tok0, int ntok, int c,
                                 const float (&rj)[R][VEC], float scale, float *__restrict__ gL,
-                                float *__restrict__ bL, float *__restrict__ mL, float *sh, int lane) {
+                                float *__restrict__ bL, float *__restrict__ mL, float *sh, int lane,
+                                uint16_t *__restrict__ g16L, float *__restrict__ b16L) {
         float *s_sh = sh;
         const int nleaf = (ntok + c - 1) / c;
         float *m_sh = sh + ntok * R;
@@ -117,6 +139,9 @@ struct LeafOps {
                 for (int e = 0; e < VEC; ++e) dst[e] = acc[j][e];
                 const float dot = warp_sum(lane_dot<VEC>(rj[j], acc[j]));
                 if (lane == (j & 31)) bL[node * R + j] = m_sh[lf * R + j] - scale * dot;
+                if (g16L)
+                    router_plane<VEC>(acc[j], rj[j], m_sh[lf * R + j], scale,
+                                      g16L + (node * R + j) * HD + lane * VEC, b16L + node * R + j, lane, j & 31);
             }
         }
         __syncwarp();
@@ -133,7 +158,7 @@ struct ParentOps {
     static __device__ void node(const float *__restrict__ gC, const float *__restrict__ bC, int64_t ch0,
                                 int nch, const float (&rj)[R][VEC], float scale, float *__restrict__ gP,
                                 float *__restrict__ bP, float *__restrict__ mP, int64_t n, float *sh,
-                                int lane) {
+                                int lane, uint16_t *__restrict__ g16P, float *__restrict__ b16P) {
         float *e_sh = sh;
         float *m_sh = sh + nch * R;
         // child estimates at every reference query
@@ -212,6 +237,9 @@ struct ParentOps {
             for (int e = 0; e < VEC; ++e) dst[e] = acc[j][e];
             const float dot = warp_sum(lane_dot<VEC>(rj[j], acc[j]));
             if (lane == (j & 31)) bP[n * R + j] = m_sh[j] - scale * dot;
+            if (g16P)
+                router_plane<VEC>(acc[j], rj[j], m_sh[j], scale, g16P + (n * R + j) * HD + lane * VEC,
+                                  b16P + n * R + j, lane, j & 31);
         }
         __syncwarp();
     }
@@ -243,7 +271,9 @@ __global__ void __launch_bounds__(BUILD_THREADS) k_build_leaves(Tree t) {
         const KT *Kh = reinterpret_cast<const KT *>(t.K) + (int64_t)kh * t.kv_cap * HD;
         const int64_t nc = t.node_cap[0];
         LeafOps<KT, HD, R>::tile(Kh, tok0, ntok, t.c, rj, t.scale, t.g[0] + (int64_t)kh * nc * R * HD,
-                                 t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, sh, lane);
+                                 t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, sh, lane,
+                                 t.g16[0] ? t.g16[0] + (int64_t)kh * nc * R * HD : nullptr,
+                                 t.g16[0] ? t.b16[0] + (int64_t)kh * nc * R : nullptr);
     }
 }
 
@@ -272,7 +302,8 @@ __global__ void __launch_bounds__(BUILD_THREADS) k_build_parents(Tree t, int lev
         ParentOps<HD, R>::node(t.g[level - 2] + (int64_t)kh * capC * R * HD, t.b[level - 2] + (int64_t)kh * capC * R,
                                ch0, nch, rj, t.scale, t.g[level - 1] + (int64_t)kh * capP * R * HD,
                                t.b[level - 1] + (int64_t)kh * capP * R, t.m[level - 1] + (int64_t)kh * capP * R,
-                               n, sh, lane);
+                               n, sh, lane, t.g16[level - 1] ? t.g16[level - 1] + (int64_t)kh * capP * R * HD : nullptr,
+                               t.g16[level - 1] ? t.b16[level - 1] + (int64_t)kh * capP * R : nullptr);
     }
 }
 
@@ -293,7 +324,8 @@ struct PlaneOps {
     // Kr: the leaf's rows, row i at Kr + i * HD (the cache, or a shared copy).
     static __device__ void leaf(const KT *Kr, int ntok, const float (&r)[VEC], int j,
                                 float scale, float *__restrict__ gL, float *__restrict__ bL, float *__restrict__ mL,
-                                int64_t n, float *sh, int lane) {
+                                int64_t n, float *sh, int lane, uint16_t *__restrict__ g16L,
+                                float *__restrict__ b16L) {
         for (int i0 = 0; i0 < ntok; i0 += 32) {
             float v[32];
 #pragma unroll
@@ -339,6 +371,7 @@ struct PlaneOps {
         for (int e = 0; e < VEC; ++e) dst[e] = acc[e];
         const float dot = warp_sum(lane_dot<VEC>(r, acc));
         if (lane == 0) bL[n * R + j] = m - scale * dot;
+        if (g16L) router_plane<VEC>(acc, r, m, scale, g16L + (n * R + j) * HD + lane * VEC, b16L + n * R + j, lane, 0);
         __syncwarp();
     }
 
@@ -348,7 +381,8 @@ struct PlaneOps {
     // gr + (i * R + j') * HD and br[i * R + j'] (the store, or a shared copy).
     static __device__ void parent(const float *gr, const float *br, int nch,
                                   const float (&r)[VEC], int j, float scale, float *__restrict__ gP,
-                                  float *__restrict__ bP, float *__restrict__ mP, int64_t n, float *sh, int lane) {
+                                  float *__restrict__ bP, float *__restrict__ mP, int64_t n, float *sh, int lane,
+                                  uint16_t *__restrict__ g16P, float *__restrict__ b16P) {
         // child estimates at r_j: max over the child's planes j'
         constexpr int CPB = 32 / R;  // children per batch of 32 dot products
         for (int c0 = 0; c0 < nch; c0 += CPB) {
@@ -403,6 +437,7 @@ struct PlaneOps {
         for (int e = 0; e < VEC; ++e) dst[e] = acc[e];
         const float dot = warp_sum(lane_dot<VEC>(r, acc));
         if (lane == 0) bP[n * R + j] = m - scale * dot;
+        if (g16P) router_plane<VEC>(acc, r, m, scale, g16P + (n * R + j) * HD + lane * VEC, b16P + n * R + j, lane, 0);
         __syncwarp();
     }
 };
@@ -490,7 +525,9 @@ __global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict_
             Kr = reinterpret_cast<const KT *>(stg);
         }
         PlaneOps<KT, HD, R>::leaf(Kr, ntok, r, j, t.scale, t.g[0] + (int64_t)kh * nc * R * HD,
-                                  t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, n, sh, lane);
+                                  t.b[0] + (int64_t)kh * nc * R, t.m[0] + (int64_t)kh * nc * R, n, sh, lane,
+                                  t.g16[0] ? t.g16[0] + (int64_t)kh * nc * R * HD : nullptr,
+                                  t.g16[0] ? t.b16[0] + (int64_t)kh * nc * R : nullptr);
     }
     __syncthreads();
     for (int level = 2; level <= t.D; ++level) {
@@ -510,7 +547,9 @@ __global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict_
         }
         PlaneOps<KT, HD, R>::parent(gr, br, nch, r, j, t.scale,
                                     t.g[level - 1] + (int64_t)kh * capP * R * HD, t.b[level - 1] + (int64_t)kh * capP * R,
-                                    t.m[level - 1] + (int64_t)kh * capP * R, n, sh, lane);
+                                    t.m[level - 1] + (int64_t)kh * capP * R, n, sh, lane,
+                                    t.g16[level - 1] ? t.g16[level - 1] + (int64_t)kh * capP * R * HD : nullptr,
+                                    t.g16[level - 1] ? t.b16[level - 1] + (int64_t)kh * capP * R : nullptr);
         __syncthreads();
     }
 }

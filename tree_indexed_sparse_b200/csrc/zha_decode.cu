@@ -98,7 +98,7 @@ __device__ __noinline__ void write_lists(const Decode &a, int kh, int tr) {
 // memory (after an LV_ALL or LV_SPLIT level) or the segments of an LV_TEAM
 // level in global memory; a level routed by every CTA after an LV_TEAM level
 // first copies those segments in.  Warps 0-7.
-template <int HD, int R, int G>
+template <int HD, int R, int G, typename RT>
 __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, unsigned char *smem, TeamSync &ts) {
     using SM = RouteSmem<G>;
     uint32_t *pref = reinterpret_cast<uint32_t *>(smem + SM::off_pref);
@@ -117,7 +117,7 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
     stages_init<G>(smem);
 #pragma unroll 1
     for (int l = D; l >= 1; --l) {
-        const int mode = level_mode<HD, R>(S, T);
+        const int mode = level_mode<HD, R, RT>(S, T);
         uint32_t F[G];
         int64_t Snext = 0;
         if (mode != LV_TEAM) {
@@ -134,14 +134,14 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
                 par_local = true;
             }
             int64_t nk = 0;
-            if (!route_level_rd<HD, R, G>(a, l, kh, T, tr, S, mode, buf, smem, ts, F, nk)) return false;
+            if (!route_level_rd<HD, R, G, RT>(a, l, kh, T, tr, S, mode, buf, smem, ts, F, nk)) return false;
             if (mode == LV_SPLIT) buf ^= 1;
             Tp = 1;
             Sp = S;
             Snext = nk * a.t.c;
         } else {
             int Tout;
-            if (!route_level<HD, R, G>(a, l, kh, T, tr, S, Tp, Sp, par_local, smem, ts, F, Tout)) return false;
+            if (!route_level<HD, R, G, RT>(a, l, kh, T, tr, S, Tp, Sp, par_local, smem, ts, F, Tout)) return false;
             par_local = false;
             Tp = Tout;
             Sp = S;
@@ -161,7 +161,7 @@ __device__ __noinline__ bool route_kvh(const Decode &a, int kh, int tr, int T, u
     return true;
 }
 
-template <typename KT, int HD, int R, int G>
+template <typename KT, int HD, int R, int G, typename RT>
 __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__ Decode a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ StageMap map;
@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__
     bool ok = true;
     if (router && warp < ACW) {
         TeamSync ts{words + kh, abortw, a.status, &s_flag, nbk, 0u, a.wait_budget};
-        ok = route_kvh<HD, R, G>(a, kh, tr, nbk, smem, ts);
+        ok = route_kvh<HD, R, G, RT>(a, kh, tr, nbk, smem, ts);
     }
     __shared__ int s_ok;
     if (threadIdx.x == 0) s_ok = 1;
@@ -225,16 +225,16 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__
     kernel_exit(words, h_kv + 3, h_kv + 1);
 }
 
-template <typename KT, int HD, int R, int G>
+template <typename KT, int HD, int R, int G, typename RT>
 static size_t decode_smem() {
     return std::max(RouteSmem<G>::bytes, ASmem<KT, HD, G>::bytes);
 }
 
-template <typename KT, int HD, int R, int G>
+template <typename KT, int HD, int R, int G, typename RT>
 static cudaError_t decode_impl(const Decode &dc, int n_cta, cudaStream_t s) {
-    const size_t smem = decode_smem<KT, HD, R, G>();
+    const size_t smem = decode_smem<KT, HD, R, G, RT>();
     static PerDeviceMax<> attr;
-    const cudaError_t err = allow_smem(k_decode<KT, HD, R, G>, smem, attr);
+    const cudaError_t err = allow_smem(k_decode<KT, HD, R, G, RT>, smem, attr);
     if (err != cudaSuccess) return err;
     // cooperative (the CTAs meet at barriers), and a programmatic dependent
     // of the previous kernel so that its launch overlaps that kernel's tail
@@ -250,42 +250,49 @@ static cudaError_t decode_impl(const Decode &dc, int n_cta, cudaStream_t s) {
     at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, k_decode<KT, HD, R, G>, dc);
+    return cudaLaunchKernelEx(&cfg, k_decode<KT, HD, R, G, RT>, dc);
 }
 
-template <typename KT, int HD, int R, int G>
+template <typename KT, int HD, int R, int G, typename RT>
 static int decode_occupancy() {
-    const size_t smem = decode_smem<KT, HD, R, G>();
+    const size_t smem = decode_smem<KT, HD, R, G, RT>();
     static PerDeviceMax<> attr;
-    if (allow_smem(k_decode<KT, HD, R, G>, smem, attr) != cudaSuccess) return 0;
+    if (allow_smem(k_decode<KT, HD, R, G, RT>, smem, attr) != cudaSuccess) return 0;
     int blocks = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k_decode<KT, HD, R, G>, A_THREADS, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, k_decode<KT, HD, R, G, RT>, A_THREADS, smem) != cudaSuccess)
         return 0;
     return blocks;
 }
 
-#define ZHA_DECODE_DISPATCH(FN, ...)                                                         \
-    do {                                                                                     \
-        const Tree &t = dc.t;                                                                \
-        if (t.kv_dtype == 1) {                                                               \
-            if (t.d == 128 && t.R == 16 && t.G == 4) return FN<uint16_t, 128, 16, 4>(__VA_ARGS__); \
-            if (t.d == 128 && t.R == 1 && t.G == 4) return FN<uint16_t, 128, 1, 4>(__VA_ARGS__);   \
-            if (t.d == 128 && t.R == 16 && t.G == 1) return FN<uint16_t, 128, 16, 1>(__VA_ARGS__); \
-            if (t.d == 128 && t.R == 1 && t.G == 1) return FN<uint16_t, 128, 1, 1>(__VA_ARGS__);   \
-            if (t.d == 64 && t.R == 16 && t.G == 4) return FN<uint16_t, 64, 16, 4>(__VA_ARGS__);   \
-            if (t.d == 64 && t.R == 1 && t.G == 4) return FN<uint16_t, 64, 1, 4>(__VA_ARGS__);     \
-            if (t.d == 64 && t.R == 16 && t.G == 1) return FN<uint16_t, 64, 16, 1>(__VA_ARGS__);   \
-            if (t.d == 64 && t.R == 1 && t.G == 1) return FN<uint16_t, 64, 1, 1>(__VA_ARGS__);     \
-        } else {                                                                             \
-            if (t.d == 128 && t.R == 16 && t.G == 4) return FN<float, 128, 16, 4>(__VA_ARGS__);    \
-            if (t.d == 128 && t.R == 1 && t.G == 4) return FN<float, 128, 1, 4>(__VA_ARGS__);      \
-            if (t.d == 128 && t.R == 16 && t.G == 1) return FN<float, 128, 16, 1>(__VA_ARGS__);    \
-            if (t.d == 128 && t.R == 1 && t.G == 1) return FN<float, 128, 1, 1>(__VA_ARGS__);      \
-            if (t.d == 64 && t.R == 16 && t.G == 4) return FN<float, 64, 16, 4>(__VA_ARGS__);      \
-            if (t.d == 64 && t.R == 1 && t.G == 4) return FN<float, 64, 1, 4>(__VA_ARGS__);        \
-            if (t.d == 64 && t.R == 16 && t.G == 1) return FN<float, 64, 16, 1>(__VA_ARGS__);      \
-            if (t.d == 64 && t.R == 1 && t.G == 1) return FN<float, 64, 1, 1>(__VA_ARGS__);        \
-        }                                                                                    \
+#define ZHA_DECODE_DISPATCH(FN, ...)                                                                      \
+    do {                                                                                                  \
+        const Tree &t = dc.t;                                                                             \
+        if (t.g16[0]) {                                                                                   \
+            if (t.kv_dtype == 1 && t.d == 128) {                                                          \
+                if (t.R == 16 && t.G == 4) return FN<uint16_t, 128, 16, 4, uint16_t>(__VA_ARGS__);        \
+                if (t.R == 1 && t.G == 4) return FN<uint16_t, 128, 1, 4, uint16_t>(__VA_ARGS__);          \
+                if (t.R == 16 && t.G == 1) return FN<uint16_t, 128, 16, 1, uint16_t>(__VA_ARGS__);        \
+                if (t.R == 1 && t.G == 1) return FN<uint16_t, 128, 1, 1, uint16_t>(__VA_ARGS__);          \
+            }                                                                                             \
+        } else if (t.kv_dtype == 1) {                                                                     \
+            if (t.d == 128 && t.R == 16 && t.G == 4) return FN<uint16_t, 128, 16, 4, float>(__VA_ARGS__); \
+            if (t.d == 128 && t.R == 1 && t.G == 4) return FN<uint16_t, 128, 1, 4, float>(__VA_ARGS__);   \
+            if (t.d == 128 && t.R == 16 && t.G == 1) return FN<uint16_t, 128, 16, 1, float>(__VA_ARGS__); \
+            if (t.d == 128 && t.R == 1 && t.G == 1) return FN<uint16_t, 128, 1, 1, float>(__VA_ARGS__);   \
+            if (t.d == 64 && t.R == 16 && t.G == 4) return FN<uint16_t, 64, 16, 4, float>(__VA_ARGS__);   \
+            if (t.d == 64 && t.R == 1 && t.G == 4) return FN<uint16_t, 64, 1, 4, float>(__VA_ARGS__);     \
+            if (t.d == 64 && t.R == 16 && t.G == 1) return FN<uint16_t, 64, 16, 1, float>(__VA_ARGS__);   \
+            if (t.d == 64 && t.R == 1 && t.G == 1) return FN<uint16_t, 64, 1, 1, float>(__VA_ARGS__);     \
+        } else {                                                                                          \
+            if (t.d == 128 && t.R == 16 && t.G == 4) return FN<float, 128, 16, 4, float>(__VA_ARGS__);    \
+            if (t.d == 128 && t.R == 1 && t.G == 4) return FN<float, 128, 1, 4, float>(__VA_ARGS__);      \
+            if (t.d == 128 && t.R == 16 && t.G == 1) return FN<float, 128, 16, 1, float>(__VA_ARGS__);    \
+            if (t.d == 128 && t.R == 1 && t.G == 1) return FN<float, 128, 1, 1, float>(__VA_ARGS__);      \
+            if (t.d == 64 && t.R == 16 && t.G == 4) return FN<float, 64, 16, 4, float>(__VA_ARGS__);      \
+            if (t.d == 64 && t.R == 1 && t.G == 4) return FN<float, 64, 1, 4, float>(__VA_ARGS__);        \
+            if (t.d == 64 && t.R == 16 && t.G == 1) return FN<float, 64, 16, 1, float>(__VA_ARGS__);      \
+            if (t.d == 64 && t.R == 1 && t.G == 1) return FN<float, 64, 1, 1, float>(__VA_ARGS__);        \
+        }                                                                                                 \
     } while (0)
 
 cudaError_t launch_decode(const Decode &dc, int n_cta, cudaStream_t s) {

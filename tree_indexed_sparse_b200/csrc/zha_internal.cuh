@@ -28,6 +28,8 @@ struct Tree {
     float *g[MAXD];
     float *b[MAXD];
     float *m[MAXD];
+    uint16_t *g16[MAXD];          // router copy of g in bf16 ([node][R][d]; null when the router reads g)
+    float *b16[MAXD];             // its plane offsets, m - r.g16/sqrt(d) ([node][R])
     const void *K;
     const void *V;
     const float *ref;             // [h_kv][R][d]
@@ -109,6 +111,6 @@ cudaError_t launch_build_levels(const Tree &t, int from, int to, cudaStream_t s,
 cudaError_t launch_decode(const Decode &dc, int n_cta, cudaStream_t s);
 int decode_blocks_per_sm(const Decode &dc);
 cudaError_t launch_dense(const Decode &dc, int n_cta, cudaStream_t s);
-bool compiled_combo(int kv_dtype, int d, int R, int G);
+bool compiled_combo(int kv_dtype, int d, int R, int G, int router);
 
 }  // namespace zha

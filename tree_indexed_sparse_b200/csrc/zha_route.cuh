@@ -243,9 +243,22 @@ __device__ __forceinline__ float head_sum(const float (&v)[G], int lane) {
     }
 }
 
-template <int HD, int R>
+// The g rows and plane offsets the router reads: fp32 (RT = float) or the
+// bf16 copy (RT = uint16_t) with its own offsets.
+template <typename RT>
+__device__ __forceinline__ const RT *router_g(const Tree &t, int l);
+template <>
+__device__ __forceinline__ const float *router_g<float>(const Tree &t, int l) { return t.g[l - 1]; }
+template <>
+__device__ __forceinline__ const uint16_t *router_g<uint16_t>(const Tree &t, int l) { return t.g16[l - 1]; }
+template <typename RT>
+__device__ __forceinline__ const float *router_b(const Tree &t, int l) {
+    return sizeof(RT) == 2 ? t.b16[l - 1] : t.b[l - 1];
+}
+
+template <int HD, int R, typename RT>
 struct ScoreStage {
-    static constexpr int NODE_BYTES = R * HD * 4;                    // g rows of one node
+    static constexpr int NODE_BYTES = R * HD * (int)sizeof(RT);      // g rows of one node (fp32 or the bf16 copy)
     static constexpr int SLOTS = SW_BYTES / NODE_BYTES < SW_ROWS_MAX / R ? SW_BYTES / NODE_BYTES
                                                                           : SW_ROWS_MAX / R;  // slots per stage
     static constexpr int ROWS = SLOTS * R;                           // summary rows per stage
@@ -257,12 +270,12 @@ struct ScoreStage {
 // nodes) into this warp's stage buffer `dst`, completing on the stage barrier
 // `bar`.  Returns the plane offset of row `lane` (slot lane / R, plane
 // lane % R; 0 past the unit): a register load whose latency the copy hides.
-template <int HD, int R, int G>
+template <int HD, int R, int G, typename RT>
 __device__ __forceinline__ float stage_issue(const Level &L, int64_t c0, int64_t c1, int64_t k0, int64_t u,
-                                             const int32_t *pid, const uint8_t *pmk, const float *gb, const float *bb,
+                                             const int32_t *pid, const uint8_t *pmk, const RT *gb, const float *bb,
                                              int c, int clog, int32_t nl, unsigned char *dst, uint64_t *bar,
                                              int32_t *cn, uint8_t *cm, int lane) {
-    using C = ScoreStage<HD, R>;
+    using C = ScoreStage<HD, R, RT>;
     const int64_t sb = c0 + u * C::SLOTS;
     const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
     int nd = -1;
@@ -361,13 +374,13 @@ __device__ __forceinline__ void stages_inval(unsigned char *smem) {
 // keeps each node's maximum over its planes in registers.  Parent window:
 // ranks [k0, ...) in pid/pmk.  Writes L.sc / L.node at (s - L.s0) and folds
 // the maxima and counts per head into wm/wc[warp][h].
-template <int HD, int R, int G>
+template <int HD, int R, int G, typename RT>
 __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64_t c0, int64_t c1, int64_t k0,
                                           const int32_t *pid, const uint8_t *pmk, unsigned char *smem, float *wm,
                                           uint32_t *wc) {
     static_assert(G == 1 || G == 4, "query heads per KV head");
     static_assert(R == 1 || R % 8 == 0, "planes per node: 1 or a multiple of 8");
-    using C = ScoreStage<HD, R>;
+    using C = ScoreStage<HD, R, RT>;
     using SM = RouteSmem<G>;
     constexpr int VEC = HD / 32;
     constexpr int NW = GT / 32;
@@ -385,8 +398,8 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         for (int e = 0; e < VEC; ++e) qs[h][e] *= a.t.scale;
     }
     const int64_t cap = a.t.node_cap[l - 1];
-    const float *gb = a.t.g[l - 1] + (int64_t)kh * cap * R * HD;
-    const float *bb = a.t.b[l - 1] + (int64_t)kh * cap * R;
+    const RT *gb = router_g<RT>(a.t, l) + (int64_t)kh * cap * R * HD;
+    const float *bb = router_b<RT>(a.t, l) + (int64_t)kh * cap * R;
     const int c = a.t.c, clog = a.t.c_log2;
     const int32_t nl = a.t.n_level[l - 1];
     const int64_t nu = (c1 - c0 + C::SLOTS - 1) / C::SLOTS;  // units
@@ -397,10 +410,10 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
     const uint32_t u0 = uses[0], u1 = uses[1];
     float b0 = 0.f, b1 = 0.f;  // plane offsets of row `lane` of stages 0 and 1
     if (nmine > 0)
-        b0 = stage_issue<HD, R, G>(L, c0, c1, k0, warp, pid, pmk, gb, bb, c, clog, nl, bufs, &bars[0], cnode,
+        b0 = stage_issue<HD, R, G, RT>(L, c0, c1, k0, warp, pid, pmk, gb, bb, c, clog, nl, bufs, &bars[0], cnode,
                                    cmask, lane);
     if (nmine > 1)
-        b1 = stage_issue<HD, R, G>(L, c0, c1, k0, warp + NW, pid, pmk, gb, bb, c, clog, nl, bufs + SW_BYTES,
+        b1 = stage_issue<HD, R, G, RT>(L, c0, c1, k0, warp + NW, pid, pmk, gb, bb, c, clog, nl, bufs + SW_BYTES,
                                    &bars[1], cnode + SW_ROWS_MAX, cmask + SW_ROWS_MAX, lane);
     const int hl = lane % G;             // head of this lane's sum
     const int rl = (lane / G) % 8;       // row of this lane's sum within the batch
@@ -417,7 +430,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         if (!mbar_wait(&bars[st], ((st ? u1 : u0) + (uint32_t)(j / SW_STAGES)) & 1u, nullptr))
             set_status(a.status, ZHA_TIMEOUT_CODE);
         const float bl = st ? b1 : b0;  // plane offset of row `lane`
-        const float *cb = reinterpret_cast<const float *>(bufs + (size_t)st * SW_BYTES);
+        const RT *cb = reinterpret_cast<const RT *>(bufs + (size_t)st * SW_BYTES);
         float est = -INFINITY;
 #pragma unroll 1
         for (int r0 = 0; r0 < C::ROWS; r0 += 8) {
@@ -428,7 +441,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
                 const int r = r0 + q;
                 float gs[VEC];
                 if (r / R < ns) {
-                    Vec<float, VEC>::load(cb + (size_t)r * HD + lane * VEC, gs);
+                    Vec<RT, VEC>::load(cb + (size_t)r * HD + lane * VEC, gs);
                 } else {
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) gs[e] = 0.f;
@@ -478,7 +491,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         }
         __syncwarp();  // stage st is free
         if (j + SW_STAGES < nmine) {
-            const float bn = stage_issue<HD, R, G>(L, c0, c1, k0, u + (int64_t)SW_STAGES * NW, pid, pmk, gb, bb, c,
+            const float bn = stage_issue<HD, R, G, RT>(L, c0, c1, k0, u + (int64_t)SW_STAGES * NW, pid, pmk, gb, bb, c,
                                                    clog, nl, bufs + (size_t)st * SW_BYTES, &bars[st],
                                                    cnode + st * SW_ROWS_MAX, cmask + st * SW_ROWS_MAX, lane);
             if (st) b1 = bn;
@@ -1312,7 +1325,7 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
 // this CTA alone).  `S` is the frontier size, `pref`/Tp/Sp the parent level's
 // segments (loaded by the caller).  F[h] receives the frontier counts.
 // Returns false when a team barrier gave up.
-template <int HD, int R, int G>
+template <int HD, int R, int G, typename RT>
 __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, int tr, int64_t S, int Tp, int64_t Sp,
                                          bool par_local, unsigned char *smem, TeamSync &ts, uint32_t (&F)[G],
                                          int &Tout) {
@@ -1358,7 +1371,7 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
         int64_t k0 = 0;  // parents already local: the whole kept list from rank 0
         if (!L.top && !par_local) load_parents(a, L, c0, c1, pref, pid, pmk, k0);
         gsync();
-        score_chunks<HD, R, G>(a, L, c0, c1, k0, pid, pmk, smem, wm, wc);
+        score_chunks<HD, R, G, RT>(a, L, c0, c1, k0, pid, pmk, smem, wm, wc);
         gsync();
     }
     if (tid < G) {
@@ -1458,9 +1471,9 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
 
 // The way level l is routed by a team of T CTAs, from its frontier size S
 // (the same on every CTA).
-template <int HD, int R>
+template <int HD, int R, typename RT>
 __device__ __forceinline__ int level_mode(int64_t S, int T) {
-    constexpr int64_t node_bytes = (int64_t)R * (HD + 1) * 4;
+    constexpr int64_t node_bytes = (int64_t)R * (HD * (int64_t)sizeof(RT) + 4);
     if (S <= LOC_CAP && (T == 1 || (S <= RDA_SLOTS && S * node_bytes <= RDA_BYTES))) return LV_ALL;
     if (S <= RDS_MAX) return LV_SPLIT;
     return LV_TEAM;
@@ -1496,7 +1509,7 @@ __device__ __forceinline__ int32_t slot_node(const Decode &a, int l, bool top, c
 // (team size 1), which the leaf lists, the trace and the attention read
 // after the grid barrier.  F[h]: frontier counts.  false: the barrier gave
 // up.
-template <int HD, int R, int G>
+template <int HD, int R, int G, typename RT>
 __device__ __noinline__ bool route_level_rd(const Decode &a, int l, int kh, int T, int tr, int64_t S, int mode,
                                             int buf, unsigned char *smem, TeamSync &ts, uint32_t (&F)[G],
                                             int64_t &nk) {
@@ -1540,7 +1553,7 @@ __device__ __noinline__ bool route_level_rd(const Decode &a, int l, int kh, int 
         wc[tid] = 0u;
     }
     gsync();
-    if (L.n > 0) score_chunks<HD, R, G>(a, L, L.s0, L.s0 + L.n, 0, pid, pmk, smem, wm, wc);
+    if (L.n > 0) score_chunks<HD, R, G, RT>(a, L, L.s0, L.s0 + L.n, 0, pid, pmk, smem, wm, wc);
     if (mode == LV_SPLIT) {
         if (!ts.sync()) return false;
         // every slot's scores (written before the barrier) and node

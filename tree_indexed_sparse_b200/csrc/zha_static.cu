@@ -83,7 +83,7 @@ int zha_dense_decode_static(const zha_config *cfg, const void *d_K, const void *
         (reinterpret_cast<uintptr_t>(d_status) & 3u))
         return ZHA_ERR_BAD_ARG;
     const int G = cfg->h_q / cfg->h_kv;
-    if (!compiled_combo(cfg->kv_dtype, cfg->d, 1, G)) return ZHA_ERR_UNSUPPORTED;
+    if (!compiled_combo(cfg->kv_dtype, cfg->d, 1, G, 0)) return ZHA_ERR_UNSUPPORTED;
 
     DevScratch ds;
     const int rc = device_scratch(ds);
