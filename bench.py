@@ -283,8 +283,9 @@ def run_zha(args, rank, world, local):
     gen_s = time.time() - t0
     dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
     router_bf16 = args.router == "bf16"
+    nb = args.batch
     cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, device=dev,
-                         router_dtype=zha.ZHA_BF16 if router_bf16 else zha.ZHA_F32)
+                         router_dtype=zha.ZHA_BF16 if router_bf16 else zha.ZHA_F32, max_batch=nb)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     n1cap = -(-w.capacity // w.c)
@@ -300,19 +301,22 @@ def run_zha(args, rank, world, local):
     torch.cuda.synchronize()
     build_ms = eb0.elapsed_time(eb1)
 
-    out = torch.empty(w.h_q, w.d, dtype=torch.float32, device=dev)
-    leaf_idx = torch.empty(w.h_q, n1cap, dtype=torch.int32, device=dev)
-    n_leaf = torch.empty(w.h_q, dtype=torch.int32, device=dev)
-    visited = torch.empty(w.h_q, dtype=torch.int64, device=dev)
-    qs = inp.Q
+    out = torch.empty(nb, w.h_q, w.d, dtype=torch.float32, device=dev)
+    leaf_idx = torch.empty(nb, w.h_q, n1cap, dtype=torch.int32, device=dev)
+    n_leaf = torch.empty(nb, w.h_q, dtype=torch.int32, device=dev)
+    visited = torch.empty(nb, w.h_q, dtype=torch.int64, device=dev)
+    # the queries of step i: [nb, h_q, d], consecutive queries of the workload
+    qsteps = torch.stack([torch.stack([inp.Q[(i * nb + t) % w.steps] for t in range(nb)])
+                          for i in range(max(w.steps, 1))])
+    qs = qsteps if nb > 1 else inp.Q
 
     def decode(q, trace=None):
         if trace is None:
-            zha.zha_decode(cache.ctx, q, w.p, out, leaf_idx, n1cap, n_leaf, visited, None, None, 0,
-                           stream.cuda_stream)
+            zha.zha_decode_batch(cache.ctx, q, nb, w.p, out, leaf_idx, n1cap, n_leaf, visited, None, None, 0,
+                                 stream.cuda_stream)
         else:
-            zha.zha_decode(cache.ctx, q, w.p, out, leaf_idx, n1cap, n_leaf, visited, trace[0], trace[1],
-                           n1cap, stream.cuda_stream)
+            zha.zha_decode_batch(cache.ctx, q, nb, w.p, out, leaf_idx, n1cap, n_leaf, visited, trace[0], trace[1],
+                                 n1cap, stream.cuda_stream)
 
     def appends(i):
         """The appends of step i (the workload's own count per step)."""
@@ -322,8 +326,8 @@ def run_zha(args, rank, world, local):
 
     # pass A: traced, untimed -- algorithmic bytes of every step, warm-up
     # steps included (one k_decode launch per step, in step order)
-    tr_ids = torch.empty(w.D, w.h_q, n1cap, dtype=torch.int32, device=dev)
-    tr_cnt = torch.empty(w.D, w.h_q, dtype=torch.int32, device=dev)
+    tr_ids = torch.empty(w.D, nb * w.h_q, n1cap, dtype=torch.int32, device=dev)
+    tr_cnt = torch.empty(w.D, nb * w.h_q, dtype=torch.int32, device=dev)
     per_step_all = []
     leaves_per_head, vis_per_head = [], []
     for i in range(W + K):
@@ -332,7 +336,12 @@ def run_zha(args, rank, world, local):
         ids = tr_ids.cpu().numpy()
         cnt = tr_cnt.cpu().numpy()
         n_now = w.n_tokens + (i + 1) * per_step
-        rb, ab, slots, slots_level = step_bytes(w, ids, cnt, n_now, router_bf16)
+        rb, ab, slots, slots_level = 0, 0, 0, [0] * (w.D + 1)
+        for t in range(nb):  # every query's own routing and token set
+            sl = slice(t * w.h_q, (t + 1) * w.h_q)
+            r_, a_, s_, l_ = step_bytes(w, ids[:, sl], cnt[:, sl], n_now, router_bf16)
+            rb, ab, slots = rb + r_, ab + a_, slots + s_
+            slots_level = [x + y for x, y in zip(slots_level, l_)]
         app_b = sum(append_bytes(w, n_now - per_step + j + 1) for j in range(per_step))
         per_step_all.append((rb, ab, app_b, slots, n_now, slots_level))
         if i >= W:
@@ -382,7 +391,7 @@ def run_zha(args, rank, world, local):
     total_ms = sum(t_step)
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_step = total_ms / K
-    us_token = job_value(K, world, total_ms)
+    us_token = job_value(K * nb, world, total_ms)
 
     # appends after the decode steps (the workload's own count, or a burst of
     # APPEND_BURST for a workload without appends), back to back, one event
@@ -484,7 +493,7 @@ def run_zha(args, rank, world, local):
     # loop would send them; the device views of that row are the API's inputs.
     cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
     qc, kc, vc = qs.cpu(), inp.K_app.cpu(), inp.V_app.cpu()
-    qb = w.h_q * w.d * 4
+    qb = nb * w.h_q * w.d * 4
     kb = w.h_kv * w.d * kc.element_size()
     rows = []
     for i in range(W + K):
@@ -494,9 +503,9 @@ def run_zha(args, rank, world, local):
             parts += [kc[r].contiguous().view(torch.uint8).flatten(), vc[r].contiguous().view(torch.uint8).flatten()]
         rows.append(torch.cat(parts))
     hin = torch.stack(rows).pin_memory()
-    hout = torch.empty(w.h_q, w.d, dtype=torch.float32).pin_memory()
+    hout = torch.empty(out.shape, dtype=torch.float32).pin_memory()
     din = torch.empty(qb + 2 * kb * per_step, dtype=torch.uint8, device=dev)
-    dq = din[:qb].view(torch.float32).view(w.h_q, w.d)
+    dq = din[:qb].view(torch.float32).view(*qs.shape[1:])
     dkv = [(din[qb + 2 * kb * j:qb + 2 * kb * j + kb].view(inp.K.dtype).view(w.h_kv, w.d),
             din[qb + 2 * kb * j + kb:qb + 2 * kb * (j + 1)].view(inp.K.dtype).view(w.h_kv, w.d))
            for j in range(per_step)]
@@ -520,7 +529,8 @@ def run_zha(args, rank, world, local):
     e2e_us = max_over_ranks(e2e_us, world, dev)
 
     step_desc = (f"{per_step} zha_append calls then one zha_decode" if per_step else "one zha_decode") + \
-        " of one token, all query heads, batch 1, one layer"
+        (f" of one token, all query heads, batch 1, one layer" if nb == 1 else
+         f"_batch of {nb} query tokens against the same cache, all query heads, one layer; value per query token")
     res = {
         "metric": METRIC, "value": us_token, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_step, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
@@ -530,6 +540,7 @@ def run_zha(args, rank, world, local):
                    "step": step_desc,
                    "appends_after_steps": burst if base.appends_after else 0,
                    "router": "bf16 copy of g (reduced-precision router)" if router_bf16 else "fp32",
+                   "queries_per_decode": nb,
                    "l2": "256 MiB written between steps, outside the per-step events",
                    "parallelism": f"replicas x{world}"},
         "hbm_gbs": gbs, "hbm_frac": gbs / peak,
@@ -549,9 +560,10 @@ def run_zha(args, rank, world, local):
                     "union_slots_per_level": {f"level_{lv}": statistics.mean(s[5][lv] for s in timed_b)
                                               for lv in range(w.D, 0, -1)},
                     "timed_pass_reproduces_traced": bool(same)},
-        "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_us / nb, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "clocks": clk,
         "gpu_launches": K * (per_step + 1),
+        "dense_note": "dense is timed for one query token per call",
         "gen_s": gen_s, "wall_timed_s": wall,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -771,6 +783,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--crossover", action="store_true",
                     help="sweep the light workload's settings over context lengths, routed vs dense")
+    ap.add_argument("--batch", type=int, default=1,
+                    help="query tokens per decode call (zha_decode_batch); value is per query token")
     ap.add_argument("--router", choices=["f32", "bf16"], default="f32",
                     help="summaries the routing reads: fp32 (default) or the bf16 router copy")
     ap.add_argument("--growth", action="store_true",

@@ -89,7 +89,9 @@ extern "C" {
  *                    ("ZHA 用树形稀疏注意力改造现有大模型", section
  *                    "几百倍加速，离实际部署还有多远": a reduced-precision
  *                    router).  Compiled for bf16 caches with d = 128.
- *   reserved         0
+ *   max_batch        most queries one zha_decode_batch call may carry (0 or
+ *                    1: one); h_kv * max_batch <= 64.  The decode scratch
+ *                    is sized for it.
  */
 typedef struct {
     int32_t h_kv, h_q, d, R, c, D;
@@ -97,7 +99,7 @@ typedef struct {
     int32_t max_depth;
     int64_t capacity_tokens;
     int32_t router_dtype;
-    int32_t reserved;
+    int32_t max_batch;
 } zha_config;
 
 typedef struct zha_ctx zha_ctx; /* opaque host-side state: pointers and sizes only */
@@ -190,6 +192,25 @@ int zha_append(zha_ctx *ctx, const void *d_k, const void *d_v, void *stream);
 int zha_decode(zha_ctx *ctx, const float *d_q, float p, float *d_out, int32_t *d_leaf_idx,
                int32_t leaf_cap, int32_t *d_n_leaf, int64_t *d_nodes_visited,
                int32_t *d_trace_ids, int32_t *d_trace_counts, int32_t trace_cap, void *stream);
+
+/*
+ * Decode n_q query tokens against the same cache in one launch: each query
+ * is routed and attended exactly as zha_decode does it for one (every query
+ * sees the whole cache as it is; none sees another).  Multi-query routing:
+ * "Дерево сокращает сам поиск нужных ключей" (rit.work article) counts the
+ * routing of every query of a sequence against the tree.  The grid gives
+ * each (query, KV head) pair its own team of CTAs, so the queries route in
+ * parallel; the G query heads of a pair share its summary and K/V reads.
+ *   n_q              1 <= n_q <= zha_config.max_batch (or 1)
+ *   d_q, d_out       [n_q][h_q][d] fp32
+ *   d_leaf_idx       [n_q][h_q][leaf_cap]; d_n_leaf, d_nodes_visited [n_q][h_q]
+ *   d_trace_ids      nullable; [D][n_q * h_q][trace_cap], d_trace_counts [D][n_q * h_q]
+ * Returns ZHA_ERR_BAD_ARG for n_q outside [1, max_batch] and
+ * ZHA_ERR_UNSUPPORTED when n_q * h_kv exceeds the CTAs of one wave.
+ */
+int zha_decode_batch(zha_ctx *ctx, const float *d_q, int32_t n_q, float p, float *d_out, int32_t *d_leaf_idx,
+                     int32_t leaf_cap, int32_t *d_n_leaf, int64_t *d_nodes_visited, int32_t *d_trace_ids,
+                     int32_t *d_trace_counts, int32_t trace_cap, void *stream);
 
 /*
  * Dense flash-decode over the same cache (the comparison kernel): exact

@@ -433,3 +433,34 @@ def test_bf16_router(name):
         assert cache.status() == zha.ZHA_OK
         check_decode(res, router_trees(cache), K, V, inp.ref, q.double().numpy(), w.p, n, w.c, w.D, w.group,
                      w.kv_dtype, case=f"bf16 router {name} step {s}")
+
+
+@pytest.mark.parametrize("name,n_q", [("tiny_f32", 4), ("wide", 3), ("deep", 4), ("light", 4)])
+def test_batch_decode(name, n_q):
+    """zha_decode_batch: n_q queries against the same cache in one launch,
+    each (query, KV head) pair routed by its own team of CTAs.  Every query's
+    routing and output match the oracle, and its output matches the
+    one-query decode of the same query."""
+    c = get_case(name)
+    w = c.w
+    dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
+    cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, max_batch=n_q)
+    cache.build(c.dK, c.dV, c.n, c.dref)
+    qs = torch.stack([c.inp.Q[s % c.inp.Q.shape[0]] for s in range(n_q)])
+    cap = oracle.level_nodes(w.capacity, w.c, 1)
+    res = cache.decode_batch(qs.cuda(), w.p, trace_cap=cap)
+    torch.cuda.synchronize()
+    assert cache.status() == zha.ZHA_OK
+    h_q = w.h_q
+    for t in range(n_q):
+        res_t = {"out": res["out"][t], "leaf_idx": res["leaf_idx"][t], "n_leaf": res["n_leaf"][t],
+                 "visited": res["visited"][t], "trace_ids": res["trace_ids"][:, t * h_q:(t + 1) * h_q],
+                 "trace_counts": res["trace_counts"][:, t * h_q:(t + 1) * h_q]}
+        check_decode(res_t, c.trees, c.K, c.V, c.inp.ref, qs[t].double().numpy(), w.p, c.n, w.c, w.D, w.group,
+                     w.kv_dtype, case=f"batch {name} query {t} of {n_q}")
+        one = cache.decode(qs[t].cuda(), w.p)
+        torch.cuda.synchronize()
+        assert torch.max(torch.abs(one["out"] - res["out"][t])).item() <= OUT_TOL[w.kv_dtype]
+    with pytest.raises(zha.ZhaError) as e:
+        cache.decode_batch(torch.zeros(n_q + 1, h_q, w.d, device="cuda"), w.p)
+    assert e.value.code == zha.ZHA_ERR_BAD_ARG

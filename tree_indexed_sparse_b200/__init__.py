@@ -27,6 +27,7 @@ ZHA_BF16 = 1
 
 # every symbol include/zha.h declares
 EXPORTS = ["zha_workspace_bytes", "zha_create", "zha_destroy", "zha_build", "zha_append", "zha_decode",
+           "zha_decode_batch",
            "zha_dense_decode", "zha_dense_decode_static", "zha_device_status", "zha_set_phase_timer",
            "zha_set_wait_budget", "zha_depth", "zha_n_tokens", "zha_summary_layout", "zha_router_layout",
            "zha_strerror"]
@@ -43,7 +44,7 @@ class zha_config(ctypes.Structure):
                 ("R", ctypes.c_int32), ("c", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("kv_dtype", ctypes.c_int32), ("max_depth", ctypes.c_int32),
                 ("capacity_tokens", ctypes.c_int64), ("router_dtype", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("max_batch", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -64,6 +65,8 @@ def _load() -> ctypes.CDLL:
     lib.zha_append.restype = ctypes.c_int
     lib.zha_decode.argtypes = [P, P, F, P, P, I32, P, P, P, P, I32, P]
     lib.zha_decode.restype = ctypes.c_int
+    lib.zha_decode_batch.argtypes = [P, P, I32, F, P, P, I32, P, P, P, P, I32, P]
+    lib.zha_decode_batch.restype = ctypes.c_int
     lib.zha_dense_decode.argtypes = [P, P, P, P]
     lib.zha_dense_decode.restype = ctypes.c_int
     lib.zha_dense_decode_static.argtypes = [CFG, P, P, I64, P, P, P, P]
@@ -142,6 +145,14 @@ def zha_decode(ctx, d_q, p: float, d_out, d_leaf_idx=None, leaf_cap: int = 0, d_
                           _vp(stream)), "zha_decode")
 
 
+def zha_decode_batch(ctx, d_q, n_q: int, p: float, d_out, d_leaf_idx=None, leaf_cap: int = 0, d_n_leaf=None,
+                     d_nodes_visited=None, d_trace_ids=None, d_trace_counts=None, trace_cap: int = 0,
+                     stream=None) -> None:
+    _check(lib.zha_decode_batch(ctx, _vp(d_q), int(n_q), float(p), _vp(d_out), _vp(d_leaf_idx), int(leaf_cap),
+                                _vp(d_n_leaf), _vp(d_nodes_visited), _vp(d_trace_ids), _vp(d_trace_counts),
+                                int(trace_cap), _vp(stream)), "zha_decode_batch")
+
+
 def zha_dense_decode(ctx, d_q, d_out, stream=None) -> None:
     _check(lib.zha_dense_decode(ctx, _vp(d_q), _vp(d_out), _vp(stream)), "zha_dense_decode")
 
@@ -200,10 +211,11 @@ class ZhaCache:
     """
 
     def __init__(self, h_kv: int, h_q: int, d: int, R: int, c: int, D: int, kv_dtype: int,
-                 capacity_tokens: int, device="cuda", max_depth: int = 0, router_dtype: int = ZHA_F32):
+                 capacity_tokens: int, device="cuda", max_depth: int = 0, router_dtype: int = ZHA_F32,
+                 max_batch: int = 1):
         import torch
 
-        self.cfg = zha_config(h_kv, h_q, d, R, c, D, kv_dtype, max_depth, capacity_tokens, router_dtype, 0)
+        self.cfg = zha_config(h_kv, h_q, d, R, c, D, kv_dtype, max_depth, capacity_tokens, router_dtype, max_batch)
         nbytes = zha_workspace_bytes(self.cfg)
         if nbytes < 0:
             raise ZhaError(nbytes, "zha_workspace_bytes")
@@ -265,6 +277,31 @@ class ZhaCache:
             tcnt = res["trace_counts"] = torch.zeros(D, h_q, dtype=torch.int32, device=dev)
         zha_decode(self.ctx, q, p, res["out"], res["leaf_idx"], leaf_cap, res["n_leaf"], res["visited"],
                    tid, tcnt, trace_cap, self._stream(stream))
+        return res
+
+    def decode_batch(self, qs, p: float, leaf_cap: int | None = None, trace_cap: int = 0, stream=None, out=None):
+        """Decode n_q queries qs [n_q, h_q, d] in one launch.  Returns a dict of
+        device tensors: out [n_q, h_q, d], leaf_idx [n_q, h_q, leaf_cap],
+        n_leaf and visited [n_q, h_q] (+ trace_ids [D, n_q * h_q, trace_cap]
+        and trace_counts [D, n_q * h_q] when trace_cap > 0)."""
+        import torch
+
+        n_q, h_q, D = qs.shape[0], self.cfg.h_q, self.depth
+        dev = self.device
+        if leaf_cap is None:
+            leaf_cap = -(-self.n_tokens // self.cfg.c)
+        res = {
+            "out": out if out is not None else torch.empty(n_q, h_q, self.cfg.d, dtype=torch.float32, device=dev),
+            "leaf_idx": torch.empty(n_q, h_q, max(leaf_cap, 1), dtype=torch.int32, device=dev),
+            "n_leaf": torch.empty(n_q, h_q, dtype=torch.int32, device=dev),
+            "visited": torch.empty(n_q, h_q, dtype=torch.int64, device=dev),
+        }
+        tid = tcnt = None
+        if trace_cap > 0:
+            tid = res["trace_ids"] = torch.full((D, n_q * h_q, trace_cap), -1, dtype=torch.int32, device=dev)
+            tcnt = res["trace_counts"] = torch.zeros(D, n_q * h_q, dtype=torch.int32, device=dev)
+        zha_decode_batch(self.ctx, qs, n_q, p, res["out"], res["leaf_idx"], leaf_cap, res["n_leaf"], res["visited"],
+                         tid, tcnt, trace_cap, self._stream(stream))
         return res
 
     def dense(self, q, out=None, stream=None):

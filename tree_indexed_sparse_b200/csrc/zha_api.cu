@@ -55,7 +55,9 @@ int check_config(const zha_config *cfg) {
     if (cfg->kv_dtype != ZHA_F32 && cfg->kv_dtype != ZHA_BF16) return ZHA_ERR_BAD_ARG;
     if (cfg->capacity_tokens < 1 || cfg->capacity_tokens > (int64_t)0x7fffffff) return ZHA_ERR_BAD_ARG;
     if (cfg->max_depth != 0 && (cfg->max_depth <= cfg->D || cfg->max_depth > MAXD)) return ZHA_ERR_BAD_ARG;
-    if ((cfg->router_dtype != ZHA_F32 && cfg->router_dtype != ZHA_BF16) || cfg->reserved != 0) return ZHA_ERR_BAD_ARG;
+    if (cfg->router_dtype != ZHA_F32 && cfg->router_dtype != ZHA_BF16) return ZHA_ERR_BAD_ARG;
+    if (cfg->max_batch < 0 || (int64_t)cfg->h_kv * (cfg->max_batch > 1 ? cfg->max_batch : 1) > 64)
+        return ZHA_ERR_BAD_ARG;
     const int G = cfg->h_q / cfg->h_kv;
     if (!compiled_combo(cfg->kv_dtype, cfg->d, cfg->R, G, cfg->router_dtype)) return ZHA_ERR_UNSUPPORTED;
     return ZHA_OK;
@@ -83,9 +85,13 @@ int depth_for(int64_t n, int c, int D0, int Dmax) {
     return D;
 }
 
+// Queries one decode call may carry (zha_decode_batch).
+int max_batch(const zha_config *cfg) { return cfg->max_batch > 1 ? cfg->max_batch : 1; }
+
 void make_layout(const zha_config *cfg, Layout *L) {
     const int G = cfg->h_q / cfg->h_kv;
-    const int64_t H = cfg->h_kv;
+    const int64_t H = cfg->h_kv;                        // summary store: per KV head
+    const int64_t HV = (int64_t)cfg->h_kv * max_batch(cfg);  // decode scratch: per (query, KV head)
     const int DL = max_levels(cfg);
     int64_t off = 0;
     for (int l = 1; l <= DL; ++l) {
@@ -116,32 +122,32 @@ void make_layout(const zha_config *cfg, Layout *L) {
     L->scratch_off = off;
     for (int l = 1; l <= DL; ++l) {
         L->kid_off[l - 1] = off;
-        off = align256(off + H * L->slot_cap[l - 1] * 4);
+        off = align256(off + HV * L->slot_cap[l - 1] * 4);
         L->kmask_off[l - 1] = off;
-        off = align256(off + H * L->slot_cap[l - 1]);
+        off = align256(off + HV * L->slot_cap[l - 1]);
     }
     auto take = [&](int64_t &at, int64_t bytes) {
         at = off;
         off = align256(off + bytes);
     };
-    take(L->seg_off, (int64_t)MAXD * H * SEG_CAP * 4);
-    take(L->hseg_off, (int64_t)MAXD * H * SEG_CAP * G * 4);
-    take(L->lvl_off, (int64_t)MAXD * H * 2 * 4);
-    take(L->rdsc_off, H * 2 * LOC_CAP * G * 4);
-    take(L->scores_off, H * sc * G * 4);
-    take(L->snode_off, H * sc * 4);
-    take(L->skeep_off, H * sc + 4);
-    take(L->tmax_off, H * SEG_CAP * G * 4);
-    take(L->tcnt_off, H * SEG_CAP * G * 4);
-    take(L->tsum_off, H * SEG_CAP * G * 8);
-    take(L->hcnt_off, H * HIST_ROUNDS * G * NB * 4);
-    take(L->hmass_off, H * HIST_ROUNDS * G * NB * 8);
-    take(L->cw_off, H * G * CAND_MAX * 8);
-    take(L->cs_off, H * G * CAND_MAX * 4);
-    take(L->ccnt_off, H * G * 4);
-    take(L->ticket_off, H * 4);
-    take(L->part_off, (int64_t)PART_CAP * H * G * (cfg->d + 4) * 4);
-    take(L->sync_off, (H + 3) * 4);
+    take(L->seg_off, (int64_t)MAXD * HV * SEG_CAP * 4);
+    take(L->hseg_off, (int64_t)MAXD * HV * SEG_CAP * G * 4);
+    take(L->lvl_off, (int64_t)MAXD * HV * 2 * 4);
+    take(L->rdsc_off, HV * 2 * LOC_CAP * G * 4);
+    take(L->scores_off, HV * sc * G * 4);
+    take(L->snode_off, HV * sc * 4);
+    take(L->skeep_off, HV * sc + 4);
+    take(L->tmax_off, HV * SEG_CAP * G * 4);
+    take(L->tcnt_off, HV * SEG_CAP * G * 4);
+    take(L->tsum_off, HV * SEG_CAP * G * 8);
+    take(L->hcnt_off, HV * HIST_ROUNDS * G * NB * 4);
+    take(L->hmass_off, HV * HIST_ROUNDS * G * NB * 8);
+    take(L->cw_off, HV * G * CAND_MAX * 8);
+    take(L->cs_off, HV * G * CAND_MAX * 4);
+    take(L->ccnt_off, HV * G * 4);
+    take(L->ticket_off, HV * 4);
+    take(L->part_off, (int64_t)PART_CAP * HV * G * (cfg->d + 4) * 4);
+    take(L->sync_off, (HV + 3) * 4);
     take(L->status_off, 4);
     L->total = off;
 }
@@ -159,6 +165,7 @@ void fill_tree_levels(zha_ctx *ctx) {
 Decode make_decode(zha_ctx *ctx) {
     Decode dc = ctx->scratch;
     dc.t = ctx->t;
+    dc.nvk = ctx->t.h_kv;
     dc.phase_ns = ctx->phase_ns;
     dc.wait_budget = ctx->wait_budget;
     return dc;
@@ -262,9 +269,7 @@ int zha_create(const zha_config *cfg, void *d_workspace, int64_t ws_bytes, zha_c
             delete ctx;
             return ZHA_ERR_CUDA;
         }
-        int n = std::min(ctx->n_sm, PART_CAP);
-        n = std::max(1, n / cfg->h_kv) * cfg->h_kv;
-        ctx->decode_cta = n;
+        ctx->decode_cta = std::min(ctx->n_sm, PART_CAP);  // rounded to a multiple of the teams per call
     }
     if (cudaMemset(ctx->scratch_begin, 0, (size_t)ctx->scratch_bytes) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess) {
@@ -323,12 +328,21 @@ int zha_append(zha_ctx *ctx, const void *d_k, const void *d_v, void *stream) {
 int zha_decode(zha_ctx *ctx, const float *d_q, float p, float *d_out, int32_t *d_leaf_idx, int32_t leaf_cap,
                int32_t *d_n_leaf, int64_t *d_nodes_visited, int32_t *d_trace_ids, int32_t *d_trace_counts,
                int32_t trace_cap, void *stream) {
+    return zha_decode_batch(ctx, d_q, 1, p, d_out, d_leaf_idx, leaf_cap, d_n_leaf, d_nodes_visited, d_trace_ids,
+                            d_trace_counts, trace_cap, stream);
+}
+
+int zha_decode_batch(zha_ctx *ctx, const float *d_q, int32_t n_q, float p, float *d_out, int32_t *d_leaf_idx,
+                     int32_t leaf_cap, int32_t *d_n_leaf, int64_t *d_nodes_visited, int32_t *d_trace_ids,
+                     int32_t *d_trace_counts, int32_t trace_cap, void *stream) {
     if (!ctx || !d_q || !d_out) return ZHA_ERR_BAD_ARG;
+    if (n_q < 1 || n_q > max_batch(&ctx->cfg)) return ZHA_ERR_BAD_ARG;
     if (!ctx->built) return ZHA_ERR_NOT_BUILT;
     if (!(p > 0.f) || std::isnan(p)) return ZHA_ERR_BAD_ARG;
     if ((d_leaf_idx && leaf_cap < 0) || (d_trace_ids && (!d_trace_counts || trace_cap < 0))) return ZHA_ERR_BAD_ARG;
     if ((reinterpret_cast<uintptr_t>(d_q) | reinterpret_cast<uintptr_t>(d_out)) & 15u) return ZHA_ERR_BAD_ARG;
     Decode dc = make_decode(ctx);
+    dc.nvk = n_q * ctx->t.h_kv;
     dc.q = d_q;
     dc.p = p;
     dc.out = d_out;
@@ -339,7 +353,11 @@ int zha_decode(zha_ctx *ctx, const float *d_q, float p, float *d_out, int32_t *d
     dc.trace_ids = d_trace_ids;
     dc.trace_cnt = d_trace_ids ? d_trace_counts : nullptr;
     dc.trace_cap = d_trace_ids ? trace_cap : 0;
-    if (launch_decode(dc, ctx->decode_cta, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZHA_ERR_CUDA;
+    // one team of CTAs per (query, KV head): the grid is the largest
+    // multiple of that count within one CTA per SM
+    const int n_cta = std::max(1, ctx->decode_cta / dc.nvk) * dc.nvk;
+    if (n_cta > std::min(ctx->n_sm, PART_CAP)) return ZHA_ERR_UNSUPPORTED;
+    if (launch_decode(dc, n_cta, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ZHA_ERR_CUDA;
     return ZHA_OK;
 }
 

@@ -13,7 +13,7 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_dense(const __grid_constant__ 
     __shared__ StageMap map;
     __shared__ int s_last[64];
     const int warp = threadIdx.x >> 5;
-    const int h_kv = a.t.h_kv, nb = gridDim.x, b = blockIdx.x;
+    const int h_kv = a.nvk, nb = gridDim.x, b = blockIdx.x;
     stage_map_init<true, StageCfg<KT, HD>::TT>(a, map);
     attn_stages<KT, HD, G, true>(a, map, smem, b, nb);
     __threadfence();

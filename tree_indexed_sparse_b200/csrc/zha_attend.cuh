@@ -497,7 +497,7 @@ struct StageMap {
 // the __syncthreads inside.  Gather: the level-1 segments written by routing.
 template <bool DENSE, int TT>
 __device__ void stage_map_init(const Decode &a, StageMap &map) {
-    const int h_kv = a.t.h_kv;
+    const int h_kv = a.nvk;  // virtual KV heads
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if ((int)threadIdx.x < h_kv) {  // level 1's team and frontier sizes, in parallel
         const int kh = threadIdx.x;
@@ -561,7 +561,7 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
     using SM = ASmem<KT, HD, G>;
     constexpr int ST = C::STAGES, RB = C::RB, GR = C::GR, TT = C::TT;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int h_kv = a.t.h_kv, c = a.t.c, clog = a.t.c_log2;
+    const int h_kv = a.nvk, c = a.t.c, clog = a.t.c_log2;  // virtual KV heads
     uint8_t *meta = smem + SM::off_meta;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + SM::off_bar);
     uint64_t *empty = full + ST;
@@ -609,8 +609,9 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                 *abort = 1;
                 break;
             }
-            const unsigned char *Kh = reinterpret_cast<const unsigned char *>(a.t.K) + (int64_t)kh * a.t.kv_cap * RB;
-            const unsigned char *Vh = reinterpret_cast<const unsigned char *>(a.t.V) + (int64_t)kh * a.t.kv_cap * RB;
+            const int pk = kh % a.t.h_kv;  // physical KV head
+            const unsigned char *Kh = reinterpret_cast<const unsigned char *>(a.t.K) + (int64_t)pk * a.t.kv_cap * RB;
+            const unsigned char *Vh = reinterpret_cast<const unsigned char *>(a.t.V) + (int64_t)pk * a.t.kv_cap * RB;
             unsigned char *sK = smem + (size_t)slot * C::STAGE_BYTES;
             uint8_t *mt = meta + slot * TT;
             const int t0 = st * TT;
@@ -805,9 +806,9 @@ __device__ __noinline__ void combine_kvh(const Decode &a, const StageMap &map, i
     float4 *racc = reinterpret_cast<float4 *>(sm);  // [GT] part columns
     float *rml = sm + 4 * GT;                          // [GT] part max, [GT] part sum
     float *hs0 = rml + 2 * GT;                         // [G] sink scores
-    const int h_kv = a.t.h_kv;
-    const KT *Kh = reinterpret_cast<const KT *>(a.t.K) + (int64_t)kh * a.t.kv_cap * HD;
-    const KT *Vh = reinterpret_cast<const KT *>(a.t.V) + (int64_t)kh * a.t.kv_cap * HD;
+    const int h_kv = a.nvk;
+    const KT *Kh = reinterpret_cast<const KT *>(a.t.K) + (int64_t)(kh % a.t.h_kv) * a.t.kv_cap * HD;
+    const KT *Vh = reinterpret_cast<const KT *>(a.t.V) + (int64_t)(kh % a.t.h_kv) * a.t.kv_cap * HD;
     if (warp < G) {
         // sink score of head `warp` (-inf when it is not added)
         const int h = warp;

@@ -66,7 +66,7 @@ __device__ __noinline__ void write_lists(const Decode &a, int kh, int tr) {
             if (leaf && a.n_leaf) a.n_leaf[hq] = (int32_t)total;
             if (leaf && a.leaf_idx && total > (uint32_t)a.leaf_cap) set_status(a.status, ZHA_CAPACITY_CODE);
             if (tr_on) {
-                a.trace_cnt[(int64_t)(l - 1) * a.t.h_q + hq] = (int32_t)total;
+                a.trace_cnt[(int64_t)(l - 1) * a.nvk * G + hq] = (int32_t)total;
                 if (total > (uint32_t)a.trace_cap) set_status(a.status, ZHA_CAPACITY_CODE);
             }
         }
@@ -85,7 +85,7 @@ __device__ __noinline__ void write_lists(const Decode &a, int kh, int tr) {
                 const int32_t id = __ldcg(ids + i);
                 if (leaf && a.leaf_idx && p < (uint32_t)a.leaf_cap) a.leaf_idx[(int64_t)hq * a.leaf_cap + p] = id;
                 if (tr_on && p < (uint32_t)a.trace_cap)
-                    a.trace_ids[((int64_t)(l - 1) * a.t.h_q + hq) * a.trace_cap + p] = id;
+                    a.trace_ids[((int64_t)(l - 1) * a.nvk * G + hq) * a.trace_cap + p] = id;
             }
             pos += __popc(bal);
         }
@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(A_THREADS, 1) k_decode(const __grid_constant__
     __shared__ int s_last[64];
     const int warp = threadIdx.x >> 5;
     const int nb = gridDim.x, b = blockIdx.x;
-    const int h_kv = a.t.h_kv;
+    const int h_kv = a.nvk;     // virtual KV heads: one team each
     const int nbk = nb / h_kv;  // CTAs per KV head team
     unsigned *words = a.sync;
     unsigned *abortw = words + h_kv + 2;

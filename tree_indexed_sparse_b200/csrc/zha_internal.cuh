@@ -44,7 +44,10 @@ struct Tree {
 // kept nodes in ascending id order.
 struct Decode {
     Tree t;
-    const float *q;               // [h_q][d]
+    int nvk;                      // virtual KV heads: (query of the batch, KV head) pairs, n_q * h_kv;
+                                  // virtual head v routes query v / h_kv against KV head v % h_kv, and
+                                  // every scratch array, team and output is indexed by v
+    const float *q;               // [n_q][h_q][d] = [nvk][G][d]
     float p;
     int32_t *kept_ids[MAXD];      // [h_kv][slot_cap[l-1]] kept node ids (segments)
     uint8_t *kept_mask[MAXD];     // [h_kv][slot_cap[l-1]] heads that kept the node

@@ -48,6 +48,10 @@
 // level on little data, so cold instruction fetch dominates unless the code is
 // short.  Loops that are not hot are kept rolled.
 //
+// `kh` below is a virtual KV head (Decode::nvk): a query of the batch paired
+// with a KV head.  Scratch, teams and lists are indexed by it; summaries are
+// read from its physical KV head, kh % h_kv.
+//
 // Every function here is called by threads 0-255 of a CTA (warps 0-7) and
 // synchronises them with the named barrier of gsync().
 #pragma once
@@ -161,13 +165,13 @@ struct TeamSync {
 // ---- level bookkeeping ---------------------------------------------------
 
 __device__ __forceinline__ uint32_t *seg_ptr(const Decode &a, int l, int kh) {
-    return a.seg + ((int64_t)(l - 1) * a.t.h_kv + kh) * SEG_CAP;
+    return a.seg + ((int64_t)(l - 1) * a.nvk + kh) * SEG_CAP;
 }
 __device__ __forceinline__ uint32_t *hseg_ptr(const Decode &a, int l, int kh) {
-    return a.hseg + ((int64_t)(l - 1) * a.t.h_kv + kh) * SEG_CAP * a.t.G;
+    return a.hseg + ((int64_t)(l - 1) * a.nvk + kh) * SEG_CAP * a.t.G;
 }
 __device__ __forceinline__ int32_t *lvl_ptr(const Decode &a, int l, int kh) {
-    return a.lvl + ((int64_t)(l - 1) * a.t.h_kv + kh) * 2;
+    return a.lvl + ((int64_t)(l - 1) * a.nvk + kh) * 2;
 }
 // First slot of team rank r's range of a level with S slots and T ranks.
 __device__ __forceinline__ int64_t seg_start(int64_t S, int T, int r) { return S * r / T; }
@@ -398,8 +402,9 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         for (int e = 0; e < VEC; ++e) qs[h][e] *= a.t.scale;
     }
     const int64_t cap = a.t.node_cap[l - 1];
-    const RT *gb = router_g<RT>(a.t, l) + (int64_t)kh * cap * R * HD;
-    const float *bb = router_b<RT>(a.t, l) + (int64_t)kh * cap * R;
+    const int pk = kh % a.t.h_kv;  // the physical KV head of virtual head kh
+    const RT *gb = router_g<RT>(a.t, l) + (int64_t)pk * cap * R * HD;
+    const float *bb = router_b<RT>(a.t, l) + (int64_t)pk * cap * R;
     const int c = a.t.c, clog = a.t.c_log2;
     const int32_t nl = a.t.n_level[l - 1];
     const int64_t nu = (c1 - c0 + C::SLOTS - 1) / C::SLOTS;  // units

@@ -110,6 +110,7 @@ int zha_dense_decode_static(const zha_config *cfg, const void *d_K, const void *
     t.K = d_K;
     t.V = d_V;
     t.scale = (float)(1.0 / std::sqrt((double)cfg->d));
+    dc.nvk = cfg->h_kv;
     dc.q = d_q;
     dc.out = d_out;
     dc.part = reinterpret_cast<float *>(ds.ptr);
