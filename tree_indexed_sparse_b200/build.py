@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libzha.so")
 SOURCES = ["zha_build.cu", "zha_decode.cu", "zha_attend.cu", "zha_api.cu", "zha_static.cu"]
-HEADERS = ["zha_attr.h", "zha_device.cuh", "zha_internal.cuh", "zha_tma.cuh", "zha_sync.cuh", "zha_route.cuh", "zha_attend.cuh", os.path.join("..", "..", "include", "zha.h")]
+HEADERS = ["zha_attr.h", "zha_mma.cuh", "zha_build_mma.cuh", "zha_device.cuh", "zha_internal.cuh", "zha_tma.cuh", "zha_sync.cuh", "zha_route.cuh", "zha_attend.cuh", os.path.join("..", "..", "include", "zha.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -24,6 +24,7 @@
 
 #include <algorithm>
 
+#include "zha_build_mma.cuh"
 #include "zha_device.cuh"
 #include "zha_internal.cuh"
 #include "zha_tma.cuh"
@@ -513,7 +514,25 @@ __global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict_
     unsigned char *stg = reinterpret_cast<unsigned char *>(bsm + R * (t.c > 32 ? t.c : 32));
     const int64_t stage_cap = append_stage_bytes<KT, HD, R>(t.c, t.D);
     int64_t n = pos / t.c;
-    {
+    bool leaf_done = false;
+    if constexpr (sizeof(KT) == 2 && R == LM_R) {
+        if (leaf_mma_applies(t.kv_dtype, HD, R, t.c)) {
+            // the leaf's unit, recomputed as the tensor-core build does it
+            unsigned char *lm = stg + stage_cap;
+            const int passes = leaf_mma_load_ref<HD>(t.ref + (int64_t)kh * R * HD, lm);
+            if (j == 0) {
+                const int U = leaf_mma_unit_tokens(t.c);
+                const int64_t u = pos / U;
+                const uint16_t *Kb = reinterpret_cast<const uint16_t *>(Kh);
+                TileRegs<HD> nxt;
+                tile_load<HD>(Kb, u * U, t.n_tokens, nxt, lane);
+                leaf_mma_unit<HD>(t, kh, u, lm, reinterpret_cast<uint16_t *>(lm + LeafMma<HD>::off_k), passes, nxt,
+                                  -1, lane);
+            }
+            leaf_done = true;
+        }
+    }
+    if (!leaf_done) {
         const int64_t tok0 = n * t.c;
         const int ntok = (int)(t.n_tokens - tok0);
         const int64_t nc = t.node_cap[0];
@@ -559,16 +578,37 @@ __global__ void __launch_bounds__(32 * R) k_append(Tree t, const KT *__restrict_
 template <typename KT, int HD, int R>
 static cudaError_t build_impl(const Tree &t, cudaStream_t s, int n_sm) {
     const int warps = BUILD_THREADS / 32;
-    const int tt = leaf_tile_tokens(t.c, R);
-    size_t smem = (size_t)warps * (tt * R + (tt / t.c + 1) * R) * sizeof(float);
     static PerDeviceMax<> leaf_attr, parent_attr;
-    cudaError_t err = allow_smem(k_build_leaves<KT, HD, R>, smem, leaf_attr);
-    if (err != cudaSuccess) return err;
-    const int64_t tiles = ((t.n_tokens + tt - 1) / tt) * t.h_kv;
-    int grid = (int)std::min<int64_t>((tiles + warps - 1) / warps, (int64_t)n_sm * 8);
-    k_build_leaves<KT, HD, R><<<grid, BUILD_THREADS, smem, s>>>(t);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
+    cudaError_t err;
+    bool leaves_done = false;
+    if constexpr (sizeof(KT) == 2 && R == LM_R) {
+        if (leaf_mma_applies(t.kv_dtype, HD, R, t.c)) {
+            // bf16 cache, 16 reference queries: leaves on the tensor cores
+            static PerDeviceMax<> mma_attr;
+            const size_t smem = LeafMma<HD>::bytes(LM_WARPS);
+            err = allow_smem(k_build_leaves_mma<HD>, smem, mma_attr);
+            if (err != cudaSuccess) return err;
+            const int U = leaf_mma_unit_tokens(t.c);
+            const int64_t units = (t.n_tokens + U - 1) / U;
+            const int gx = (int)std::max<int64_t>(
+                1, std::min<int64_t>((units + LM_WARPS - 1) / LM_WARPS, std::max(1, n_sm * 4 / t.h_kv)));
+            k_build_leaves_mma<HD><<<dim3(gx, t.h_kv), LM_WARPS * 32, smem, s>>>(t);
+            err = cudaGetLastError();
+            if (err != cudaSuccess) return err;
+            leaves_done = true;
+        }
+    }
+    if (!leaves_done) {
+        const int tt = leaf_tile_tokens(t.c, R);
+        size_t smem = (size_t)warps * (tt * R + (tt / t.c + 1) * R) * sizeof(float);
+        err = allow_smem(k_build_leaves<KT, HD, R>, smem, leaf_attr);
+        if (err != cudaSuccess) return err;
+        const int64_t tiles = ((t.n_tokens + tt - 1) / tt) * t.h_kv;
+        int grid = (int)std::min<int64_t>((tiles + warps - 1) / warps, (int64_t)n_sm * 8);
+        k_build_leaves<KT, HD, R><<<grid, BUILD_THREADS, smem, s>>>(t);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
     size_t psmem = (size_t)warps * (t.c * R + R) * sizeof(float);
     err = allow_smem(k_build_parents<HD, R>, psmem, parent_attr);
     if (err != cudaSuccess) return err;
@@ -606,6 +646,8 @@ static cudaError_t append_impl(const Tree &t, const void *k, const void *v, cuda
     // per plane warp: one score per token of a leaf, or one estimate per child
     size_t smem = (size_t)R * (t.c > 32 ? t.c : 32) * sizeof(float);
     smem += (size_t)append_stage_bytes<KT, HD, R>(t.c, t.D);  // the shared copy of the rows every plane reads
+    if (sizeof(KT) == 2 && R == LM_R && leaf_mma_applies(t.kv_dtype, HD, R, t.c))
+        smem += LeafMma<HD>::bytes(1);  // the tensor-core leaf of one warp
     static PerDeviceMax<> attr;
     const cudaError_t err = allow_smem(k_append<KT, HD, R>, smem, attr);
     if (err != cudaSuccess) return err;
