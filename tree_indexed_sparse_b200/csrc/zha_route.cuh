@@ -1370,9 +1370,16 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
     }
     int32_t *pid = reinterpret_cast<int32_t *>(smem + SM::off_pid);
     uint8_t *pmk = smem + SM::off_pmk;
+    // slots scored per pipeline run: the local arrays' capacity, or, when
+    // they spill to global memory anyway, as many as one parent window covers
+    // (the whole slice when the parents are the local kept list): fewer runs
+    // drain the copy pipeline fewer times
+    const int64_t chunk = L.n <= LOC_CAP ? (int64_t)LOC_CAP
+                          : (par_local || L.top) ? L.n
+                                                 : max((int64_t)LOC_CAP, (int64_t)(PAR_CAP - 2) * a.t.c);
 #pragma unroll 1
-    for (int64_t c0 = L.s0; c0 < L.s0 + L.n; c0 += LOC_CAP) {
-        const int64_t c1 = min(L.s0 + L.n, c0 + LOC_CAP);
+    for (int64_t c0 = L.s0; c0 < L.s0 + L.n; c0 += chunk) {
+        const int64_t c1 = min(L.s0 + L.n, c0 + chunk);
         int64_t k0 = 0;  // parents already local: the whole kept list from rank 0
         if (!L.top && !par_local) load_parents(a, L, c0, c1, pref, pid, pmk, k0);
         gsync();
