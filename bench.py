@@ -772,6 +772,45 @@ def run_crossover(args, local):
                        "l2": "256 MiB written before every call"}}
 
 
+def record_traffic(csv_path: str, steps_path: str, launch: int) -> None:
+    """Write profiles/k_decode_traffic.json from one ncu capture: the DRAM
+    bytes (read + write) of k_decode launch `launch` (0-based, the first
+    traced pass of this script runs the decodes in step order) from the ncu
+    CSV, next to that launch's algorithmic bytes from the ZHA_STEP_BYTES file
+    of the same command, under the hash of the kernel sources they were
+    taken on."""
+    import csv
+
+    rows = list(csv.reader(open(csv_path)))
+    hdr = next(i for i, r in enumerate(rows) if "Metric Name" in r)
+    cols = rows[hdr]
+    name_i, metric_i, value_i = cols.index("Kernel Name"), cols.index("Metric Name"), cols.index("Metric Value")
+    unit_i = cols.index("Metric Unit")
+    scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "ns": 1e-3, "usecond": 1.0, "us": 1.0,
+             "msecond": 1e3, "ms": 1e3}
+    vals = {}  # bytes, or microseconds for the duration
+    for r in rows[hdr + 1:]:
+        if len(r) > value_i and "k_decode" in r[name_i]:
+            vals[r[metric_i]] = float(r[value_i].replace(",", "")) * scale.get(r[unit_i], 1.0)
+    dram = vals["dram__bytes_read.sum"] + vals["dram__bytes_write.sum"]
+    steps = json.load(open(steps_path))
+    algo = steps["decode_bytes"][launch]
+    path = os.path.join(ROOT, "profiles", "k_decode_traffic.json")
+    try:
+        rec = json.load(open(path))
+    except (OSError, ValueError):
+        rec = {}
+    if rec.get("source_hash") != kernel_source_hash():
+        rec = {"source_hash": kernel_source_hash(), "workloads": {}, "not_captured": rec.get("not_captured", {})}
+    rec["not_captured"]["extreme_10m"] = ("not captured: its cache holds about 24 GB on the device, above the size "
+                                          "at which a counter capture may run on this pool")
+    rec["workloads"][steps["workload"]] = {"launch": launch, "dram_bytes": dram, "algorithmic_bytes": algo,
+                                           "ncu_duration_us": vals.get("gpu__time_duration.sum")}
+    with open(path, "w") as f:
+        json.dump(rec, f, indent=1)
+    print(json.dumps(rec["workloads"][steps["workload"]]))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -789,7 +828,12 @@ def main():
                     help="summaries the routing reads: fp32 (default) or the bf16 router copy")
     ap.add_argument("--growth", action="store_true",
                     help="time the step where a tree with room to grow adds a level (light settings, 2M tokens)")
+    ap.add_argument("--record-traffic", nargs=3, metavar=("NCU_CSV", "STEP_BYTES_JSON", "LAUNCH"),
+                    help="write profiles/k_decode_traffic.json from an ncu capture of k_decode (no GPU needed)")
     args = ap.parse_args()
+    if args.record_traffic:
+        record_traffic(args.record_traffic[0], args.record_traffic[1], int(args.record_traffic[2]))
+        return
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_setup(args.gpus)
     if args.crossover or args.growth:
