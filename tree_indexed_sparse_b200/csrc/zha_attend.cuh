@@ -411,6 +411,20 @@ __device__ __noinline__ void merge_partials(const float *merge, float *dst, int 
     gsync();
 }
 
+// Head masks of `n` consecutive stage rows: mk for the first `valid`, 0 after.
+__device__ __forceinline__ void mask_rows(uint8_t *mt, uint32_t mk, int valid, int n) {
+    if ((n & 3) == 0) {
+        for (int w = 0; w < n; w += 4) {
+            uint32_t v = 0u;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) v |= (w + b < valid ? mk : 0u) << (8 * b);
+            *reinterpret_cast<uint32_t *>(mt + w) = v;
+        }
+    } else {
+        for (int w = 0; w < n; ++w) mt[w] = (uint8_t)(w < valid ? mk : 0u);
+    }
+}
+
 // x / c for token positions (< 2^32): a shift when c is a power of two.
 __device__ __forceinline__ uint32_t div_c(uint32_t x, int c, int clog) {
     return clog >= 0 ? (x >> clog) : x / (uint32_t)c;
@@ -567,32 +581,51 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
         map.locate(u0, kh, st64);
         int st = (int)st64;
         // lane gi < 8: K rows of group gi; lane 8 + gi: V rows of group gi
+        // (fast = 0); fast = 1: a group never spans two leaves; fast = 2:
+        // whole leaves tile each group (GR / c of them, a power of two) and
+        // a stage holds at most 32 leaves
+        const int fast = DENSE ? 0 : (c % GR == 0 ? 1 : (GR % c == 0 && TT / c <= 32 ? 2 : 0));
+        const int lps = fast == 2 ? TT / c : 0;      // leaves per stage
+        const int nlm = fast == 2 ? GR / c - 1 : 0;  // leaves per group - 1
         const int gi = lane & 7;
         const bool act = lane < 16;
         const bool isV = lane >= 8;
+        // per KV head: its rows, kept leaves and last stage of this CTA
+        int jnext = 0, L = 0;
+        const unsigned char *Kh = nullptr, *Vh = nullptr;
+        auto enter_head = [&]() {
+            const int pk = kh % a.t.h_kv;  // physical KV head
+            Kh = reinterpret_cast<const unsigned char *>(a.t.K) + (int64_t)pk * a.t.kv_cap * RB;
+            Vh = reinterpret_cast<const unsigned char *>(a.t.V) + (int64_t)pk * a.t.kv_cap * RB;
+            L = DENSE ? 0 : (int)map.cnt[kh];
+            jnext = (int)(min(u1, map.pref[kh + 1]) - u0);
+        };
+        enter_head();
+        int slot = 0;
+        uint32_t round = 0u;
 #pragma unroll 1
         for (int j = 0; j < n; ++j, ++st) {
-            while (kh + 1 < h_kv && u0 + j >= map.pref[kh + 1]) {
-                ++kh;
+            if (j >= jnext) {
+                while (kh + 1 < h_kv && u0 + j >= map.pref[kh + 1]) ++kh;
                 st = 0;
+                enter_head();
             }
-            const int slot = j % ST;
-            const uint32_t round = (uint32_t)(j / ST);
             if (round > 0 && !mbar_wait(&empty[slot], (round - 1) & 1u, abort)) {
                 set_status(a.status, ZHA_TIMEOUT_CODE);
                 *abort = 1;
                 break;
             }
-            const int pk = kh % a.t.h_kv;  // physical KV head
-            const unsigned char *Kh = reinterpret_cast<const unsigned char *>(a.t.K) + (int64_t)pk * a.t.kv_cap * RB;
-            const unsigned char *Vh = reinterpret_cast<const unsigned char *>(a.t.V) + (int64_t)pk * a.t.kv_cap * RB;
             unsigned char *sK = smem + (size_t)slot * C::STAGE_BYTES;
             uint8_t *mt = meta + slot * TT;
             const int t0 = st * TT;
-            int L = 0;
+            const int cur = slot;
+            if (++slot == ST) {
+                slot = 0;
+                ++round;
+            }
+            int kf = 0;
             if (!DENSE) {
-                L = (int)map.cnt[kh];
-                const int kf = (int)div_c((uint32_t)t0, c, clog);
+                kf = (int)div_c((uint32_t)t0, c, clog);
                 const int kl = min(L - 1, (int)div_c((uint32_t)(t0 + TT - 1), c, clog));
                 if (kh != win_kh || kl >= win_k0 + LEAF_WIN || kf < win_k0) {
                     // refill the window from leaf rank kf up to the last leaf
@@ -602,17 +635,106 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                     const int nwin = min(LEAF_WIN, klast - kf + 1);
                     win_kh = kh;
                     win_k0 = kf;
-                    const int64_t kbase = (int64_t)kh * a.slot_cap[0];
-                    // ranks kf + lane, + 32, ...: the segment only moves forward
+                    const int32_t *kid = a.kept_ids[0] + (int64_t)kh * a.slot_cap[0];
+                    const uint8_t *kmk = a.kept_mask[0] + (int64_t)kh * a.slot_cap[0];
+                    // ranks kf + lane, + 32, ...: the segment only moves
+                    // forward; all of a lane's loads are in flight at once
+                    constexpr int PERL = LEAF_WIN / 32;
                     int rseg = 0;
-#pragma unroll 4
-                    for (int i = lane; i < nwin; i += 32) {
-                        const int64_t at = kbase + map.leaf_at_from(kh, kf + i, rseg);
-                        win_ids[i] = __ldcg(a.kept_ids[0] + at);
-                        win_msk[i] = __ldcg(a.kept_mask[0] + at);
+                    int32_t wid[PERL];
+                    uint32_t wmk[PERL];
+#pragma unroll
+                    for (int t = 0; t < PERL; ++t) {
+                        const int i = lane + 32 * t;
+                        if (i < nwin) {
+                            const int at = (int)map.leaf_at_from(kh, kf + i, rseg);
+                            wid[t] = __ldcg(kid + at);
+                            wmk[t] = __ldcg(kmk + at);
+                        }
+                    }
+#pragma unroll
+                    for (int t = 0; t < PERL; ++t) {
+                        const int i = lane + 32 * t;
+                        if (i < nwin) {
+                            win_ids[i] = wid[t];
+                            win_msk[i] = (uint8_t)wmk[t];
+                        }
                     }
                     __syncwarp();
                 }
+            }
+            if (fast) {
+                // leaves that tile the groups: at most one run per lane, all
+                // lanes at once (the generic path below walks leaves one by one)
+                int rows = 0, row0 = 0, srow = 0;  // the lane's run: rows, first source row, first stage row
+                int own = 0, valid = 0;            // stage rows the lane describes, and how many hold a token
+                if (fast == 1) {
+                    // every group lies inside one leaf: lane g < NG takes group g
+                    if (lane < C::NG) {
+                        const int ug = t0 + lane * GR;
+                        uint32_t mk = 0u;
+                        if (ug < L * c) {
+                            const int k = (int)div_c((uint32_t)ug, c, clog);
+                            mk = win_msk[k - win_k0];
+                            row0 = win_ids[k - win_k0] * c + (ug - k * c);
+                            rows = max(0, min(GR, N - row0));
+                        }
+                        srow = lane * GR;
+                        own = GR;
+                        valid = rows;
+                        mask_rows(mt + srow, mk, valid, own);
+                    }
+                } else {
+                    // lane q takes the stage's leaf q; a run starts at a
+                    // group's first leaf or where the leaf ids stop following
+                    // on (a leaf before another is always whole: only the
+                    // sequence's last leaf can be partial)
+                    const int k = kf + lane;
+                    int id = 0;
+                    uint32_t mk = 0u;
+                    bool cont = false;
+                    if (lane < lps && k < L) {
+                        id = win_ids[k - win_k0];
+                        mk = win_msk[k - win_k0];
+                        valid = min(c, N - id * c);
+                        if ((lane & nlm) != 0) cont = win_ids[k - 1 - win_k0] == id - 1;
+                    }
+                    const uint32_t cm = __ballot_sync(FULL, cont);
+                    // leaves the run takes after its first: the continuing lanes just above
+                    const int e = lane < 31 ? __ffs(~(cm >> (lane + 1))) - 1 : 0;
+                    if (lane < lps) {
+                        if (valid > 0 && !cont) {
+                            row0 = id * c;
+                            rows = min((e + 1) * c, N - row0);
+                        }
+                        srow = lane * c;
+                        own = c;
+                        mask_rows(mt + srow, mk, valid, own);
+                    }
+                }
+                const uint32_t bytes = __reduce_add_sync(FULL, (uint32_t)rows) * (uint32_t)RB;
+                // rows without a token: zeros (see below)
+                if (valid < own) {
+#pragma unroll 1
+                    for (int w = srow + valid; w < srow + own; ++w) {
+                        unsigned char *rk = sK + (w / GR) * C::GS + (w % GR) * RB;
+                        for (int i = 0; i < RB / 16; ++i) {
+                            reinterpret_cast<uint4 *>(rk)[i] = make_uint4(0u, 0u, 0u, 0u);
+                            reinterpret_cast<uint4 *>(rk + C::HALF)[i] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive_expect_tx(&full[cur], 2u * bytes);
+                __syncwarp();
+                if (rows > 0) {
+                    unsigned char *dk = sK + (srow / GR) * C::GS + (srow % GR) * RB;
+                    bulk_g2s_hint(dk, Kh + (size_t)row0 * RB, (uint32_t)(rows * RB), &full[cur], pol);
+                    bulk_g2s_hint(dk + C::HALF, Vh + (size_t)row0 * RB, (uint32_t)(rows * RB), &full[cur], pol);
+                }
+                issued = j + 1;
+                continue;
             }
             // rows of this lane's group: flattened positions ug .. ug + GR - 1
             const int ug = t0 + gi * GR;
@@ -670,11 +792,11 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
+            if (lane == 0) mbar_arrive_expect_tx(&full[cur], bytes);
             __syncwarp();
             if (act && nvalid > 0u) {
                 if (DENSE) {
-                    bulk_g2s_hint(dst, src + (size_t)ug * RB, nvalid * RB, &full[slot], pol);
+                    bulk_g2s_hint(dst, src + (size_t)ug * RB, nvalid * RB, &full[cur], pol);
                 } else {
                     // one copy per run of consecutive rows: adjacent leaves merge
                     int u = ug, k = (int)div_c((uint32_t)ug, c, clog), off = ug - k * c;
@@ -687,7 +809,7 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                         } else {
                             if (run_len > 0)
                                 bulk_g2s_hint(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB),
-                                              &full[slot], pol);
+                                              &full[cur], pol);
                             run_w = u - ug;
                             run_row = r0;
                             run_len = len;
@@ -696,7 +818,7 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                         ++k;
                         off = 0;
                     }
-                    bulk_g2s_hint(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB), &full[slot],
+                    bulk_g2s_hint(dst + run_w * RB, src + (size_t)run_row * RB, (uint32_t)(run_len * RB), &full[cur],
                                   pol);
                 }
             }
