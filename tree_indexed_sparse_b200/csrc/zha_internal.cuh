@@ -11,7 +11,7 @@ namespace zha {
 constexpr int MAXD = 16;          // deepest tree supported
 constexpr int BUILD_THREADS = 256;
 constexpr int NB = 1024;          // top-p buckets per round
-constexpr int CAND_MAX = 1024;    // boundary candidates ranked exactly per head
+constexpr int CAND_MAX = 768;     // boundary candidates ranked exactly per head
 constexpr int SEG_CAP = 256;      // most CTAs in one KV head's team (grid <= 256 CTAs)
 constexpr int HIST_ROUNDS = 3;    // bucket widths 1/32, 1/32768, 1/2^25 of a log-mass unit
 constexpr int LOC_CAP = 2048;     // frontier slots one CTA holds in shared memory

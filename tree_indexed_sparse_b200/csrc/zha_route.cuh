@@ -56,6 +56,8 @@
 // synchronises them with the named barrier of gsync().
 #pragma once
 
+#include <type_traits>
+
 #include "zha_device.cuh"
 #include "zha_internal.cuh"
 #include "zha_sync.cuh"
@@ -108,14 +110,23 @@ struct RouteSmem {
     static constexpr size_t off_keep = off_node + (size_t)LOC_CAP * 4;    // [LOC_CAP] u8
     static constexpr size_t off_u = off_keep + LOC_CAP;                   // union: chunks | cut scratch
     static constexpr size_t off_chunk = off_u;                            // [8 warps][SW_STAGES][SW_BYTES]
-    static constexpr size_t off_hc = off_u;                               // [G][NB] u32
+    // the cut scratch closes the union: the histograms during the rounds,
+    // then the boundary lists in the same bytes (the rounds are over by then)
+    static constexpr size_t hist_bytes = (size_t)G * NB * 12;
+    static constexpr size_t cand_bytes = (size_t)G * CAND_MAX * 16;
+    static constexpr size_t scr_bytes = hist_bytes > cand_bytes ? hist_bytes : cand_bytes;
+    static constexpr size_t u_end = off_u + ((size_t)SW_N * SW_BYTES > scr_bytes ? (size_t)SW_N * SW_BYTES : scr_bytes);
+    static constexpr size_t off_scr = u_end - scr_bytes;
+    static constexpr size_t off_hc = off_scr;                             // [G][NB] u32
     static constexpr size_t off_hm = off_hc + (size_t)G * NB * 4;         // [G][NB] u64 (solo: [SOLO_MAX][G] masses)
-    static constexpr size_t off_cw = off_hm + (size_t)G * NB * 8;         // [G][CAND_MAX] u64
+    static constexpr size_t off_cw = off_scr;                             // [G][CAND_MAX] u64
     static constexpr size_t off_cs = off_cw + (size_t)G * CAND_MAX * 8;   // [G][CAND_MAX] u32
     static constexpr size_t off_own = off_cs + (size_t)G * CAND_MAX * 4;  // [G*CAND_MAX] u32
-    static constexpr size_t u_end = off_own + (size_t)G * CAND_MAX * 4 > off_u + (size_t)SW_N * SW_BYTES
-                                        ? off_own + (size_t)G * CAND_MAX * 4
-                                        : off_u + (size_t)SW_N * SW_BYTES;
+    // A slice that spills (more than LOC_CAP slots) comes back on chip for
+    // its cut when its scores fit below the scratch: the local arrays and
+    // the scoring stages are idle then (its node ids and keep bits stay in
+    // global memory)
+    static constexpr int64_t SPILL_CAP = (int64_t)(off_scr / (G * 4));
     static constexpr size_t off_pid = u_end;                              // [PAR_CAP] i32 parents
     static constexpr size_t off_pmk = off_pid + (size_t)PAR_CAP * 4;      // [PAR_CAP] u8 their head masks
     static constexpr size_t off_pref = (off_pmk + PAR_CAP + 15) / 16 * 16;  // [SEG_CAP + 1] u32
@@ -128,7 +139,9 @@ struct RouteSmem {
     static constexpr size_t off_cnode = off_uses + SW_N * 4;              // [SW_N][SW_ROWS_MAX] i32
     static constexpr size_t off_cmask = off_cnode + (size_t)SW_N * SW_ROWS_MAX * 4;  // [SW_N][SW_ROWS_MAX] u8
     static constexpr size_t off_misc = (off_cmask + (size_t)SW_N * SW_ROWS_MAX + 15) / 16 * 16;  // u32 counters
-    static constexpr size_t bytes = off_misc + 64;
+    static constexpr size_t off_cbar = off_misc + 64;                     // u64: barrier of the scores' return
+    static constexpr size_t off_cuse = off_cbar + 8;                      // u32: its completed phases
+    static constexpr size_t bytes = off_cuse + 8;
     static_assert(SOLO_MAX * G * 8 <= G * NB * 8, "solo masses fit the histogram area");
     static_assert(off_u % 16 == 0, "bulk copies land on 16-byte boundaries");
 };
@@ -141,6 +154,7 @@ struct Level {
     int Tp;                 // team size of the parent level
     int64_t Sp;             // frontier size of the parent level
     float *sc;              // [n][G] local scores (shared memory, or global when n > LOC_CAP)
+    bool sc_local;          // sc is in shared memory
     int32_t *node;          // [n] node of each local slot (-1: no such child)
     uint8_t *keep;          // [n] heads that keep the slot
 };
@@ -297,11 +311,9 @@ __device__ __forceinline__ float stage_issue(const Level &L, int64_t c0, int64_t
         cm[lane] = nd >= 0 ? (uint8_t)mk : 0;
     }
     const uint32_t nvalid = __popc(__ballot_sync(FULL, nd >= 0));
-    if (lane == 0) {
-        // the stage was read through the generic proxy; the copies write it
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(bar, nvalid * (uint32_t)C::NODE_BYTES);
-    }
+    // (the stage's earlier contents were only read, and those reads completed
+    // before the warp got here: a bulk copy may overwrite it without a fence)
+    if (lane == 0) mbar_arrive_expect_tx(bar, nvalid * (uint32_t)C::NODE_BYTES);
     __syncwarp();
     // a run starts where the node does not follow its left neighbour's
     const int left = __shfl_up_sync(FULL, nd, 1);
@@ -351,6 +363,10 @@ __device__ __forceinline__ void stages_init(unsigned char *smem) {
             mbar_init(&bars[st], 1);
             uses[st] = 0u;
         }
+        if (warp == 0) {
+            mbar_init(reinterpret_cast<uint64_t *>(smem + SM::off_cbar), 1);
+            *reinterpret_cast<uint32_t *>(smem + SM::off_cuse) = 0u;
+        }
         mbar_init_fence();
     }
     __syncwarp();
@@ -365,6 +381,7 @@ __device__ __forceinline__ void stages_inval(unsigned char *smem) {
         uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::off_bar) + warp * SW_STAGES;
 #pragma unroll
         for (int st = 0; st < SW_STAGES; ++st) mbar_inval(&bars[st]);
+        if (warp == 0) mbar_inval(reinterpret_cast<uint64_t *>(smem + SM::off_cbar));
     }
     __syncwarp();
 }
@@ -413,6 +430,10 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
     // phases each stage barrier has completed before this call
     uint32_t *uses = reinterpret_cast<uint32_t *>(smem + SM::off_uses) + warp * SW_STAGES;
     const uint32_t u0 = uses[0], u1 = uses[1];
+    // the stages' bytes were last written through the generic proxy (the
+    // previous level's cut scratch): fenced once here, before any copy lands
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    gsync();
     float b0 = 0.f, b1 = 0.f;  // plane offsets of row `lane` of stages 0 and 1
     if (nmine > 0)
         b0 = stage_issue<HD, R, G, RT>(L, c0, c1, k0, warp, pid, pmk, gb, bb, c, clog, nl, bufs, &bars[0], cnode,
@@ -424,9 +445,11 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
     const int rl = (lane / G) % 8;       // row of this lane's sum within the batch
     float mymax = -INFINITY;             // this lane's head's maximum (lanes < G report)
     uint32_t mycnt = 0u;
-#pragma unroll 1
-    for (int j = 0; j < nmine; ++j) {
-        const int st = j % SW_STAGES;
+    // unit j in stage st (a compile-time constant, so that the plane offsets
+    // loaded for the stage land in b0 / b1 directly and nothing waits for them
+    // before they are used)
+    auto unit = [&](const int j, auto stc, float &bst) {
+        constexpr int st = decltype(stc)::value;
         const int64_t u = warp + (int64_t)j * NW;
         const int64_t sb = c0 + u * C::SLOTS;
         const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
@@ -434,10 +457,10 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         const uint8_t *cm = cmask + st * SW_ROWS_MAX;
         if (!mbar_wait(&bars[st], ((st ? u1 : u0) + (uint32_t)(j / SW_STAGES)) & 1u, nullptr))
             set_status(a.status, ZHA_TIMEOUT_CODE);
-        const float bl = st ? b1 : b0;  // plane offset of row `lane`
+        const float bl = bst;  // plane offset of row `lane`
         const RT *cb = reinterpret_cast<const RT *>(bufs + (size_t)st * SW_BYTES);
         float est = -INFINITY;
-#pragma unroll 1
+#pragma unroll 2
         for (int r0 = 0; r0 < C::ROWS; r0 += 8) {
             // rows r0 .. r0 + 7: slot r / R, plane r % R
             float v[8 * G];
@@ -499,9 +522,13 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
             const float bn = stage_issue<HD, R, G, RT>(L, c0, c1, k0, u + (int64_t)SW_STAGES * NW, pid, pmk, gb, bb, c,
                                                    clog, nl, bufs + (size_t)st * SW_BYTES, &bars[st],
                                                    cnode + st * SW_ROWS_MAX, cmask + st * SW_ROWS_MAX, lane);
-            if (st) b1 = bn;
-            else b0 = bn;
+            bst = bn;
         }
+    };
+#pragma unroll 1
+    for (int j = 0; j < nmine; j += SW_STAGES) {
+        unit(j, std::integral_constant<int, 0>{}, b0);
+        if (j + 1 < nmine) unit(j + 1, std::integral_constant<int, 1>{}, b1);
     }
     __syncwarp();
     if (lane == 0) {
@@ -738,18 +765,15 @@ __device__ __noinline__ void sort_cut(const Level &L, const HeadCut *cut, float 
 }
 
 // Local histogram of round r over this CTA's slots on the path of every open
-// head, into hc/hm (shared; cleared here).
+// head: counts into hc, masses into hw.  A mass (at most 2^40 in units of
+// 2^-40) is added as its low 20 bits and the rest into two 32-bit words, the
+// bucket's pair in hw (the 8 bytes of its 64-bit mass): 64-bit atomics on
+// shared memory cost about ten times as much as 32-bit ones.  Both sums stay
+// below 2^31 for up to HIST_WIN slots, after which fold_window() or
+// fold_local() must take them.  Slots of heads whose mass is 0 add nothing.
+constexpr int HIST_WIN = 2048;
 template <int G>
-__device__ __noinline__ void local_hist(const Level &L, const HeadCut *cut, int r, uint32_t *hc,
-                                        unsigned long long *hm, bool clear = true) {
-    if (clear) {
-#pragma unroll 1
-        for (int i = threadIdx.x; i < G * NB; i += GT) {
-            hc[i] = 0u;
-            hm[i] = 0ull;
-        }
-        gsync();
-    }
+__device__ __noinline__ void local_hist(const Level &L, const HeadCut *cut, int r, uint32_t *hc, uint32_t *hw) {
     // GT is a multiple of G: every entry this thread visits belongs to head tid % G
     const int h = (int)(threadIdx.x % G);
     const PathReg H(cut[h]);
@@ -763,11 +787,43 @@ __device__ __noinline__ void local_hist(const Level &L, const HeadCut *cut, int 
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 if (e[u] == -INFINITY || H.cmp(e[u], r) != 0) continue;
-                const int b = H.bucket(e[u], r);
-                atomicAdd(&hc[h * NB + b], 1u);
-                atomicAdd(&hm[h * NB + b], mass_fx(expf(e[u] - H.M)));
+                const int b = h * NB + H.bucket(e[u], r);
+                const unsigned long long m = mass_fx(expf(e[u] - H.M));
+                const uint32_t lo = (uint32_t)(m & 0xfffffull), hi = (uint32_t)(m >> 20);
+                atomicAdd(&hc[b], 1u);
+                if (lo) atomicAdd(&hw[2 * b], lo);
+                if (hi) atomicAdd(&hw[2 * b + 1], hi);
             }
         }
+    }
+    gsync();
+}
+
+// A window's counts and masses into the team's histogram of the round
+// (global, exact integer sums); the shared words are left cleared.
+template <int G>
+__device__ __forceinline__ void fold_window(uint32_t *hc, uint32_t *hw, uint32_t *gc, unsigned long long *gm) {
+#pragma unroll 1
+    for (int i = threadIdx.x; i < G * NB; i += GT) {
+        const uint32_t n = hc[i];
+        if (n) {
+            atomicAdd(gc + i, n);
+            atomicAdd(gm + i, (unsigned long long)hw[2 * i] + ((unsigned long long)hw[2 * i + 1] << 20));
+            hc[i] = 0u;
+            hw[2 * i] = 0u;
+            hw[2 * i + 1] = 0u;
+        }
+    }
+    gsync();
+}
+
+// One window's mass words turned, in place, into the 64-bit masses find_cut reads.
+template <int G>
+__device__ __forceinline__ void fold_local(uint32_t *hw) {
+#pragma unroll 1
+    for (int i = threadIdx.x; i < G * NB; i += GT) {
+        const unsigned long long m = (unsigned long long)hw[2 * i] + ((unsigned long long)hw[2 * i + 1] << 20);
+        reinterpret_cast<unsigned long long *>(hw)[i] = m;
     }
     gsync();
 }
@@ -856,8 +912,12 @@ __device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsign
     const int64_t iters = (L.n + GT - 1) / GT;
     // every head's cut state in registers (see PathReg)
     PathReg Hr[G];
+    unsigned long long osum_t[G];  // this thread's boundary masses of CUT_ORDER heads
 #pragma unroll
-    for (int h = 0; h < G; ++h) Hr[h] = PathReg(cut[h]);
+    for (int h = 0; h < G; ++h) {
+        Hr[h] = PathReg(cut[h]);
+        osum_t[h] = 0ull;
+    }
 #pragma unroll 1
     for (int64_t it = 0; it < iters; ++it) {
         const int64_t i = it * GT + threadIdx.x;
@@ -880,7 +940,7 @@ __device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsign
                     else if (pc == 0) {
                         w = mass_fx(expf(e - H.M));
                         if (H.mode == CUT_RANK) cand = true;
-                        else atomicAdd(&osum[h], w);
+                        else osum_t[h] += w;
                     }
                 }
             }
@@ -907,6 +967,13 @@ __device__ __noinline__ void classify(const Level &L, const HeadCut *cut, unsign
             }
         }
         if (i < L.n) L.keep[i] = (uint8_t)kbits;
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        unsigned long long x = osum_t[h];
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+        if (lane == 0 && x) atomicAdd(&osum[h], x);
     }
     gsync();
 }
@@ -1076,6 +1143,7 @@ __device__ __forceinline__ Level chunk_level(const Level &L, int64_t c0, int64_t
     C.s0 = L.s0 + c0;
     C.n = n;
     C.sc = ssc;
+    C.sc_local = true;
     C.node = L.node + c0;
     C.keep = L.keep + c0;
     return C;
@@ -1188,29 +1256,43 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
 #pragma unroll 1
         for (int h = 0; h < G; ++h) open |= cut[h].mode == CUT_OPEN;
         if (!open) break;
-        if (L.n <= LOC_CAP) {
-            local_hist<G>(L, cut, r, hc, hm);
-        } else {
-            // spilled slots: by chunks through the shared score array
-            float *ssc = reinterpret_cast<float *>(smem + SM::off_sc);
+        // windows of HIST_WIN slots (the spilled ones by chunks through the
+        // shared score array); a team folds each into its global histogram,
+        // a lone CTA (at most HIST_WIN slots: teams take larger slices) in place
+        uint32_t *gc = a.hist_cnt + hbase + (int64_t)r * G * NB;
+        unsigned long long *gm = a.hist_mass + hbase + (int64_t)r * G * NB;
+        uint32_t *hw = reinterpret_cast<uint32_t *>(hm);
 #pragma unroll 1
-            for (int64_t c0 = 0; c0 < L.n; c0 += LOC_CAP) {
-                const int64_t n = min((int64_t)LOC_CAP, L.n - c0);
-                chunk_scores_in<G>(L, c0, n, ssc);
+        for (int i = tid; i < G * NB; i += GT) {
+            hc[i] = 0u;
+            hm[i] = 0ull;
+        }
+        gsync();
+        static_assert(HIST_WIN == LOC_CAP, "a spilled chunk is one histogram window");
+        float *ssc = reinterpret_cast<float *>(smem + SM::off_sc);
+#pragma unroll 1
+        for (int64_t w0 = 0; w0 < L.n; w0 += HIST_WIN) {
+            const int64_t n = min((int64_t)HIST_WIN, L.n - w0);
+            if (!L.sc_local) {
+                chunk_scores_in<G>(L, w0, n, ssc);
                 gsync();
-                local_hist<G>(chunk_level(L, c0, n, ssc), cut, r, hc, hm, c0 == 0);
             }
+            local_hist<G>(chunk_level(L, w0, n, L.sc_local ? L.sc + w0 * G : ssc), cut, r, hc, hw);
+            if (team || L.n > HIST_WIN) fold_window<G>(hc, hw, gc, gm);
         }
         rounds_used = r + 1;
-        if (team) {
-            uint32_t *gc = a.hist_cnt + hbase + (int64_t)r * G * NB;
-            unsigned long long *gm = a.hist_mass + hbase + (int64_t)r * G * NB;
-#pragma unroll 1
-            for (int i = tid; i < G * NB; i += GT)
-                if (hc[i]) {
-                    atomicAdd(gc + i, hc[i]);
-                    atomicAdd(gm + i, hm[i]);
-                }
+        if (!team && L.n > HIST_WIN) {
+            // (a lone CTA with more slots: the sums went through the global histogram)
+#pragma unroll 16
+            for (int i = tid; i < G * NB; i += GT) {
+                hm[i] = __ldcg(gm + i);
+                hc[i] = __ldcg(gc + i);
+                gm[i] = 0ull;
+                gc[i] = 0u;
+            }
+            gsync();
+            find_cut<G>(cut, r, hc, nullptr, hm, a.p, red);
+        } else if (team) {
             if (!ts.sync()) return false;  // B
             // the team's bucket masses into shared memory: independent loads
 #pragma unroll 16
@@ -1218,6 +1300,7 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
             gsync();
             find_cut<G>(cut, r, hc, gc, hm, a.p, red);
         } else {
+            fold_local<G>(hw);
             find_cut<G>(cut, r, hc, nullptr, hm, a.p, red);
         }
     }
@@ -1228,7 +1311,7 @@ __device__ __noinline__ bool hist_cut(const Decode &a, const Level &L, unsigned 
     gsync();
     // candidates go to shared lists first (shared counters); a team then
     // reserves room in its global lists with one atomic per head
-    if (L.n <= LOC_CAP) {
+    if (L.sc_local) {
         classify<G>(L, cut, cw, cs, misc + 4, own, misc, osum);
     } else {
         float *ssc = reinterpret_cast<float *>(smem + SM::off_sc);
@@ -1353,7 +1436,8 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
     L.Sp = Sp;
     Tout = T;
     const bool team = T > 1;
-    if (L.n > LOC_CAP) {
+    L.sc_local = L.n <= LOC_CAP;
+    if (!L.sc_local) {
         const int64_t base = (int64_t)kh * a.score_cap + L.s0;
         L.sc = a.scores + base * G;
         L.node = a.slot_node + base;
@@ -1385,6 +1469,21 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
         gsync();
         score_chunks<HD, R, G, RT>(a, L, c0, c1, k0, pid, pmk, smem, wm, wc);
         gsync();
+    }
+    // a spilled slice that fits below the cut scratch comes back on chip in
+    // one bulk copy, whose latency the maxima's barrier hides
+    uint64_t *cbar = reinterpret_cast<uint64_t *>(smem + SM::off_cbar);
+    const bool back = G == 4 && !L.sc_local && L.n <= SM::SPILL_CAP;
+    if (back) {
+        // this thread's score stores (global) and earlier writes to the
+        // destination (shared), ordered before the copy
+        asm volatile("fence.proxy.async;" ::: "memory");
+        gsync();
+        if (tid == 0) {
+            const uint32_t nbytes = (uint32_t)(L.n * G * 4);
+            mbar_arrive_expect_tx(cbar, nbytes);
+            bulk_g2s(smem + SM::off_sc, L.sc, nbytes, cbar);
+        }
     }
     if (tid < G) {
         float m = -INFINITY;
@@ -1434,6 +1533,14 @@ __device__ __noinline__ bool route_level(const Decode &a, int l, int kh, int T, 
             cut[tid].M = mm;
             cut[tid].F = cc;
         }
+    }
+    if (back) {
+        uint32_t *cuse = reinterpret_cast<uint32_t *>(smem + SM::off_cuse);
+        if (!mbar_wait(cbar, *cuse & 1u, nullptr)) set_status(a.status, ZHA_TIMEOUT_CODE);
+        gsync();
+        if (tid == 0) *cuse += 1u;
+        L.sc = reinterpret_cast<float *>(smem + SM::off_sc);
+        L.sc_local = true;
     }
     const bool keep_all = !(a.p < 1.f);
     const bool solo = L.T == 1;
@@ -1548,6 +1655,7 @@ __device__ __noinline__ bool route_level_rd(const Decode &a, int l, int kh, int 
     L.Tp = 1;
     L.Sp = 0;
     L.keep = keep;
+    L.sc_local = mode == LV_ALL;
     if (mode == LV_ALL) {
         L.s0 = 0;
         L.n = S;
@@ -1627,6 +1735,7 @@ __device__ __noinline__ bool route_level_rd(const Decode &a, int l, int kh, int 
     LA.s0 = 0;
     LA.n = S;
     LA.sc = sc;
+    LA.sc_local = true;
     LA.node = node;
     if (!(a.p < 1.f)) {
 #pragma unroll 1
