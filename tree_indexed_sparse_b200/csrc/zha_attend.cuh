@@ -571,9 +571,20 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
 
     if (warp == ACW) {
         // ---------------- producer warp ----------------
+        // the kept leaves of the current KV head, ranks [., rhi) of them at
+        // rank % LEAF_WIN: a ring refilled a chunk of RING_CHUNK ranks at a
+        // time, each chunk's loads issued a chunk ahead of its use, so that
+        // their latency hides behind the stages between
         int32_t *win_ids = reinterpret_cast<int32_t *>(smem + SM::off_win);
         uint8_t *win_msk = smem + SM::off_win + (size_t)LEAF_WIN * 4;
-        int win_kh = -1, win_k0 = 0;
+        constexpr int RING_CHUNK = 128, PERL = RING_CHUNK / 32;
+        static_assert((LEAF_WIN & (LEAF_WIN - 1)) == 0 && RING_CHUNK <= LEAF_WIN / 2, "leaf ring");
+        int win_kh = -1, rhi = 0, rend = 0, rseg = 0;
+        bool pending = false;
+        const int32_t *kid = nullptr;
+        const uint8_t *kmk = nullptr;
+        int32_t cid[PERL];
+        uint32_t cmk[PERL];
         int issued = 0;
         const uint64_t pol = l2_evict_first();  // K/V rows are read once
         int kh;
@@ -627,40 +638,48 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
             if (!DENSE) {
                 kf = (int)div_c((uint32_t)t0, c, clog);
                 const int kl = min(L - 1, (int)div_c((uint32_t)(t0 + TT - 1), c, clog));
-                if (kh != win_kh || kl >= win_k0 + LEAF_WIN || kf < win_k0) {
-                    // refill the window from leaf rank kf up to the last leaf
-                    // this CTA needs in this KV head: independent loads
+                if (kh != win_kh) {
+                    // a new KV head: its kept leaves from rank kf up to the last
+                    // one this CTA needs
                     const int jl = (int)(min(u1, map.pref[kh + 1]) - 1 - map.pref[kh]);
-                    const int klast = min(L - 1, (int)div_c((uint32_t)(jl * TT + TT - 1), c, clog));
-                    const int nwin = min(LEAF_WIN, klast - kf + 1);
                     win_kh = kh;
-                    win_k0 = kf;
-                    const int32_t *kid = a.kept_ids[0] + (int64_t)kh * a.slot_cap[0];
-                    const uint8_t *kmk = a.kept_mask[0] + (int64_t)kh * a.slot_cap[0];
-                    // ranks kf + lane, + 32, ...: the segment only moves
-                    // forward; all of a lane's loads are in flight at once
-                    constexpr int PERL = LEAF_WIN / 32;
-                    int rseg = 0;
-                    int32_t wid[PERL];
-                    uint32_t wmk[PERL];
+                    rend = min(L - 1, (int)div_c((uint32_t)(jl * TT + TT - 1), c, clog)) + 1;
+                    rhi = kf;
+                    rseg = 0;
+                    pending = false;
+                    kid = a.kept_ids[0] + (int64_t)kh * a.slot_cap[0];
+                    kmk = a.kept_mask[0] + (int64_t)kh * a.slot_cap[0];
+                }
+                // ranks below kf are done with; a chunk goes out as soon as the
+                // ring has room for it, and lands (its loads waited for) only
+                // when a stage needs its ranks
+#pragma unroll 1
+                while (true) {
+                    if (!pending && rhi < rend && rhi + RING_CHUNK - kf <= LEAF_WIN) {
+                        // ranks rhi + lane + 32 t (the lane's segment only moves forward)
 #pragma unroll
-                    for (int t = 0; t < PERL; ++t) {
-                        const int i = lane + 32 * t;
-                        if (i < nwin) {
-                            const int at = (int)map.leaf_at_from(kh, kf + i, rseg);
-                            wid[t] = __ldcg(kid + at);
-                            wmk[t] = __ldcg(kmk + at);
+                        for (int t = 0; t < PERL; ++t) {
+                            const int k = rhi + lane + 32 * t;
+                            if (k < rend) {
+                                const int at = (int)map.leaf_at_from(kh, k, rseg);
+                                cid[t] = __ldcg(kid + at);
+                                cmk[t] = __ldcg(kmk + at);
+                            }
                         }
+                        pending = true;
                     }
+                    if (rhi > kl) break;
 #pragma unroll
                     for (int t = 0; t < PERL; ++t) {
-                        const int i = lane + 32 * t;
-                        if (i < nwin) {
-                            win_ids[i] = wid[t];
-                            win_msk[i] = (uint8_t)wmk[t];
+                        const int k = rhi + lane + 32 * t;
+                        if (k < rend) {
+                            win_ids[k & (LEAF_WIN - 1)] = cid[t];
+                            win_msk[k & (LEAF_WIN - 1)] = (uint8_t)cmk[t];
                         }
                     }
                     __syncwarp();
+                    rhi = min(rend, rhi + RING_CHUNK);
+                    pending = false;
                 }
             }
             if (fast) {
@@ -675,8 +694,8 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                         uint32_t mk = 0u;
                         if (ug < L * c) {
                             const int k = (int)div_c((uint32_t)ug, c, clog);
-                            mk = win_msk[k - win_k0];
-                            row0 = win_ids[k - win_k0] * c + (ug - k * c);
+                            mk = win_msk[k & (LEAF_WIN - 1)];
+                            row0 = win_ids[k & (LEAF_WIN - 1)] * c + (ug - k * c);
                             rows = max(0, min(GR, N - row0));
                         }
                         srow = lane * GR;
@@ -694,10 +713,10 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                     uint32_t mk = 0u;
                     bool cont = false;
                     if (lane < lps && k < L) {
-                        id = win_ids[k - win_k0];
-                        mk = win_msk[k - win_k0];
+                        id = win_ids[k & (LEAF_WIN - 1)];
+                        mk = win_msk[k & (LEAF_WIN - 1)];
                         valid = min(c, N - id * c);
-                        if ((lane & nlm) != 0) cont = win_ids[k - 1 - win_k0] == id - 1;
+                        if ((lane & nlm) != 0) cont = win_ids[(k - 1) & (LEAF_WIN - 1)] == id - 1;
                     }
                     const uint32_t cm = __ballot_sync(FULL, cont);
                     // leaves the run takes after its first: the continuing lanes just above
@@ -755,8 +774,8 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                 // [k c, (k + 1) c) of the flattened list, rows id_k c + (0 .. c-1)
                 int u = ug, k = (int)div_c((uint32_t)ug, c, clog), off = ug - k * c;
                 while (u < ug + GR && k < L) {
-                    const int id = win_ids[k - win_k0];
-                    const uint32_t mk = win_msk[k - win_k0];
+                    const int id = win_ids[k & (LEAF_WIN - 1)];
+                    const uint32_t mk = win_msk[k & (LEAF_WIN - 1)];
                     const int len = min(c - off, ug + GR - u);
                     const int vlen = max(0, min(len, N - (id * c + off)));
                     if (!isV) {
@@ -802,7 +821,7 @@ __device__ void attn_stages(const Decode &a, const StageMap &map, unsigned char 
                     int u = ug, k = (int)div_c((uint32_t)ug, c, clog), off = ug - k * c;
                     int run_w = 0, run_row = -1, run_len = 0;
                     while (u < ug + (int)nvalid) {
-                        const int r0 = win_ids[k - win_k0] * c + off;
+                        const int r0 = win_ids[k & (LEAF_WIN - 1)] * c + off;
                         const int len = min(c - off, ug + (int)nvalid - u);
                         if (run_len > 0 && r0 == run_row + run_len) {
                             run_len += len;

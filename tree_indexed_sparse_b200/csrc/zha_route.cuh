@@ -56,8 +56,6 @@
 // synchronises them with the named barrier of gsync().
 #pragma once
 
-#include <type_traits>
-
 #include "zha_device.cuh"
 #include "zha_internal.cuh"
 #include "zha_sync.cuh"
@@ -138,7 +136,8 @@ struct RouteSmem {
     static constexpr size_t off_uses = off_bar + SW_N * 8;               // [SW_N] u32 completed phases
     static constexpr size_t off_cnode = off_uses + SW_N * 4;              // [SW_N][SW_ROWS_MAX] i32
     static constexpr size_t off_cmask = off_cnode + (size_t)SW_N * SW_ROWS_MAX * 4;  // [SW_N][SW_ROWS_MAX] u8
-    static constexpr size_t off_misc = (off_cmask + (size_t)SW_N * SW_ROWS_MAX + 15) / 16 * 16;  // u32 counters
+    static constexpr size_t off_cb = (off_cmask + (size_t)SW_N * SW_ROWS_MAX + 15) / 16 * 16;  // [SW_N][SW_ROWS_MAX] f32
+    static constexpr size_t off_misc = off_cb + (size_t)SW_N * SW_ROWS_MAX * 4;  // u32 counters
     static constexpr size_t off_cbar = off_misc + 64;                     // u64: barrier of the scores' return
     static constexpr size_t off_cuse = off_cbar + 8;                      // u32: its completed phases
     static constexpr size_t bytes = off_cuse + 8;
@@ -284,15 +283,16 @@ struct ScoreStage {
 };
 
 // One warp: node ids of the slots of unit u (SLOTS consecutive local slots
-// from c0) and bulk copies of their g rows (one copy per run of consecutive
-// nodes) into this warp's stage buffer `dst`, completing on the stage barrier
-// `bar`.  Returns the plane offset of row `lane` (slot lane / R, plane
-// lane % R; 0 past the unit): a register load whose latency the copy hides.
+// from c0), bulk copies of their g rows (one copy per run of consecutive
+// nodes) into this warp's stage buffer `dst`, and the plane offset of each
+// row (slot r / R, plane r % R) into cb[r] by 4-byte asynchronous copies, all
+// completing on the stage barrier `bar` (each copying lane adds one pending
+// arrival that its copy's completion clears, before the expect-tx arrive).
 template <int HD, int R, int G, typename RT>
-__device__ __forceinline__ float stage_issue(const Level &L, int64_t c0, int64_t c1, int64_t k0, int64_t u,
-                                             const int32_t *pid, const uint8_t *pmk, const RT *gb, const float *bb,
-                                             int c, int clog, int32_t nl, unsigned char *dst, uint64_t *bar,
-                                             int32_t *cn, uint8_t *cm, int lane) {
+__device__ __forceinline__ void stage_issue(const Level &L, int64_t c0, int64_t c1, int64_t k0, int64_t u,
+                                            const int32_t *pid, const uint8_t *pmk, const RT *gb, const float *bb,
+                                            int c, int clog, int32_t nl, unsigned char *dst, uint64_t *bar,
+                                            int32_t *cn, uint8_t *cm, float *cb, int lane) {
     using C = ScoreStage<HD, R, RT>;
     const int64_t sb = c0 + u * C::SLOTS;
     const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
@@ -311,6 +311,14 @@ __device__ __forceinline__ float stage_issue(const Level &L, int64_t c0, int64_t
         cm[lane] = nd >= 0 ? (uint8_t)mk : 0;
     }
     const uint32_t nvalid = __popc(__ballot_sync(FULL, nd >= 0));
+    const int ndr = __shfl_sync(FULL, nd, (lane / R) & 31);
+    if (lane < C::ROWS && ndr >= 0) {
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(cb + lane)),
+                     "l"(bb + (size_t)ndr * R + lane % R)
+                     : "memory");
+        asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+    }
+    __syncwarp();
     // (the stage's earlier contents were only read, and those reads completed
     // before the warp got here: a bulk copy may overwrite it without a fence)
     if (lane == 0) mbar_arrive_expect_tx(bar, nvalid * (uint32_t)C::NODE_BYTES);
@@ -325,8 +333,6 @@ __device__ __forceinline__ float stage_issue(const Level &L, int64_t c0, int64_t
         bulk_g2s_hint(dst + (size_t)lane * C::NODE_BYTES, gb + (size_t)nd * R * HD, (uint32_t)(len * C::NODE_BYTES),
                       bar, l2_evict_first());
     }
-    const int ndr = __shfl_sync(FULL, nd, (lane / R) & 31);
-    return (lane < C::ROWS && ndr >= 0) ? __ldg(bb + (size_t)ndr * R + lane % R) : 0.f;
 }
 
 // Sums over the warp of 8 rows x G heads of per-lane partial dots, v[row*G + h].
@@ -411,6 +417,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SM::off_bar) + warp * SW_STAGES;
     int32_t *cnode = reinterpret_cast<int32_t *>(smem + SM::off_cnode) + warp * SW_STAGES * SW_ROWS_MAX;
     uint8_t *cmask = smem + SM::off_cmask + warp * SW_STAGES * SW_ROWS_MAX;
+    float *cbs = reinterpret_cast<float *>(smem + SM::off_cb) + warp * SW_STAGES * SW_ROWS_MAX;
     float qs[G][VEC];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -426,7 +433,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
     const int32_t nl = a.t.n_level[l - 1];
     const int64_t nu = (c1 - c0 + C::SLOTS - 1) / C::SLOTS;  // units
     const int nmine = nu > warp ? (int)((nu - 1 - warp) / NW + 1) : 0;
-    static_assert(SW_STAGES == 2, "two stages: plane offsets in b0 / b1");
+    static_assert(SW_STAGES == 2, "two stages: units 0 and 1 go out before the loop");
     // phases each stage barrier has completed before this call
     uint32_t *uses = reinterpret_cast<uint32_t *>(smem + SM::off_uses) + warp * SW_STAGES;
     const uint32_t u0 = uses[0], u1 = uses[1];
@@ -434,22 +441,19 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
     // previous level's cut scratch): fenced once here, before any copy lands
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     gsync();
-    float b0 = 0.f, b1 = 0.f;  // plane offsets of row `lane` of stages 0 and 1
     if (nmine > 0)
-        b0 = stage_issue<HD, R, G, RT>(L, c0, c1, k0, warp, pid, pmk, gb, bb, c, clog, nl, bufs, &bars[0], cnode,
-                                   cmask, lane);
+        stage_issue<HD, R, G, RT>(L, c0, c1, k0, warp, pid, pmk, gb, bb, c, clog, nl, bufs, &bars[0], cnode, cmask,
+                                  cbs, lane);
     if (nmine > 1)
-        b1 = stage_issue<HD, R, G, RT>(L, c0, c1, k0, warp + NW, pid, pmk, gb, bb, c, clog, nl, bufs + SW_BYTES,
-                                   &bars[1], cnode + SW_ROWS_MAX, cmask + SW_ROWS_MAX, lane);
+        stage_issue<HD, R, G, RT>(L, c0, c1, k0, warp + NW, pid, pmk, gb, bb, c, clog, nl, bufs + SW_BYTES, &bars[1],
+                                  cnode + SW_ROWS_MAX, cmask + SW_ROWS_MAX, cbs + SW_ROWS_MAX, lane);
     const int hl = lane % G;             // head of this lane's sum
     const int rl = (lane / G) % 8;       // row of this lane's sum within the batch
     float mymax = -INFINITY;             // this lane's head's maximum (lanes < G report)
     uint32_t mycnt = 0u;
-    // unit j in stage st (a compile-time constant, so that the plane offsets
-    // loaded for the stage land in b0 / b1 directly and nothing waits for them
-    // before they are used)
-    auto unit = [&](const int j, auto stc, float &bst) {
-        constexpr int st = decltype(stc)::value;
+#pragma unroll 1
+    for (int j = 0; j < nmine; ++j) {
+        const int st = j % SW_STAGES;
         const int64_t u = warp + (int64_t)j * NW;
         const int64_t sb = c0 + u * C::SLOTS;
         const int ns = (int)min((int64_t)C::SLOTS, c1 - sb);
@@ -457,10 +461,10 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         const uint8_t *cm = cmask + st * SW_ROWS_MAX;
         if (!mbar_wait(&bars[st], ((st ? u1 : u0) + (uint32_t)(j / SW_STAGES)) & 1u, nullptr))
             set_status(a.status, ZHA_TIMEOUT_CODE);
-        const float bl = bst;  // plane offset of row `lane`
+        const float *cbr = cbs + st * SW_ROWS_MAX;  // plane offsets of the stage's rows
         const RT *cb = reinterpret_cast<const RT *>(bufs + (size_t)st * SW_BYTES);
         float est = -INFINITY;
-#pragma unroll 2
+#pragma unroll 1
         for (int r0 = 0; r0 < C::ROWS; r0 += 8) {
             // rows r0 .. r0 + 7: slot r / R, plane r % R
             float v[8 * G];
@@ -479,7 +483,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
             }
             const float sum = batch_sum<G>(v, lane);
             const int r = r0 + rl;
-            const float e = __shfl_sync(FULL, bl, r) + sum;
+            const float e = cbr[r] + sum;
             if constexpr (R == 1) {
                 // every row is its own slot
                 const int i = r;
@@ -518,17 +522,10 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
             }
         }
         __syncwarp();  // stage st is free
-        if (j + SW_STAGES < nmine) {
-            const float bn = stage_issue<HD, R, G, RT>(L, c0, c1, k0, u + (int64_t)SW_STAGES * NW, pid, pmk, gb, bb, c,
-                                                   clog, nl, bufs + (size_t)st * SW_BYTES, &bars[st],
-                                                   cnode + st * SW_ROWS_MAX, cmask + st * SW_ROWS_MAX, lane);
-            bst = bn;
-        }
-    };
-#pragma unroll 1
-    for (int j = 0; j < nmine; j += SW_STAGES) {
-        unit(j, std::integral_constant<int, 0>{}, b0);
-        if (j + 1 < nmine) unit(j + 1, std::integral_constant<int, 1>{}, b1);
+        if (j + SW_STAGES < nmine)
+            stage_issue<HD, R, G, RT>(L, c0, c1, k0, u + (int64_t)SW_STAGES * NW, pid, pmk, gb, bb, c, clog, nl,
+                                      bufs + (size_t)st * SW_BYTES, &bars[st], cnode + st * SW_ROWS_MAX,
+                                      cmask + st * SW_ROWS_MAX, cbs + st * SW_ROWS_MAX, lane);
     }
     __syncwarp();
     if (lane == 0) {
