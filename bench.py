@@ -772,6 +772,70 @@ def run_crossover(args, local):
                        "l2": "256 MiB written before every call"}}
 
 
+def run_kv_shards(args, local):
+    """KV-head sharding of the workload over N GPUs, measured on one GPU: each
+    shard (its KV heads' cache, built from the same inputs) decodes every
+    step alone, L2 flushed before each call; shards share no data on the
+    decode path, so an N-GPU job's time per token is the slowest shard's.
+    The whole cache is timed beside them on the same steps."""
+    import tree_indexed_sparse_b200 as zha
+    from tree_indexed_sparse_b200.shard import ShardedZhaCache
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    w = workloads.WORKLOADS[args.workload]
+    N = args.kv_shards
+    W, K = args.warmup, args.steps
+    inp = workloads.generate(w, dev)
+    dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
+    whole = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, device=dev)
+    whole.build(inp.K, inp.V, w.n_tokens, inp.ref)
+    shards = []
+    for r in range(N):
+        sh = ShardedZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, rank=r, world=N, device=dev)
+        sh.build(sh.local_kv(inp.K).contiguous(), sh.local_kv(inp.V).contiguous(), w.n_tokens,
+                 sh.local_kv(inp.ref).contiguous())
+        shards.append(sh)
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(fn):
+        flush.zero_()
+        torch.cuda._sleep(HOLD_CYCLES)
+        ea.record(stream)
+        fn()
+        eb.record(stream)
+        torch.cuda.synchronize()
+        return ea.elapsed_time(eb) * 1e3
+
+    t_whole, t_shard = [], [[] for _ in range(N)]
+    clocks = Clocks(local)
+    for i in range(W + K):
+        q = inp.Q[i % w.steps]
+        if i == W:
+            clocks.start()
+        tw = timed(lambda: whole.decode(q, w.p))
+        ts = [timed(lambda: sh.decode(q, w.p)) for sh in shards]
+        if i >= W:
+            t_whole.append(tw)
+            for r in range(N):
+                t_shard[r].append(ts[r])
+    clk = clocks.stop()
+    assert whole.status() == 0 and all(sh.status() == 0 for sh in shards)
+    per_step = [max(t_shard[r][i] for r in range(N)) for i in range(K)]
+    job_us = statistics.mean(per_step)
+    return {"metric": "us per decoded token per layer, KV heads split over N GPUs (each shard timed alone on one GPU)",
+            "unit": "us/token", "value": job_us, "higher_is_better": False, "n_gpus_emulated": N, "steps": K,
+            "warmup": W, "scaling": "strong", "data": "synthetic",
+            "whole_cache_us": statistics.mean(t_whole), "speedup": statistics.mean(t_whole) / job_us,
+            "shards": [{"kv_heads": [sh.kv0, sh.kv1], "us": statistics.mean(t_shard[r])} for r, sh in enumerate(shards)],
+            "clocks": clk,
+            "config": {"workload": w.name, "parallelism": f"kv-heads x{N} (emulated: shards run one after another)",
+                       "l2": "256 MiB written before every call"}}
+
+
 def record_traffic(csv_path: str, steps_path: str, launch: int) -> None:
     """Write profiles/k_decode_traffic.json from one ncu capture: the DRAM
     bytes (read + write) of k_decode launch `launch` (0-based, the first
@@ -828,6 +892,8 @@ def main():
                     help="summaries the routing reads: fp32 (default) or the bf16 router copy")
     ap.add_argument("--growth", action="store_true",
                     help="time the step where a tree with room to grow adds a level (light settings, 2M tokens)")
+    ap.add_argument("--kv-shards", type=int, default=0, metavar="N",
+                    help="time the workload split by KV head over N GPUs, each shard alone on this GPU")
     ap.add_argument("--record-traffic", nargs=3, metavar=("NCU_CSV", "STEP_BYTES_JSON", "LAUNCH"),
                     help="write profiles/k_decode_traffic.json from an ncu capture of k_decode (no GPU needed)")
     args = ap.parse_args()
@@ -836,9 +902,10 @@ def main():
         return
     args.warmup = max(args.warmup, 3)
     rank, world, local = dist_setup(args.gpus)
-    if args.crossover or args.growth:
+    if args.crossover or args.growth or args.kv_shards:
         if rank == 0:
-            print(json.dumps(run_crossover(args, local) if args.crossover else run_growth(args, local)), flush=True)
+            run = run_crossover if args.crossover else run_growth if args.growth else run_kv_shards
+            print(json.dumps(run(args, local)), flush=True)
         if world > 1:
             torch.distributed.destroy_process_group()
         return

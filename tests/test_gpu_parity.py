@@ -464,3 +464,40 @@ def test_batch_decode(name, n_q):
     with pytest.raises(zha.ZhaError) as e:
         cache.decode_batch(torch.zeros(n_q + 1, h_q, w.d, device="cuda"), w.p)
     assert e.value.code == zha.ZHA_ERR_BAD_ARG
+
+
+@pytest.mark.parametrize("name,world", [("wide", 2), ("light", 4), ("deep", 3)])
+def test_kv_head_shards(name, world):
+    """A cache split by KV head (tree_indexed_sparse_b200.shard): every
+    shard, built from its heads' slices and decoding its query heads, passes
+    the oracle protocol on those heads and matches the whole cache's decode
+    of them (leaf sets exactly, outputs within the tolerance).  The shards
+    run one after another on this GPU: their decodes never exchange data."""
+    from tree_indexed_sparse_b200.shard import ShardedZhaCache
+
+    c = get_case(name)
+    w = c.w
+    dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
+    cap = oracle.level_nodes(w.capacity, w.c, 1)
+    q = c.inp.Q[0]
+    whole = c.cache.decode(q.cuda(), w.p)
+    torch.cuda.synchronize()
+    covered = []
+    for rank in range(world):
+        sh = ShardedZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, rank=rank, world=world)
+        # the whole cache may have appended rows past n: shards take the same prefix
+        sh.build(sh.local_kv(c.dK).contiguous(), sh.local_kv(c.dV).contiguous(), c.n, sh.local_kv(c.dref).contiguous())
+        res = sh.decode(q.cuda(), w.p, trace_cap=cap)
+        torch.cuda.synchronize()
+        assert sh.status() == zha.ZHA_OK
+        k0, k1, q0, q1 = sh.kv0, sh.kv1, sh.q0, sh.q1
+        covered += list(range(k0, k1))
+        check_decode(res, c.trees[k0:k1], c.K[k0:k1], c.V[k0:k1], c.inp.ref[k0:k1], q[q0:q1].double().numpy(), w.p,
+                     c.n, w.c, w.D, w.group, w.kv_dtype, case=f"{name} KV-head shard {rank} of {world}")
+        assert torch.equal(res["n_leaf"], whole["n_leaf"][q0:q1])
+        for h in range(q1 - q0):
+            n = int(res["n_leaf"][h])
+            assert torch.equal(res["leaf_idx"][h, :n], whole["leaf_idx"][q0 + h, :n])
+        assert torch.max(torch.abs(res["out"] - whole["out"][q0:q1])).item() <= OUT_TOL[w.kv_dtype]
+        sh.close()
+    assert covered == list(range(w.h_kv))
