@@ -464,7 +464,7 @@ __device__ __noinline__ void score_chunks(const Decode &a, const Level &L, int64
         const float *cbr = cbs + st * SW_ROWS_MAX;  // plane offsets of the stage's rows
         const RT *cb = reinterpret_cast<const RT *>(bufs + (size_t)st * SW_BYTES);
         float est = -INFINITY;
-#pragma unroll 1
+#pragma unroll 2
         for (int r0 = 0; r0 < C::ROWS; r0 += 8) {
             // rows r0 .. r0 + 7: slot r / R, plane r % R
             float v[8 * G];
