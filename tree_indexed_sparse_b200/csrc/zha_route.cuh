@@ -632,38 +632,50 @@ __device__ __forceinline__ void keep_or(uint8_t *keep, int64_t i, uint32_t bit) 
 // and sums the masses before it.  w: shared [SOLO_MAX][G] masses.
 template <int G>
 __device__ __noinline__ void solo_cut(const Level &L, HeadCut *cut, unsigned long long *w, float p) {
-    const int tid = threadIdx.x;
+    static_assert(RANK_MAX * G <= GT, "one thread per (slot, head)");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n = (int)L.n;
-#pragma unroll 1
-    for (int idx = tid; idx < n * G; idx += GT) {
-        const float e = L.sc[idx];
-        w[idx] = (e == -INFINITY) ? 0ull : mass_fx(expf(e - cut[idx % G].M));
+    // thread idx = slot * G + head: its mass, then the head's total over the
+    // warps (lanes with equal idx % G; integer sums, any order)
+    unsigned long long *wz = w + RANK_MAX * G;  // [GT / 32][G] per-warp totals
+    const int h = tid % G;
+    float ei = -INFINITY;
+    unsigned long long wi = 0ull;
+    if (tid < n * G) {
+        ei = L.sc[tid];
+        if (ei != -INFINITY) wi = mass_fx(expf(ei - cut[h].M));
+        w[tid] = wi;
     }
+    unsigned long long z = wi;
+#pragma unroll
+    for (int off = G; off < 32; off <<= 1) z += __shfl_xor_sync(FULL, z, off);
+    if (lane < G) wz[warp * G + lane] = z;
     gsync();
     if (tid < G) {
         unsigned long long Z = 0ull;
-#pragma unroll 1
-        for (int i = 0; i < n; ++i) Z += w[i * G + tid];
+#pragma unroll
+        for (int v = 0; v < GT / 32; ++v) Z += wz[v * G + tid];
         cut[tid].Z = Z;
         cut[tid].target = target_of(Z, p);
     }
     gsync();
-    if (tid < n) {
-        uint32_t kb = 0u;
-#pragma unroll 1
-        for (int h = 0; h < G; ++h) {
-            const float ei = L.sc[tid * G + h];
-            if (ei == -INFINITY) continue;
-            unsigned long long pre = 0ull;
+    // rank (slot, head) against the head's other slots: (estimate descending, slot ascending)
+    bool kept = false;
+    if (tid < n * G && ei != -INFINITY) {
+        const int i = tid / G;
+        unsigned long long pre = 0ull;
 #pragma unroll 4
-            for (int j = 0; j < n; ++j) {
-                const float ej = L.sc[j * G + h];
-                if (ej > ei || (ej == ei && j < tid)) pre += w[j * G + h];
-            }
-            if (pre < cut[h].target) kb |= 1u << h;
+        for (int j = 0; j < n; ++j) {
+            const float ej = L.sc[j * G + h];
+            if (ej > ei || (ej == ei && j < i)) pre += w[j * G + h];
         }
-        L.keep[tid] = (uint8_t)kb;
+        kept = pre < cut[h].target;
     }
+    // the slot's keep bits: lanes i * G .. i * G + G - 1 of one warp (G divides 32)
+    uint32_t kb = kept ? 1u << h : 0u;
+#pragma unroll
+    for (int off = 1; off < G; off <<= 1) kb |= __shfl_xor_sync(FULL, kb, off);
+    if (tid < n * G && h == 0) L.keep[tid / G] = (uint8_t)kb;
     gsync();
 }
 
