@@ -24,7 +24,9 @@ over the same K steps from a rebuilt cache, with a third event between the
 two launches; the roofline entry uses that pass's decode durations.
 
 --impl reference times the fp64 CPU oracle on the same workload instead.
-Multi-GPU: replicas only (each rank runs the whole workload on its GPU).
+Multi-GPU: --gpus N runs N replicas (each rank the whole workload on its
+GPU); --kv-shards N times the workload split by KV head over N GPUs, each
+shard alone on this GPU (shards exchange nothing while decoding).
 """
 from __future__ import annotations
 
