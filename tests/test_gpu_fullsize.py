@@ -146,3 +146,38 @@ def test_fullsize_extreme_10m():
                            heads=_heads(kh, G), case=f"extreme_10m after appends kv head {kh}")
         print(f"extreme_10m: after {w.appends_after} appends, KV head {kh}, ambiguous nodes {amb}")
         del tree, K_h, V_h
+
+
+def test_batch_with_spilled_leaf_slices():
+    """13 queries of the 1M light workload's settings, at 3M tokens, in one
+    zha_decode_batch: 52 virtual KV heads, so teams of two CTAs, whose leaf
+    level slices (12K-60K slots each by the oracle's routing of these
+    queries, beyond the 7,808 that come back on chip) stay in global memory
+    and run the chunked histogram and classification passes.  Every query's routing and
+    output are replayed against the oracle for all 16 query heads."""
+    from parity import oracle_trees
+
+    n_q = 13
+    w = W["light_1m"].scaled(3_000_000, steps=n_q)
+    inp = workloads.generate(w, "cuda")
+    dt = zha.ZHA_BF16 if w.kv_dtype == "bf16" else zha.ZHA_F32
+    cache = zha.ZhaCache(w.h_kv, w.h_q, w.d, w.R, w.c, w.D, dt, w.capacity, max_batch=n_q)
+    cache.build(inp.K, inp.V, w.n_tokens, inp.ref)
+    cap = oracle.level_nodes(w.capacity, w.c, 1)
+    qs = inp.Q[:n_q].contiguous()
+    res = cache.decode_batch(qs, w.p, trace_cap=cap)
+    torch.cuda.synchronize()
+    assert cache.status() == zha.ZHA_OK
+    res = {k: v.cpu() for k, v in res.items()}
+    K_cpu, V_cpu, ref_cpu = inp.K.cpu(), inp.V.cpu(), inp.ref.cpu()
+    del inp, cache
+    torch.cuda.empty_cache()
+    trees = oracle_trees(K_cpu, ref_cpu, w.n_tokens, w.c, w.D, capacity=w.capacity)
+    h_q = w.h_q
+    qs = qs.cpu()
+    for t in range(n_q):
+        res_t = {"out": res["out"][t], "leaf_idx": res["leaf_idx"][t], "n_leaf": res["n_leaf"][t],
+                 "visited": res["visited"][t], "trace_ids": res["trace_ids"][:, t * h_q:(t + 1) * h_q],
+                 "trace_counts": res["trace_counts"][:, t * h_q:(t + 1) * h_q]}
+        check_decode(res_t, trees, K_cpu, V_cpu, ref_cpu, qs[t].double().numpy(), w.p, w.n_tokens, w.c, w.D,
+                     w.group, w.kv_dtype, case=f"light settings at 3M, batch of {n_q}, query {t}")
