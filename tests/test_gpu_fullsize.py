@@ -8,7 +8,9 @@ Each workload runs its own schedule:
     replayed, and after the 256 appends every node they touched is checked;
   * extreme_10m: 64 decodes, then 1,024 appends, then one more decode; the
     first and last of the 64 and the decode after the appends are replayed
-    for all 16 query heads, and every node the appends touched is checked.
+    for all 16 query heads, and every node the appends touched is checked;
+  * light_1m's settings at 3M tokens, 13 queries in one batched decode (the
+    leaf level's slices too large to come back on chip), all replayed.
 The oracle side runs one KV head at a time (its tree, keys and values), so
 the 10M case needs about 10 GB of host memory at once.  Build parity is
 checked on sampled nodes of every level (always including the last, partial
